@@ -1,0 +1,142 @@
+"""Exact scaled-dot-product attention on B200 (sm_100a): Python binding of libattn.so.
+
+PyTorch is used here only for device memory and streams; every step of the
+computation runs in the library's CUDA kernels, reached through the C ABI of
+include/attn.h (see ``_abi``).  There is no CPU or PyTorch fallback: on a
+machine without the built library or without a CUDA device these functions
+raise.
+
+    o, lse = fwd(q, k, v, causal=True)            # q [B,S_q,H_q,D], k/v [B,S_k,H_kv,D] bf16
+    dq, dk, dv = bwd(q, k, v, o, lse, do, causal=True)
+
+Inputs may also be CPU tensors: they are copied to the current device, the
+kernels run there, and the results are copied back to the host (the
+end-to-end path that the benchmark's ``e2e`` figure times).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+import torch
+
+from . import _abi
+from ._abi import FwdOptions, load, status_string  # noqa: F401
+
+__all__ = ["fwd", "bwd", "device_status", "set_wait_limit_ns", "exp2_poly_eval", "bwd_workspace_size",
+           "load", "status_string"]
+
+
+def _stream_ptr(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _check_tensor(name, t, shape, dtype=torch.bfloat16):
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (BSHD, D innermost)")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _shapes(q, k):
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, S, H, D]")
+    B, S_q, H_q, D = q.shape
+    S_k, H_kv = k.shape[1], k.shape[2]
+    return B, S_q, H_q, S_k, H_kv, D
+
+
+def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
+        rescale_threshold: float = 8.0, poly_exp_every: int = 8, rescale_count=None, stream=None):
+    """Forward attention.  Returns (o bf16 [B,S_q,H_q,D], lse fp32 [B,H_q,S_q]).
+
+    CPU inputs are copied to the current CUDA device and the outputs are
+    returned on the CPU.  ``rescale_count``: optional int64 CUDA tensor of one
+    element that accumulates the number of O rescales (diagnostic).
+    """
+    on_host = not q.is_cuda
+    if on_host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        q, k, v = (t.to(dev, non_blocking=True) for t in (q, k, v))
+    B, S_q, H_q, S_k, H_kv, D = _shapes(q, k)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    _check_tensor("q", q, (B, S_q, H_q, D))
+    _check_tensor("k", k, (B, S_k, H_kv, D))
+    _check_tensor("v", v, (B, S_k, H_kv, D))
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H_q, S_q), dtype=torch.float32, device=q.device)
+    _check_tensor("out", out, (B, S_q, H_q, D))
+    _check_tensor("lse", lse, (B, H_q, S_q), torch.float32)
+    opt = FwdOptions(float(rescale_threshold), int(poly_exp_every),
+                     rescale_count.data_ptr() if rescale_count is not None else None)
+    code = load().attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                              B, H_q, H_kv, S_q, S_k, D, int(bool(causal)), scale, ctypes.byref(opt),
+                              _stream_ptr(stream))
+    _abi.check(code, "attn_fwd")
+    if on_host:
+        return out.cpu(), lse.cpu()
+    return out, lse
+
+
+def bwd_workspace_size(B, H_q, S_q, D) -> int:
+    return int(load().attn_bwd_workspace_size(B, H_q, S_q, D))
+
+
+def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, dq=None, dk=None, dv=None,
+        workspace=None, stream=None):
+    """Backward attention.  Returns (dq, dk, dv) bf16 with the shapes of q, k, v."""
+    on_host = not q.is_cuda
+    if on_host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        q, k, v, o, lse, do = (t.to(dev, non_blocking=True) for t in (q, k, v, o, lse, do))
+    B, S_q, H_q, S_k, H_kv, D = _shapes(q, k)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    _check_tensor("q", q, (B, S_q, H_q, D))
+    _check_tensor("k", k, (B, S_k, H_kv, D))
+    _check_tensor("v", v, (B, S_k, H_kv, D))
+    _check_tensor("o", o, (B, S_q, H_q, D))
+    _check_tensor("lse", lse, (B, H_q, S_q), torch.float32)
+    _check_tensor("do", do, (B, S_q, H_q, D))
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for n, t, shp in (("dq", dq, q.shape), ("dk", dk, k.shape), ("dv", dv, v.shape)):
+        _check_tensor(n, t, shp)
+    need = bwd_workspace_size(B, H_q, S_q, D)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace.numel() * workspace.element_size() < need or not workspace.is_cuda:
+        raise ValueError(f"workspace must be a CUDA buffer of at least {need} bytes")
+    code = load().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                           B, H_q, H_kv, S_q, S_k, D, int(bool(causal)), scale, _stream_ptr(stream))
+    _abi.check(code, "attn_bwd")
+    if on_host:
+        return dq.cpu(), dk.cpu(), dv.cpu()
+    return dq, dk, dv
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream; return (and clear) the kernels' device status code."""
+    return int(load().attn_device_status(_stream_ptr(stream)))
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    load().attn_set_wait_limit_ns(int(ns))
+
+
+def exp2_poly_eval(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """The kernels' FMA-pipe cubic 2^x evaluated on a CUDA fp32 tensor (diagnostic)."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA float32 tensor")
+    y = torch.empty_like(x)
+    _abi.check(load().attn_exp2_poly_eval(x.data_ptr(), y.data_ptr(), x.numel(), _stream_ptr(stream)),
+               "attn_exp2_poly_eval")
+    return y

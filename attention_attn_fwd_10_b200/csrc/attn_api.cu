@@ -1,0 +1,239 @@
+// C-ABI entry points of libattn.so (declared in include/attn.h): argument
+// validation, TMA descriptor encoding, kernel selection and launch.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "fwd_kernel.cuh"
+#include "sm100_common.cuh"
+
+namespace attn {
+
+// Device status word: kernels record kDevWaitTimeout here when they abandon a wait.
+__device__ int g_status = 0;
+
+namespace {
+
+constexpr unsigned long long kDefaultWaitLimitNs = 4000000000ull;
+std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 BSHD tensor viewed as (D, H, S, B); boxes of 64 x 1 x 128 x 1, 128-byte swizzle.
+bool make_bshd_map(CUtensorMap* map, const void* ptr, int B, int S, int H, int D) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
+                                 static_cast<cuuint64_t>(S) * H * D * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estride[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estride,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int* status_ptr() {
+  static int* ptr = nullptr;
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  int dev = -1;
+  static int ptr_dev = -2;
+  cudaGetDevice(&dev);
+  if (ptr == nullptr || ptr_dev != dev) {
+    void* sym = nullptr;
+    if (cudaGetSymbolAddress(&sym, g_status) != cudaSuccess) return nullptr;
+    ptr = static_cast<int*>(sym);
+    ptr_dev = dev;
+  }
+  return ptr;
+}
+
+attn_status_t check_common(int B, int H_q, int H_kv, int S_q, int S_k, int D, int causal, float scale) {
+  if (B < 1 || H_q < 1 || H_kv < 1 || S_q < 1 || S_k < 1) return ATTN_ERR_INVALID_ARG;
+  if (H_q % H_kv != 0) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  // index arithmetic inside the kernels is 32-bit per head row; keep products in range
+  const double rows = static_cast<double>(B) * (S_q > S_k ? S_q : S_k);
+  if (rows * (H_q > H_kv ? H_q : H_kv) * D >= 9.0e18 || static_cast<double>(B) * H_q * ((S_q + 127) / 128) >= 2.0e9)
+    return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+template <int D, bool CAUSAL, int POLY>
+cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
+                       unsigned grid, cudaStream_t st) {
+  using L = FwdLayout<D>;
+  auto kern = attn_fwd_kernel<D, CAUSAL, POLY>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  kern<<<grid, L::THREADS, L::SMEM_BYTES, st>>>(mq, mk, mv, p);
+  return cudaGetLastError();
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch_fwd_poly(int poly, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                            const FwdParams& p, unsigned grid, cudaStream_t st) {
+  switch (poly) {
+    case 0: return launch_fwd<D, CAUSAL, 0>(mq, mk, mv, p, grid, st);
+    case 4: return launch_fwd<D, CAUSAL, 4>(mq, mk, mv, p, grid, st);
+    default: return launch_fwd<D, CAUSAL, 8>(mq, mk, mv, p, grid, st);
+  }
+}
+
+__global__ void exp2_poly_eval_kernel(const float* x, float* y, long long n) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x)
+    y[i] = exp2_poly(x[i]);
+}
+
+}  // namespace
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" {
+
+int attn_abi_version(void) { return 1; }
+
+const char* attn_status_string(attn_status_t s) {
+  switch (s) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG: invalid size, scale, causal flag or null pointer";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED: request not served by this build (D must be 64 or 128)";
+    case ATTN_ERR_MISALIGNED: return "ATTN_ERR_MISALIGNED: tensor pointers must be 16-byte aligned";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA: a CUDA call failed";
+    case ATTN_ERR_DEVICE_TIMEOUT: return "ATTN_ERR_DEVICE_TIMEOUT: a kernel abandoned a bounded wait";
+  }
+  return "ATTN_ERR_UNKNOWN";
+}
+
+void attn_fwd_default_options(attn_fwd_options_t* opt) {
+  if (!opt) return;
+  opt->rescale_threshold = 8.0f;
+  opt->poly_exp_every = 8;
+  opt->rescale_count = nullptr;
+}
+
+attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H_q,
+                          int H_kv, int S_q, int S_k, int D, int causal, float scale,
+                          const attn_fwd_options_t* opt_in, void* stream) {
+  attn_fwd_options_t opt;
+  attn_fwd_default_options(&opt);
+  if (opt_in) opt = *opt_in;
+  attn_status_t st = check_common(B, H_q, H_kv, S_q, S_k, D, causal, scale);
+  if (st != ATTN_OK) return st;
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!(opt.rescale_threshold >= 0.f && opt.rescale_threshold <= 16.f)) return ATTN_ERR_INVALID_ARG;
+  if (opt.poly_exp_every != 0 && opt.poly_exp_every != 4 && opt.poly_exp_every != 8) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_MISALIGNED;
+
+  CUtensorMap mq, mk, mv;
+  if (!make_bshd_map(&mq, q, B, S_q, H_q, D) || !make_bshd_map(&mk, k, B, S_k, H_kv, D) ||
+      !make_bshd_map(&mv, v, B, S_k, H_kv, D))
+    return ATTN_ERR_CUDA;
+  int* status = status_ptr();
+  if (!status) return ATTN_ERR_CUDA;
+
+  FwdParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.H_q = H_q;
+  p.H_kv = H_kv;
+  p.S_q = S_q;
+  p.S_k = S_k;
+  p.n_q_tiles = (S_q + 127) / 128;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.tau = opt.rescale_threshold;
+  p.status = status;
+  p.rescale_count = opt.rescale_count;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  const unsigned grid = static_cast<unsigned>(p.n_q_tiles) * B * H_q;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t err;
+  if (D == 128)
+    err = causal ? launch_fwd_poly<128, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s)
+                 : launch_fwd_poly<128, false>(opt.poly_exp_every, mq, mk, mv, p, grid, s);
+  else
+    err = causal ? launch_fwd_poly<64, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s)
+                 : launch_fwd_poly<64, false>(opt.poly_exp_every, mq, mk, mv, p, grid, s);
+  return err == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H_q, int H_kv,
+                       int S_q, int S_k, int D, int causal, float scale, void* stream) {
+  return attn_fwd_ex(q, k, v, o, lse, B, H_q, H_kv, S_q, S_k, D, causal, scale, nullptr, stream);
+}
+
+size_t attn_bwd_workspace_size(int B, int H_q, int S_q, int D) {
+  if (B < 1 || H_q < 1 || S_q < 1 || (D != 64 && D != 128)) return 0;
+  const size_t dq_acc = static_cast<size_t>(B) * S_q * H_q * D * sizeof(float);
+  const size_t delta = static_cast<size_t>(B) * H_q * S_q * sizeof(float);
+  return ((dq_acc + 255) / 256) * 256 + ((delta + 255) / 256) * 256;
+}
+
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                       void* dq, void* dk, void* dv, void* workspace, int B, int H_q, int H_kv, int S_q, int S_k,
+                       int D, int causal, float scale, void* stream) {
+  attn_status_t st = check_common(B, H_q, H_kv, S_q, S_k, D, causal, scale);
+  if (st != ATTN_OK) return st;
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
+  (void)stream;
+  return ATTN_ERR_UNSUPPORTED;
+}
+
+attn_status_t attn_device_status(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
+  int* status = status_ptr();
+  if (!status) return ATTN_ERR_CUDA;
+  int host = 0;
+  if (cudaMemcpy(&host, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
+  const int zero = 0;
+  if (host != 0 && cudaMemcpy(status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return host == 0 ? ATTN_OK : static_cast<attn_status_t>(host);
+}
+
+void attn_set_wait_limit_ns(unsigned long long ns) { g_wait_limit_ns.store(ns ? ns : kDefaultWaitLimitNs); }
+
+attn_status_t attn_exp2_poly_eval(const float* x, float* y, long long n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return ATTN_ERR_INVALID_ARG;
+  if (n == 0) return ATTN_OK;
+  const long long blocks_ll = (n + 255) / 256;
+  const unsigned blocks = static_cast<unsigned>(blocks_ll < 148 * 16 ? blocks_ll : 148 * 16);
+  exp2_poly_eval_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,368 @@
+// Forward attention kernel for sm_100a:  O = softmax(scale * Q K^T [+ causal]) V, lse.
+//
+// One CTA owns one 128-row Q tile of one (batch, query head) and streams the
+// key/value blocks that tile can see.  Warp roles:
+//   warps 0-3  softmax warpgroup: thread t owns query row t of the tile (TMEM lane t)
+//   warp  4    TMA producer: Q once, then K_j / V_j into a 2-stage ring
+//   warp  5    TMEM allocator and single-thread tcgen05.mma issuer
+// Tensor-memory map (32-bit columns): S_0, S_1 (two 128x128 fp32 score
+// buffers), O (128 x D fp32), P_0, P_1 (128x128 bf16 probabilities, two per
+// column).  Issue order on the tensor pipe: S_0, S_1, PV_0, S_2, PV_1, ... so
+// the softmax of block j overlaps the S MMA of block j+1 and the PV MMA of
+// block j-1 (the fully asynchronous MMA pipeline of FlashAttention-4: "AI
+// Infra series ch. 6, GPU performance engineering (II)", section 7, and
+// "NVIDIA's strongest B200 wastes 60%", second move).
+//
+// Softmax (per row, base-2 units t = s * scale * log2 e):
+//   m_new = max(m_used, rowmax(t)); the running max actually used for the
+//   exponentials, m_used, moves only when m_new - m_used > tau (conditional
+//   rescaling, same article section 7 item 2); then O and l are rescaled by
+//   2^(m_used_old - m_new).  Between rescales p = 2^(t - m_used) <= 2^tau.
+//   The final O / l and lse = (m_used + log2 l) * ln 2 are exact whatever tau is.
+//   A fixed subset of columns uses the FMA-pipe cubic 2^x, the rest MUFU ex2
+//   (same article section 7 item 1; the hybrid of "NVIDIA's strongest B200
+//   wastes 60%", first move).
+#pragma once
+
+#include "sm100_common.cuh"
+
+namespace attn {
+
+struct FwdParams {
+  __nv_bfloat16* o;  // [B, S_q, H_q, D]
+  float* lse;        // [B, H_q, S_q]
+  int B, H_q, H_kv, S_q, S_k;
+  int n_q_tiles;     // ceil(S_q / 128)
+  float scale_log2;  // scale * log2(e)
+  float tau;         // rescale threshold (base-2 units); 0 = rescale on every increase
+  int* status;       // device status word
+  unsigned long long* rescale_count;  // optional: number of (row, block) rescales of O
+  uint64_t wait_limit_ns;
+};
+
+template <int D>
+struct FwdLayout {
+  static constexpr int BM = 128;                 // query rows per tile
+  static constexpr int BN = 128;                 // keys per block
+  static constexpr int STAGES = 2;               // K/V ring depth
+  static constexpr int NBOX = D / 64;            // 64-element (128 B) TMA boxes per row block
+  static constexpr int BOX_BYTES = 128 * 128;    // one 128 x 64 bf16 box
+  static constexpr int TILE_BYTES = 128 * D * 2; // one 128 x D bf16 tile
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = Q_OFF + TILE_BYTES;
+  static constexpr int V_OFF = K_OFF + STAGES * TILE_BYTES;
+  static constexpr int BAR_OFF = V_OFF + STAGES * TILE_BYTES;
+  // barrier slots (8 bytes each)
+  static constexpr int B_Q_FULL = 0;
+  static constexpr int B_K_FULL = 1;                  // + stage
+  static constexpr int B_V_FULL = B_K_FULL + STAGES;  // + stage
+  static constexpr int B_KV_EMPTY = B_V_FULL + STAGES;
+  static constexpr int B_S_FULL = B_KV_EMPTY + STAGES;  // + buffer
+  static constexpr int B_S_FREE = B_S_FULL + 2;
+  static constexpr int B_P_FULL = B_S_FREE + 2;
+  static constexpr int B_PV_DONE = B_P_FULL + 2;
+  static constexpr int B_O_FINAL = B_PV_DONE + 1;
+  static constexpr int B_DRAIN = B_O_FINAL + 1;
+  static constexpr int N_BARS = B_DRAIN + 1;
+  static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * N_BARS;
+  static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 4;
+  static constexpr int SMEM_USED = ABORT_OFF + 4;
+  // 1 KiB of slack to align the base to 1024 bytes (128-byte swizzle atoms);
+  // at least 120 KiB so a single CTA occupies an SM (its TMEM request is 512 columns).
+  static constexpr int SMEM_BYTES = (SMEM_USED + 1024) > 122880 ? (SMEM_USED + 1024) : 122880;
+  // tensor memory columns
+  static constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL = 256;
+  static constexpr uint32_t P_COL0 = 256 + D, P_COL1 = 256 + D + 64;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int THREADS = 192;
+};
+
+// p = 2^(s * c - m) for one 128-column score row, packed to bf16 pairs; returns
+// the fp32 sum of the unrounded p.  Column pair cp (columns 2cp, 2cp+1) takes
+// the FMA-pipe cubic when cp % POLY_EVERY == POLY_EVERY - 1, MUFU ex2 otherwise.
+template <int POLY_EVERY>
+__device__ __forceinline__ float exp_block(const float* s, float c, float m, uint32_t* pk) {
+  float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+  for (int cp = 0; cp < 64; ++cp) {
+    const float x0 = fmaf(s[2 * cp], c, -m);
+    const float x1 = fmaf(s[2 * cp + 1], c, -m);
+    float e0, e1;
+    if (POLY_EVERY > 0 && (cp % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1) {
+      e0 = exp2_poly(x0);
+      e1 = exp2_poly(x1);
+    } else {
+      e0 = exp2_mufu(x0);
+      e1 = exp2_mufu(x1);
+    }
+    sum0 += e0;
+    sum1 += e1;
+    pk[cp] = pack_bf16x2(e0, e1);
+  }
+  return sum0 + sum1;
+}
+
+// POLY_EVERY: a column pair cp (columns 2cp, 2cp+1) of each score block takes
+// the FMA-pipe cubic when cp % POLY_EVERY == POLY_EVERY - 1 (0 = never).
+template <int D, bool CAUSAL, int POLY_EVERY>
+__global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using L = FwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* const sptr = smem_raw + (sbase - raw);
+  auto bar = [&](int slot) -> uint32_t { return sbase + L::BAR_OFF + 8u * slot; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + L::ABORT_OFF);
+  const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work decode: longest tiles first for causal (blocks are dispatched in index order)
+  const int BH = p.B * p.H_q;
+  int qt = blockIdx.x / BH;
+  const int bh = blockIdx.x - qt * BH;
+  if (CAUSAL) qt = p.n_q_tiles - 1 - qt;
+  const int b = bh / p.H_q;
+  const int h = bh - b * p.H_q;
+  const int hkv = h / (p.H_q / p.H_kv);
+  const int q0 = qt * L::BM;
+  const int diag = p.S_k - p.S_q;  // bottom-right causal offset: key j visible to row i iff j <= i + diag
+  const int n_kv_total = (p.S_k + L::BN - 1) / L::BN;
+  int n_blocks = n_kv_total;
+  if (CAUSAL) {
+    const int last_row = min(q0 + L::BM, p.S_q) - 1;
+    const int last_key = last_row + diag;
+    n_blocks = last_key < 0 ? 0 : min(n_kv_total, last_key / L::BN + 1);
+  }
+
+  // ---- setup
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::N_BARS; ++i) {
+      uint32_t count = 1;
+      if (i == L::B_S_FREE || i == L::B_S_FREE + 1 || i == L::B_P_FULL || i == L::B_P_FULL + 1) count = 128;
+      mbar_init(bar(i), count);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(sbase + L::TMEM_SLOT_OFF, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 4 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sptr + L::TMEM_SLOT_OFF);
+
+  if (warp == 4) {
+    // ===================== TMA producer =====================
+    if (lane == 0 && n_blocks > 0) {
+      mbar_arrive_expect_tx(bar(L::B_Q_FULL), L::TILE_BYTES);
+#pragma unroll
+      for (int x = 0; x < L::NBOX; ++x)
+        tma_load_4d(sbase + L::Q_OFF + x * L::BOX_BYTES, &tm_q, bar(L::B_Q_FULL), x * 64, h, q0, b);
+      int issued = 0;
+      for (int j = 0; j < n_blocks; ++j) {
+        const int s = j % L::STAGES;
+        if (j >= L::STAGES && !mbar_wait(bar(L::B_KV_EMPTY + s), ((j / L::STAGES) - 1) & 1, ctl)) break;
+        mbar_arrive_expect_tx(bar(L::B_K_FULL + s), L::TILE_BYTES);
+#pragma unroll
+        for (int x = 0; x < L::NBOX; ++x)
+          tma_load_4d(sbase + L::K_OFF + s * L::TILE_BYTES + x * L::BOX_BYTES, &tm_k, bar(L::B_K_FULL + s),
+                      x * 64, hkv, j * L::BN, b);
+        mbar_arrive_expect_tx(bar(L::B_V_FULL + s), L::TILE_BYTES);
+#pragma unroll
+        for (int x = 0; x < L::NBOX; ++x)
+          tma_load_4d(sbase + L::V_OFF + s * L::TILE_BYTES + x * L::BOX_BYTES, &tm_v, bar(L::B_V_FULL + s),
+                      x * 64, hkv, j * L::BN, b);
+        issued = j + 1;
+      }
+      // Drain: every load this thread issued has landed before the CTA may exit.
+      mbar_wait_drain(bar(L::B_Q_FULL), 0, 1000000000ull);
+      for (int s = 0; s < L::STAGES && s < issued; ++s) {
+        const int uses = (issued - 1 - s) / L::STAGES + 1;
+        mbar_wait_drain(bar(L::B_K_FULL + s), (uses - 1) & 1, 1000000000ull);
+        mbar_wait_drain(bar(L::B_V_FULL + s), (uses - 1) & 1, 1000000000ull);
+      }
+    }
+  } else if (warp == 5) {
+    // ===================== MMA issuer =====================
+    if (lane == 0 && n_blocks > 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
+      bool ok = mbar_wait(bar(L::B_Q_FULL), 0, ctl);
+      for (int j = 0; ok && j <= n_blocks; ++j) {
+        if (j < n_blocks) {
+          const int s = j % L::STAGES;
+          const int buf = j & 1;
+          if (!mbar_wait(bar(L::B_K_FULL + s), (j / L::STAGES) & 1, ctl)) break;
+          if (j >= 2 && !mbar_wait(bar(L::B_S_FREE + buf), ((j - 2) >> 1) & 1, ctl)) break;
+          tc_fence_after();
+          const uint32_t d_tmem = tmem + (buf ? L::S_COL1 : L::S_COL0);
+          const uint32_t q_base = sbase + L::Q_OFF;
+          const uint32_t k_base = sbase + L::K_OFF + s * L::TILE_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32;
+            umma_ss(d_tmem, sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(k_base + off, 16, 1024), IDESC_S,
+                    kk > 0 ? 1u : 0u);
+          }
+          umma_commit(bar(L::B_S_FULL + buf));
+        }
+        if (j >= 1) {
+          const int jj = j - 1;
+          const int s = jj % L::STAGES;
+          const int buf = jj & 1;
+          if (!mbar_wait(bar(L::B_P_FULL + buf), (jj >> 1) & 1, ctl)) break;
+          if (!mbar_wait(bar(L::B_V_FULL + s), (jj / L::STAGES) & 1, ctl)) break;
+          tc_fence_after();
+          const uint32_t v_base = sbase + L::V_OFF + s * L::TILE_BYTES;
+          const uint32_t p_tmem = tmem + (buf ? L::P_COL1 : L::P_COL0);
+#pragma unroll
+          for (int kk = 0; kk < L::BN / 16; ++kk) {
+            // 16 keys = 16 rows of 128 B = 2048 bytes; column blocks of 64 d-values are BOX_BYTES apart.
+            umma_ts(tmem + L::O_COL, p_tmem + kk * 8, sdesc_sw128(v_base + kk * 2048, L::BOX_BYTES, 1024),
+                    IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(bar(L::B_KV_EMPTY + s));
+          umma_commit(bar(L::B_PV_DONE));
+          if (jj == n_blocks - 1) umma_commit(bar(L::B_O_FINAL));
+        }
+      }
+      // Drain: no MMA may still be writing TMEM when it is released.
+      umma_commit(bar(L::B_DRAIN));
+      mbar_wait_drain(bar(L::B_DRAIN), 0, 1000000000ull);
+    }
+  } else {
+    // ===================== softmax warpgroup (warps 0-3) =====================
+    const int row = threadIdx.x;  // 0..127 == TMEM lane
+    const int qi = q0 + row;
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const float c = p.scale_log2;
+    const int lim = min(qi + (CAUSAL ? diag : p.S_k), p.S_k - 1);  // last visible key of this row
+    float m_used = -INFINITY;
+    float l = 0.f;
+    unsigned rescales = 0;
+    bool ok = true;
+    for (int j = 0; j < n_blocks; ++j) {
+      const int buf = j & 1;
+      ok = mbar_wait(bar(L::B_S_FULL + buf), (j >> 1) & 1, ctl);
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sr[128];
+      const uint32_t s_addr = tmem + lane_addr + (buf ? L::S_COL1 : L::S_COL0);
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) tmem_ld32(s_addr + ch * 32, sr + ch * 32);
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) tmem_ld_wait(sr + ch * 32);
+      tc_fence_before();
+      mbar_arrive(bar(L::B_S_FREE + buf));
+
+      float* s = reinterpret_cast<float*>(sr);
+      const int kbase = j * L::BN;
+      const bool need_mask = (kbase + L::BN - 1 > (CAUSAL ? q0 + diag : p.S_k - 1)) || (kbase + L::BN > p.S_k);
+      if (need_mask) {
+        const int lim_c = lim - kbase;
+#pragma unroll
+        for (int cc = 0; cc < 128; ++cc)
+          if (cc > lim_c) s[cc] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int cc = 1; cc < 128; ++cc) mx = fmaxf(mx, s[cc]);
+      const float m_new = fmaxf(m_used, mx * c);
+      const bool resc = (m_new - m_used) > p.tau;  // false for NaN (-inf - -inf)
+      float alpha = 1.f;
+      if (resc) {
+        alpha = exp2_mufu(m_used - m_new);  // 0 when m_used = -inf
+        m_used = m_new;
+        l *= alpha;
+        if (j > 0) ++rescales;
+      }
+      const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
+      uint32_t pk[64];
+      // Masked blocks take MUFU ex2 only: it maps -inf to an exact 0.
+      const float rowsum = need_mask ? exp_block<0>(s, c, m_eff, pk) : exp_block<POLY_EVERY>(s, c, m_eff, pk);
+      l += rowsum;
+      const uint32_t p_addr = tmem + lane_addr + (buf ? L::P_COL1 : L::P_COL0);
+      tmem_st32(p_addr, pk);
+      tmem_st32(p_addr + 32, pk + 32);
+      tmem_st_wait();
+      if (j > 0 && __any_sync(0xffffffffu, resc)) {
+        // O must hold P_{j-1} V_{j-1} before it is rescaled.
+        ok = mbar_wait(bar(L::B_PV_DONE), (j - 1) & 1, ctl);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t o_addr = tmem + lane_addr + L::O_COL;
+#pragma unroll 1
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t orr[32];
+          tmem_ld32(o_addr + ch * 32, orr);
+          tmem_ld_wait(orr);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+          tmem_st32(o_addr + ch * 32, orr);
+        }
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(L::B_P_FULL + buf));
+    }
+    if (p.rescale_count != nullptr && rescales) atomicAdd(p.rescale_count, (unsigned long long)rescales);
+
+    // ---- epilogue: O / l -> bf16, lse
+    if (ok && n_blocks > 0) {
+      ok = mbar_wait(bar(L::B_O_FINAL), 0, ctl);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const bool valid = qi < p.S_q;
+      __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.S_q + qi) * p.H_q + h) * D;
+      const uint32_t o_addr = tmem + lane_addr + L::O_COL;
+#pragma unroll 1
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t orr[32];
+        if (n_blocks > 0) {
+          tmem_ld32(o_addr + ch * 32, orr);
+          tmem_ld_wait(orr);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) orr[i] = 0u;
+        }
+        uint32_t pkd[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pkd[i] = pack_bf16x2(__uint_as_float(orr[2 * i]) * inv_l, __uint_as_float(orr[2 * i + 1]) * inv_l);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2], pkd[4 * i + 3]);
+        }
+      }
+      if (valid) {
+        p.lse[(static_cast<size_t>(b) * p.H_q + h) * p.S_q + qi] =
+            l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      }
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+}  // namespace attn

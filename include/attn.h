@@ -1,0 +1,135 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) exact-attention library (libattn.so).
+ *
+ * What it computes (forward):
+ *     S   = scale * Q K^T            (per batch b and query head h; K, V of head h / (H_q / H_kv))
+ *     S_ij = -inf where causal and j > i + (S_k - S_q)   (bottom-right alignment)
+ *     P   = softmax(S) row-wise,  O = P V,  lse_i = log(sum_j exp(S_ij))   (natural log)
+ * This is the attention kernel that "AI Infra series ch. 6, GPU performance
+ * engineering (II)" analyses in its section 1 (GEMMs plus softmax
+ * exponentials, quoting the FlashAttention-4 paper) and whose Blackwell
+ * techniques its section 7 lists (asynchronous MMA pipeline, software
+ * exponential, conditional rescaling, 2-CTA MMA with TMEM intermediates).
+ * The backward returns dQ, dK, dV of L = sum(dO * O) using the forward's O
+ * and lse (P is recomputed, same article section 5, "recomputation").
+ *
+ * Tensors (all device pointers, caller-owned, never retained after a call returns):
+ *   q, o, dO, dq : bf16 [B, S_q, H_q, D]   contiguous ("BSHD", D innermost)
+ *   k, v, dk, dv : bf16 [B, S_k, H_kv, D]  contiguous
+ *   lse          : fp32 [B, H_q, S_q]
+ * Every pointer must be 16-byte aligned.  D is 64 or 128; H_q % H_kv == 0;
+ * S_q, S_k >= 1; scale finite and > 0; causal is 0 or 1.
+ *
+ * Execution: calls enqueue work on `stream` (a cudaStream_t; NULL = legacy
+ * default stream) and return without synchronising.  The return value reports
+ * argument and launch errors only.  A kernel that gives up on an internal wait
+ * (it never spins without a bound) records ATTN_ERR_DEVICE_TIMEOUT in a device
+ * status word that attn_device_status() reads.  The library allocates no
+ * device memory on any call: scratch space (the backward's workspace) is
+ * passed in by the caller.  All entry points are thread-safe.
+ */
+#ifndef ATTN_B200_ATTN_H_
+#define ATTN_B200_ATTN_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,    /* a size, scale, causal flag or pointer is invalid */
+  ATTN_ERR_UNSUPPORTED = 2,    /* a valid request this build does not serve (e.g. D not in {64,128}) */
+  ATTN_ERR_MISALIGNED = 3,     /* a tensor pointer is not 16-byte aligned */
+  ATTN_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed (no device, launch failure ...) */
+  ATTN_ERR_DEVICE_TIMEOUT = 5  /* a kernel abandoned a bounded internal wait (see attn_device_status) */
+} attn_status_t;
+
+/* Version of this ABI (bumped on any incompatible change). */
+int attn_abi_version(void);
+
+/* Human-readable name of a status code (static storage). */
+const char* attn_status_string(attn_status_t s);
+
+/*
+ * Forward pass.  Writes o [B,S_q,H_q,D] (bf16) and lse [B,H_q,S_q] (fp32).
+ * Rows that see no key (only possible when causal and S_q > S_k) get O = 0, lse = -inf.
+ */
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H_q,
+                       int H_kv, int S_q, int S_k, int D, int causal, float scale, void* stream);
+
+/*
+ * Tunables and diagnostics of the forward; none of them changes the exact
+ * result, only rounding.
+ *   rescale_threshold : tau, in base-2 units of the scores.  O is rescaled only
+ *                       when a row's running max grows by more than tau
+ *                       ("conditional softmax rescaling", AI Infra series ch. 6
+ *                       section 7 item 2).  0 = rescale on every increase.
+ *                       Must be in [0, 16].  Default 8.
+ *   poly_exp_every    : of every `poly_exp_every` column pairs of a score block,
+ *                       one pair takes the FMA-pipe cubic 2^x instead of the
+ *                       MUFU unit (same section, item 1: 10-25 % of the
+ *                       exponentials).  Allowed: 0 (MUFU only), 4 (25 %),
+ *                       8 (12.5 %).  Default 8.
+ *   rescale_count     : optional device pointer to an unsigned 64-bit counter;
+ *                       the kernel adds the number of (row, key block) O rescales
+ *                       it performed after a row's first block.  NULL = off.
+ */
+typedef struct {
+  float rescale_threshold;
+  int poly_exp_every;
+  unsigned long long* rescale_count;
+} attn_fwd_options_t;
+
+/* Fills `opt` with the defaults above. */
+void attn_fwd_default_options(attn_fwd_options_t* opt);
+
+/* attn_fwd with explicit options (`opt` NULL = defaults). */
+attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H_q,
+                          int H_kv, int S_q, int S_k, int D, int causal, float scale,
+                          const attn_fwd_options_t* opt, void* stream);
+
+/*
+ * Bytes of device workspace attn_bwd needs: an fp32 dQ accumulator
+ * [B, S_q, H_q, D] and the fp32 row terms delta_i = sum_d dO_id O_id [B, H_q, S_q].
+ * Returns 0 for invalid sizes.
+ */
+size_t attn_bwd_workspace_size(int B, int H_q, int S_q, int D);
+
+/*
+ * Backward pass.  q, k, v, o, lse as produced/consumed by attn_fwd with the
+ * same arguments; dO is the gradient of the loss w.r.t. o.  Writes dq, dk, dv
+ * (bf16).  `workspace` must hold attn_bwd_workspace_size(...) bytes, 16-byte
+ * aligned; its contents on entry are ignored.  The dQ accumulation uses atomic
+ * fp32 additions, so results may differ in the last bits from run to run.
+ */
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                       const void* dO, void* dq, void* dk, void* dv, void* workspace, int B, int H_q,
+                       int H_kv, int S_q, int S_k, int D, int causal, float scale, void* stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word:
+ * ATTN_OK, or ATTN_ERR_DEVICE_TIMEOUT if a kernel gave up on a wait since the
+ * last call, or ATTN_ERR_CUDA if the synchronisation itself failed.
+ */
+attn_status_t attn_device_status(void* stream);
+
+/*
+ * Upper bound, in nanoseconds, of any single internal wait of the kernels
+ * (default 4e9).  Tests lower it to exercise the timeout path without a hang.
+ * 0 restores the default.
+ */
+void attn_set_wait_limit_ns(unsigned long long ns);
+
+/*
+ * Diagnostic: y[i] = the kernels' FMA-pipe cubic 2^x applied to x[i]
+ * (device pointers, n >= 0), for checking its error bound.
+ */
+attn_status_t attn_exp2_poly_eval(const float* x, float* y, long long n, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_ATTN_H_ */

@@ -1,0 +1,48 @@
+"""Shared tolerances and comparison helpers for the GPU-vs-oracle parity tests.
+
+Tolerances (inputs ~ N(0, 1), bf16 in/out, fp32 accumulation):
+  O    : max |O_gpu - O_ref| <= 1.5e-2 and mean |O_gpu - O_ref| <= 2e-3
+  lse  : max |lse_gpu - lse_ref| <= 1e-3
+  grads: max |g_gpu - g_ref| <= 3e-2 * max |g_ref|, per tensor
+and every output finite (rows that see no key: O = 0, lse = -inf exactly).
+"""
+import numpy as np
+import torch
+
+O_MAX_ABS = 1.5e-2
+O_MEAN_ABS = 2e-3
+LSE_MAX_ABS = 1e-3
+GRAD_REL_MAX = 3e-2
+
+
+def to_np(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def check_o(o_gpu, o_ref, what=""):
+    o = to_np(o_gpu) if isinstance(o_gpu, torch.Tensor) else o_gpu
+    assert np.all(np.isfinite(o)), f"{what}: non-finite O"
+    err = np.abs(o - o_ref)
+    assert err.max() <= O_MAX_ABS, f"{what}: O max-abs {err.max():.3e} > {O_MAX_ABS}"
+    assert err.mean() <= O_MEAN_ABS, f"{what}: O mean-abs {err.mean():.3e} > {O_MEAN_ABS}"
+    return float(err.max()), float(err.mean())
+
+
+def check_lse(l_gpu, l_ref, what=""):
+    l = to_np(l_gpu) if isinstance(l_gpu, torch.Tensor) else l_gpu
+    inf_ref = np.isneginf(l_ref)
+    assert np.array_equal(np.isneginf(l), inf_ref), f"{what}: -inf pattern of lse differs"
+    fin = ~inf_ref
+    assert np.all(np.isfinite(l[fin])), f"{what}: non-finite lse"
+    err = np.abs(l[fin] - l_ref[fin]) if fin.any() else np.zeros(1)
+    assert err.max() <= LSE_MAX_ABS, f"{what}: lse max-abs {err.max():.3e} > {LSE_MAX_ABS}"
+    return float(err.max())
+
+
+def check_grad(g_gpu, g_ref, what=""):
+    g = to_np(g_gpu) if isinstance(g_gpu, torch.Tensor) else g_gpu
+    assert np.all(np.isfinite(g)), f"{what}: non-finite gradient"
+    scale = max(np.abs(g_ref).max(), 1e-30)
+    err = np.abs(g - g_ref).max()
+    assert err <= GRAD_REL_MAX * scale, f"{what}: max-abs {err:.3e} > {GRAD_REL_MAX} * {scale:.3e}"
+    return float(err / scale)

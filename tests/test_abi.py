@@ -1,0 +1,88 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/attn.h declares, and rejects invalid arguments
+before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from attention_attn_fwd_10_b200 import _abi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _abi.load()
+
+
+def _declared():
+    text = open(os.path.join(ROOT, "include", "attn.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared()
+    assert declared, "no declarations parsed"
+    assert sorted(_abi.EXPORTED) == declared
+    for name in declared:
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in _abi.STATUS_NAMES.items():
+        assert _abi.status_string(code).startswith(name)
+    assert lib.attn_abi_version() == 1
+
+
+def _fwd(lib, **kw):
+    a = dict(q=16, k=32, v=48, o=64, lse=80, B=1, H_q=2, H_kv=2, S_q=8, S_k=8, D=64, causal=0, scale=0.125)
+    a.update(kw)
+    return lib.attn_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H_q"], a["H_kv"], a["S_q"],
+                        a["S_k"], a["D"], a["causal"], a["scale"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=0), 1), (dict(S_q=0), 1), (dict(S_k=-3), 1), (dict(H_q=3, H_kv=2), 1),
+    (dict(causal=2), 1), (dict(scale=0.0), 1), (dict(scale=float("nan")), 1), (dict(scale=float("inf")), 1),
+    (dict(D=96), 2), (dict(D=256), 2), (dict(q=0), 1), (dict(lse=0), 1), (dict(q=17), 3), (dict(o=8), 3),
+])
+def test_fwd_rejects_bad_arguments(lib, kw, code):
+    assert _fwd(lib, **kw) == code
+
+
+def test_fwd_options_validation(lib):
+    opt = _abi.FwdOptions()
+    lib.attn_fwd_default_options(ctypes.byref(opt))
+    assert opt.rescale_threshold == 8.0 and opt.poly_exp_every == 8 and opt.rescale_count is None
+    for field, bad in (("rescale_threshold", -1.0), ("rescale_threshold", 17.0), ("poly_exp_every", 3)):
+        o = _abi.FwdOptions(opt.rescale_threshold, opt.poly_exp_every, None)
+        setattr(o, field, bad)
+        r = lib.attn_fwd_ex(16, 32, 48, 64, 80, 1, 2, 2, 8, 8, 64, 0, 0.125, ctypes.byref(o), None)
+        assert r == 1
+
+
+def test_bwd_workspace_size(lib):
+    B, H, S, D = 2, 16, 8192, 128
+    n = lib.attn_bwd_workspace_size(B, H, S, D)
+    assert n >= B * S * H * D * 4 + B * H * S * 4
+    assert n % 256 == 0
+    assert lib.attn_bwd_workspace_size(0, H, S, D) == 0
+    assert lib.attn_bwd_workspace_size(B, H, S, 96) == 0
+
+
+def test_bwd_rejects_bad_arguments(lib):
+    p = [16] * 10
+    assert lib.attn_bwd(*p, 1, 3, 2, 8, 8, 64, 0, 0.125, None) == 1
+    assert lib.attn_bwd(*p, 1, 2, 2, 8, 8, 80, 0, 0.125, None) == 2
+    p0 = list(p)
+    p0[9] = 0
+    assert lib.attn_bwd(*p0, 1, 2, 2, 8, 8, 64, 0, 0.125, None) == 1
+
+
+def test_exp2_eval_rejects_bad_arguments(lib):
+    assert lib.attn_exp2_poly_eval(None, None, -1, None) == 1
+    assert lib.attn_exp2_poly_eval(None, None, 0, None) == 0

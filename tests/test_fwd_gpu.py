@@ -1,0 +1,128 @@
+"""GPU forward vs the fp64 oracle, through the C ABI (ctypes binding), on seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import reference as ref
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _attn():
+    import attention_attn_fwd_10_b200 as attn
+
+    return attn
+
+
+def _run(w, **kw):
+    x = workloads.make_inputs(w)
+    dev = "cuda"
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    o, lse = _attn().fwd(q, k, v, causal=w.causal, scale=w.scale, **kw)
+    torch.cuda.synchronize()
+    assert _attn().device_status() == 0
+    return x, o, lse
+
+
+def test_tiny_config_full():
+    w = workloads.TINY
+    x, o, lse = _run(w)
+    o_ref, lse_ref = ref.forward(x["q"], x["k"], x["v"], w.causal, w.scale)
+    parity.check_o(o, o_ref, w.name)
+    parity.check_lse(lse, lse_ref, w.name)
+
+
+@pytest.mark.parametrize("S_q,S_k", [(1, 1), (17, 17), (127, 127), (128, 128), (129, 129), (255, 255),
+                                     (300, 300), (64, 200), (200, 64), (1, 333), (333, 1)])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("D", [64, 128])
+def test_small_shapes(S_q, S_k, causal, D):
+    w = workloads.small(B=2, H_q=2, S_q=S_q, S_k=S_k, D=D, causal=causal, seed=S_q * 1000 + S_k)
+    x, o, lse = _run(w)
+    o_ref, lse_ref = ref.forward(x["q"], x["k"], x["v"], causal, w.scale)
+    parity.check_o(o, o_ref, w.name)
+    parity.check_lse(lse, lse_ref, w.name)
+
+
+@pytest.mark.parametrize("H_q,H_kv", [(4, 1), (8, 2), (6, 3)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa(H_q, H_kv, causal):
+    w = workloads.small(B=1, H_q=H_q, H_kv=H_kv, S_q=400, S_k=400, D=128, causal=causal, seed=11)
+    x, o, lse = _run(w)
+    o_ref, lse_ref = ref.forward(x["q"], x["k"], x["v"], causal, w.scale)
+    parity.check_o(o, o_ref, w.name)
+    parity.check_lse(lse, lse_ref, w.name)
+
+
+@pytest.mark.parametrize("tau", [0.0, 8.0, 16.0])
+@pytest.mark.parametrize("poly", [0, 4, 8])
+def test_rescale_threshold_and_poly_fraction(tau, poly):
+    w = workloads.small(B=1, H_q=2, S_q=1024, S_k=1024, D=128, causal=True, seed=5, spiky_keys=True)
+    x, o, lse = _run(w, rescale_threshold=tau, poly_exp_every=poly)
+    o_ref, lse_ref = ref.forward(x["q"], x["k"], x["v"], True, w.scale)
+    parity.check_o(o, o_ref, f"{w.name} tau={tau} poly={poly}")
+    parity.check_lse(lse, lse_ref, f"{w.name} tau={tau} poly={poly}")
+
+
+def test_noncausal_config_full():
+    w = workloads.FWD_NONCAUSAL
+    x, o, lse = _run(w)
+    o_ref, lse_ref = ref.forward(x["q"], x["k"], x["v"], w.causal, w.scale)
+    parity.check_o(o, o_ref, w.name)
+    parity.check_lse(lse, lse_ref, w.name)
+
+
+def _sampled(w, o, lse, x, heads, rows):
+    o_c, lse_c = o.cpu(), lse.cpu()
+    for (b, h) in heads:
+        o_ref, lse_ref = ref.forward_rows(x["q"], x["k"], x["v"], w.causal, w.scale, b, h, rows)
+        parity.check_o(o_c[b, rows, h, :], o_ref, f"{w.name} b={b} h={h}")
+        parity.check_lse(lse_c[b, h, rows], lse_ref, f"{w.name} b={b} h={h}")
+    assert torch.isfinite(o_c.float()).all() and torch.isfinite(lse_c).all()
+
+
+def _rows(S, n=48, seed=0):
+    g = np.random.default_rng(seed)
+    fixed = [0, 1, 127, 128, 129, S // 2, S - 129, S - 128, S - 1]
+    return sorted(set(fixed) | set(g.choice(S, n, replace=False).tolist()))
+
+
+@pytest.mark.parametrize("w", [workloads.FWD_CAUSAL, workloads.FWD_CAUSAL_SPIKY], ids=lambda w: w.name)
+def test_causal_config_sampled(w):
+    cnt = torch.zeros(1, dtype=torch.int64, device="cuda")
+    x, o, lse = _run(w, rescale_count=cnt)
+    _sampled(w, o, lse, x, [(0, 0), (1, 15), (1, 7)], _rows(w.S_q))
+    if w.spiky_keys:
+        assert int(cnt.item()) > 0  # the spiky keys exercise the rescale path
+
+
+def test_gqa_long_config_sampled():
+    w = workloads.FWD_CAUSAL_GQA
+    x, o, lse = _run(w)
+    # one full GQA group (query heads 4..7 share key/value head 1) plus the last head
+    _sampled(w, o, lse, x, [(0, 4), (0, 5), (0, 6), (0, 7), (0, 31)], _rows(w.S_q, n=24))
+
+
+def test_deterministic_and_overwrites_poison():
+    w = workloads.small(B=2, H_q=4, S_q=700, S_k=700, D=128, causal=True, seed=3)
+    x = workloads.make_inputs(w)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    o1 = torch.full_like(q, float("nan"))
+    l1 = torch.full((2, 4, 700), float("nan"), device="cuda")
+    _attn().fwd(q, k, v, causal=True, out=o1, lse=l1)
+    o2, l2 = _attn().fwd(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert torch.isfinite(o1.float()).all() and torch.isfinite(l1).all()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_host_buffers_round_trip():
+    w = workloads.small(B=1, H_q=2, S_q=300, S_k=300, D=64, causal=False, seed=9)
+    x = workloads.make_inputs(w)
+    o, lse = _attn().fwd(x["q"].pin_memory(), x["k"].pin_memory(), x["v"].pin_memory(), causal=False)
+    assert not o.is_cuda
+    o_ref, lse_ref = ref.forward(x["q"], x["k"], x["v"], False, w.scale)
+    parity.check_o(o, o_ref)
+    parity.check_lse(lse, lse_ref)
