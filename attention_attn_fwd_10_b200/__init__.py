@@ -23,7 +23,7 @@ import torch
 from . import _abi
 from ._abi import FwdOptions, load, status_string  # noqa: F401
 
-__all__ = ["fwd", "bwd", "device_status", "set_wait_limit_ns", "exp2_poly_eval", "bwd_workspace_size",
+__all__ = ["fwd", "bwd", "fwd_bwd", "device_status", "set_wait_limit_ns", "exp2_poly_eval", "bwd_workspace_size",
            "load", "status_string"]
 
 
@@ -121,6 +121,28 @@ def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, d
     if on_host:
         return dq.cpu(), dk.cpu(), dv.cpu()
     return dq, dk, dv
+
+
+def fwd_bwd(q, k, v, do, causal: bool = False, scale: float | None = None, host_out: dict | None = None,
+            stream=None):
+    """One training step of attention from host buffers: copy q, k, v, dO to the
+    current device, run the forward and the backward there, and copy o, lse,
+    dq, dk, dv back into ``host_out`` (pinned CPU tensors, allocated if None).
+    Returns the dict of host results."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    qd, kd, vd, dod = (t.to(dev, non_blocking=True) for t in (q, k, v, do))
+    o, lse = fwd(qd, kd, vd, causal=causal, scale=scale, stream=stream)
+    dq, dk, dv = bwd(qd, kd, vd, o, lse, dod, causal=causal, scale=scale, stream=stream)
+    if host_out is None:
+        host_out = {}
+    res = {"o": o, "lse": lse, "dq": dq, "dk": dk, "dv": dv}
+    for name, t in res.items():
+        if name in host_out:
+            host_out[name].copy_(t, non_blocking=True)
+        else:
+            host_out[name] = t.to("cpu")
+    torch.cuda.current_stream().synchronize()
+    return host_out
 
 
 def device_status(stream=None) -> int:

@@ -1,0 +1,407 @@
+"""Benchmark: exact attention forward + backward on B200, one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+the forward (O, lse) and then the backward (dQ, dK, dV from dO and the
+forward's O and lse), causal, B=2, H=16, S=8192, D=128, bf16 (the causal
+forward workload and the backward workload share these shapes).  FLOPs
+follow the convention 4*B*H*S_q*S_k*D for the forward, 2.5x that for the
+backward, halved for causal.
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events
+on the launching stream; L2 is flushed (a 256 MiB write) before every timed
+step, outside the events.  For N > 1 (torchrun, one process per GPU) every
+rank runs the same workload independently (replicas: the path has no
+exchange step), steps are bracketed by barriers and the slowest rank's time
+is reported; value = all ranks' FLOPs / that time.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (the one other use of oracle/ here, besides the
+cpu_baseline leg).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "attention fwd/bwd TFLOPS (bf16, D=128) and % of B200 dense BF16 peak"
+SPEC_PEAK_TFLOPS = 2250.0  # dense bf16 tensor peak the pages quote for B200
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+WORKLOADS = {
+    "causal8k": (workloads.FWD_CAUSAL, workloads.BWD_CAUSAL),
+}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.flush()
+        with open(self.file.name) as f:
+            rows = [r.strip().split(", ") for r in f if r.strip()]
+        os.unlink(self.file.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, r[5:9]):
+                if val.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# --------------------------------------------------------------------------- distributed plumbing
+
+def dist_setup(n_gpus: int):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    if world != n_gpus and rank == 0:
+        print(f"warning: --gpus {n_gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(world, x: float) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- oracle (CPU) timing
+
+def oracle_sample_time(wf, wb, budget_s: float = 15.0):
+    """Time the fp64 oracle's forward+backward on whole (b, h) heads of the workload
+    until about budget_s of CPU time; returns (TFLOPS by convention, sample text, cores)."""
+    import numpy as np
+
+    from oracle import reference as ref
+
+    x = workloads.make_inputs(wb)
+    cores = len(os.sched_getaffinity(0))
+    per_head_flops = (wf.fwd_flops() + wb.bwd_flops()) / (wf.B * wf.H_q)
+    done, t0 = 0, time.perf_counter()
+    heads = [(b, h) for b in range(wf.B) for h in range(wf.H_q)]
+    for (b, h) in heads:
+        qh = x["q"][b:b + 1, :, h:h + 1]
+        kh = x["k"][b:b + 1, :, h:h + 1]
+        vh = x["v"][b:b + 1, :, h:h + 1]
+        doh = x["do"][b:b + 1, :, h:h + 1]
+        ref.forward(qh, kh, vh, wf.causal, wf.scale)
+        ref.backward(qh, kh, vh, doh, wb.causal, wb.scale)
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    del np
+    return per_head_flops * done / dt / 1e12, f"{done} of {len(heads)} (b,h) heads, fwd+bwd, full S", cores, dt
+
+
+# --------------------------------------------------------------------------- our implementation
+
+def run_ours(args):
+    import torch
+
+    import attention_attn_fwd_10_b200 as attn
+
+    world, rank, local = dist_setup(args.gpus)
+    wf, wb = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local if world > 1 else 0)
+    x = workloads.make_inputs(wb)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    o = torch.empty_like(q)
+    lse = torch.empty((wf.B, wf.H_q, wf.S_q), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(attn.bwd_workspace_size(wb.B, wb.H_q, wb.S_q, wb.D), dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    have_bwd = True
+    try:
+        attn.bwd(q, k, v, o, lse, do, causal=True, dq=dq, dk=dk, dv=dv, workspace=ws)
+    except RuntimeError:
+        have_bwd = False
+
+    def fwd():
+        attn.fwd(q, k, v, causal=wf.causal, scale=wf.scale, out=o, lse=lse)
+
+    def bwd():
+        attn.bwd(q, k, v, o, lse, do, causal=wb.causal, scale=wb.scale, dq=dq, dk=dk, dv=dv, workspace=ws)
+
+    for _ in range(args.warmup):
+        fwd()
+        if have_bwd:
+            bwd()
+    torch.cuda.synchronize()
+    if attn.device_status() != 0:
+        raise RuntimeError("device status not OK after warm-up")
+
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    f_ms, b_ms, s_ms = [], [], []
+    with ClockSampler(dev.index) as clk:
+        for _ in range(args.steps):
+            flush.fill_(1)
+            barrier(world)
+            torch.cuda.synchronize()
+            e0, e1, e2 = ev(), ev(), ev()
+            e0.record(stream)
+            fwd()
+            e1.record(stream)
+            if have_bwd:
+                bwd()
+            e2.record(stream)
+            torch.cuda.synchronize()
+            f_ms.append(e0.elapsed_time(e1))
+            b_ms.append(e1.elapsed_time(e2))
+            s_ms.append(e0.elapsed_time(e2))
+        barrier(world)
+    clocks = clk.summary()
+    if attn.device_status() != 0:
+        raise RuntimeError("device status not OK after the timed region")
+
+    step_ms = max_over_ranks(world, sum(s_ms) / len(s_ms))
+    fwd_ms = sum(f_ms) / len(f_ms)
+    bwd_ms = sum(b_ms) / len(b_ms) if have_bwd else 0.0
+    flops_step = wf.fwd_flops() + (wb.bwd_flops() if have_bwd else 0.0)
+    value = world * flops_step / (step_ms * 1e-3) / 1e12
+
+    # end to end through the public API with pinned host buffers
+    e2e = run_e2e(args, attn, x, wf, wb, have_bwd, dev, world)
+
+    peaks, peaks_src = measured_peaks()
+    fwd_tf = wf.fwd_flops() / (fwd_ms * 1e-3) / 1e12
+    bwd_tf = wb.bwd_flops() / (bwd_ms * 1e-3) / 1e12 if have_bwd else None
+    # dominant kernel: the one with the larger share of the step
+    if have_bwd and bwd_ms > fwd_ms:
+        dom, dom_flops, dom_ms = "attn_bwd (3 kernels)", wb.bwd_flops(), bwd_ms
+    else:
+        dom, dom_flops, dom_ms = "attn_fwd_kernel", wf.fwd_flops(), fwd_ms
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) rounded to bf16)",
+        "config": {
+            "workload": wf.name.replace("fwd_", "fwd+bwd_") if have_bwd else wf.name,
+            "step": "forward + backward" if have_bwd else "forward only (backward not built)",
+            "B": wf.B, "H_q": wf.H_q, "H_kv": wf.H_kv, "S": wf.S_q, "D": wf.D, "causal": wf.causal,
+            "global_batch": wf.B * world, "seq_len": wf.S_q, "parallelism": f"replicas x{world}",
+            "l2": "flushed (256 MiB write) before every timed step",
+        },
+        "fwd": {"ms": round(fwd_ms, 4), "tflops": round(fwd_tf, 1),
+                "frac_of_spec_2250": round(fwd_tf / SPEC_PEAK_TFLOPS, 4),
+                "frac_of_measured": round(fwd_tf / peak, 4)},
+        "bwd": ({"ms": round(bwd_ms, 4), "tflops": round(bwd_tf, 1),
+                 "frac_of_spec_2250": round(bwd_tf / SPEC_PEAK_TFLOPS, 4),
+                 "frac_of_measured": round(bwd_tf / peak, 4)} if have_bwd else None),
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json bf16_tflops)"
+                     if peaks_src == "measured" else "fallback 1.59 PFLOP/s burst",
+                     "traffic": None},
+        "e2e": e2e,
+        "gpu_launches": args.steps * (1 + (3 if have_bwd else 0)),
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, sample, cores, dt = oracle_sample_time(wf, wb if have_bwd else wb, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": tf, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                                "sample": sample + f" ({dt:.1f} s, fp64 numpy)"}
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, attn, x, wf, wb, have_bwd, dev, world):
+    """Same metric through the public API with pinned host buffers: the timed
+    region holds the host->device copies of q, k, v (and dO), the kernels, and
+    the device->host copies of o, lse (and dq, dk, dv)."""
+    import torch
+
+    hq, hk, hv, hdo = (x[n].pin_memory() for n in ("q", "k", "v", "do"))
+    host_out = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in
+                (("o", hq), ("dq", hq), ("dk", hk), ("dv", hv))}
+    host_out["lse"] = torch.empty((wf.B, wf.H_q, wf.S_q), dtype=torch.float32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in ((hq, hk, hv, hdo) if have_bwd else (hq, hk, hv)))
+    d2h_names = ("o", "lse", "dq", "dk", "dv") if have_bwd else ("o", "lse")
+    d2h = sum(host_out[n].numel() * host_out[n].element_size() for n in d2h_names)
+
+    def step():
+        if have_bwd:
+            attn.fwd_bwd(hq, hk, hv, hdo, causal=wf.causal, scale=wf.scale, host_out=host_out)
+        else:
+            o, lse = attn.fwd(hq, hk, hv, causal=wf.causal, scale=wf.scale)
+            host_out["o"].copy_(o)
+            host_out["lse"].copy_(lse)
+
+    n_steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(n_steps):
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        step()
+        e1.record()
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    step_ms = max_over_ranks(world, sum(ms) / len(ms))
+    flops = wf.fwd_flops() + (wb.bwd_flops() if have_bwd else 0.0)
+    return {"value": round(world * flops / (step_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
+            "ms_per_step": round(step_ms, 3), "steps": n_steps,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+# --------------------------------------------------------------------------- reference arm (the oracle)
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return  # rank 0 alone runs the CPU oracle
+    wf, wb = WORKLOADS[args.workload]
+    budget = max(5.0, min(60.0, args.cpu_budget))
+    vals, samples = [], []
+    t_all = time.perf_counter()
+    for _ in range(args.steps):
+        tf, sample, cores, dt = oracle_sample_time(wf, wb, budget_s=budget / max(1, args.steps))
+        vals.append(tf)
+        samples.append(dt)
+    value = statistics.mean(vals)
+    step_ms = statistics.mean(samples) * 1e3
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(step_ms, 1), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) rounded to bf16)",
+        "impl": "reference",
+        "config": {"workload": wf.name.replace("fwd_", "fwd+bwd_"), "B": wf.B, "H_q": wf.H_q, "S": wf.S_q,
+                   "D": wf.D, "causal": wf.causal, "parallelism": "CPU oracle on rank 0"},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                         "sample": sample + " per step (fp64 numpy)"},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": round(time.perf_counter() - t_all, 1),
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="causal8k")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU time to sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
