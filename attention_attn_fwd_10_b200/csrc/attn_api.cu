@@ -172,13 +172,13 @@ attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, 
   p.H_kv = H_kv;
   p.S_q = S_q;
   p.S_k = S_k;
-  p.n_q_tiles = (S_q + 127) / 128;
+  p.n_units = (S_q + 255) / 256;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.tau = opt.rescale_threshold;
   p.status = status;
   p.rescale_count = opt.rescale_count;
   p.wait_limit_ns = g_wait_limit_ns.load();
-  const unsigned grid = static_cast<unsigned>(p.n_q_tiles) * B * H_q;
+  const unsigned grid = static_cast<unsigned>(p.n_units) * B * H_q;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t err;
   if (D == 128)

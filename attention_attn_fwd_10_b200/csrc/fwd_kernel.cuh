@@ -1,17 +1,22 @@
 // Forward attention kernel for sm_100a:  O = softmax(scale * Q K^T [+ causal]) V, lse.
 //
-// One CTA owns one 128-row Q tile of one (batch, query head) and streams the
-// key/value blocks that tile can see.  Warp roles:
-//   warps 0-3  softmax warpgroup: thread t owns query row t of the tile (TMEM lane t)
-//   warp  4    TMA producer: Q once, then K_j / V_j into a 2-stage ring
-//   warp  5    TMEM allocator and single-thread tcgen05.mma issuer
-// Tensor-memory map (32-bit columns): S_0, S_1 (two 128x128 fp32 score
-// buffers), O (128 x D fp32), P_0, P_1 (128x128 bf16 probabilities, two per
-// column).  Issue order on the tensor pipe: S_0, S_1, PV_0, S_2, PV_1, ... so
-// the softmax of block j overlaps the S MMA of block j+1 and the PV MMA of
-// block j-1 (the fully asynchronous MMA pipeline of FlashAttention-4: "AI
-// Infra series ch. 6, GPU performance engineering (II)", section 7, and
-// "NVIDIA's strongest B200 wastes 60%", second move).
+// One CTA owns a work unit of 256 query rows of one (batch, query head) -- two
+// 128-row Q tiles, A and B -- and streams the key/value blocks they can see;
+// each K_j / V_j block is loaded once and used by both tiles.  Warp roles:
+//   warps 0-3   softmax warpgroup of tile A (thread t owns row t: TMEM lane t)
+//   warps 4-7   softmax warpgroup of tile B
+//   warp  8     TMA producer: Q_A, Q_B once, then K_j / V_j into a 2-stage ring
+//   warp  9     TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 10-11 idle (they complete the third warpgroup)
+// Tensor memory (32-bit columns): S_A, S_B (128 x 128 fp32 scores each),
+// O_A, O_B (128 x D fp32).  The softmax writes P_t (bf16, two per column)
+// over the first 64 columns of S_t, and the PV MMA reads it from there.
+// Tensor-pipe issue order per key block j:  PV_A(j), PV_B(j), S_A(j+1),
+// S_B(j+1); S_t(j+1) is issued only once PV_t(j) has completed (it overwrites
+// P_t(j)).  While one tile's softmax runs, the tensor pipe works on the other
+// tile's MMAs: the fully asynchronous MMA pipeline with softmax/MMA overlap of
+// FlashAttention-4 ("AI Infra series ch. 6, GPU performance engineering (II)",
+// section 7; "NVIDIA's strongest B200 wastes 60%", second move).
 //
 // Softmax (per row, base-2 units t = s * scale * log2 e):
 //   m_new = max(m_used, rowmax(t)); the running max actually used for the
@@ -32,7 +37,7 @@ struct FwdParams {
   __nv_bfloat16* o;  // [B, S_q, H_q, D]
   float* lse;        // [B, H_q, S_q]
   int B, H_q, H_kv, S_q, S_k;
-  int n_q_tiles;     // ceil(S_q / 128)
+  int n_units;       // ceil(S_q / 256) work units per (batch, head)
   float scale_log2;  // scale * log2(e)
   float tau;         // rescale threshold (base-2 units); 0 = rescale on every increase
   int* status;       // device status word
@@ -43,26 +48,26 @@ struct FwdParams {
 template <int D>
 struct FwdLayout {
   static constexpr int BM = 128;                 // query rows per tile
+  static constexpr int UNIT = 256;               // query rows per work unit (two tiles)
   static constexpr int BN = 128;                 // keys per block
   static constexpr int STAGES = 2;               // K/V ring depth
   static constexpr int NBOX = D / 64;            // 64-element (128 B) TMA boxes per row block
   static constexpr int BOX_BYTES = 128 * 128;    // one 128 x 64 bf16 box
   static constexpr int TILE_BYTES = 128 * D * 2; // one 128 x D bf16 tile
-  static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + TILE_BYTES;
+  static constexpr int Q_OFF = 0;                // two Q tiles
+  static constexpr int K_OFF = Q_OFF + 2 * TILE_BYTES;
   static constexpr int V_OFF = K_OFF + STAGES * TILE_BYTES;
   static constexpr int BAR_OFF = V_OFF + STAGES * TILE_BYTES;
-  // barrier slots (8 bytes each)
-  static constexpr int B_Q_FULL = 0;
-  static constexpr int B_K_FULL = 1;                  // + stage
-  static constexpr int B_V_FULL = B_K_FULL + STAGES;  // + stage
-  static constexpr int B_KV_EMPTY = B_V_FULL + STAGES;
-  static constexpr int B_S_FULL = B_KV_EMPTY + STAGES;  // + buffer
-  static constexpr int B_S_FREE = B_S_FULL + 2;
-  static constexpr int B_P_FULL = B_S_FREE + 2;
-  static constexpr int B_PV_DONE = B_P_FULL + 2;
-  static constexpr int B_O_FINAL = B_PV_DONE + 1;
-  static constexpr int B_DRAIN = B_O_FINAL + 1;
+  // barrier slots (8 bytes each); [t] = per Q tile, [s] = per ring stage
+  static constexpr int B_Q_FULL = 0;                    // [t]
+  static constexpr int B_K_FULL = B_Q_FULL + 2;         // [s]
+  static constexpr int B_V_FULL = B_K_FULL + STAGES;    // [s]
+  static constexpr int B_KV_EMPTY = B_V_FULL + STAGES;  // [s]
+  static constexpr int B_S_FULL = B_KV_EMPTY + STAGES;  // [t]
+  static constexpr int B_P_FULL = B_S_FULL + 2;         // [t]  (128 arrivals)
+  static constexpr int B_PV_DONE = B_P_FULL + 2;        // [t]
+  static constexpr int B_O_FINAL = B_PV_DONE + 2;       // [t]
+  static constexpr int B_DRAIN = B_O_FINAL + 2;
   static constexpr int N_BARS = B_DRAIN + 1;
   static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * N_BARS;
   static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 4;
@@ -71,10 +76,15 @@ struct FwdLayout {
   // at least 120 KiB so a single CTA occupies an SM (its TMEM request is 512 columns).
   static constexpr int SMEM_BYTES = (SMEM_USED + 1024) > 122880 ? (SMEM_USED + 1024) : 122880;
   // tensor memory columns
-  static constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL = 256;
-  static constexpr uint32_t P_COL0 = 256 + D, P_COL1 = 256 + D + 64;
+  __device__ static constexpr uint32_t s_col(int t) { return static_cast<uint32_t>(t) * 128u; }
+  __device__ static constexpr uint32_t o_col(int t) { return 256u + static_cast<uint32_t>(t) * D; }
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 192;
+  static constexpr int THREADS = 384;
+  static constexpr int WARP_TMA = 8, WARP_MMA = 9;
+  // Register split: launched at 168 per thread (384 x 168 = 64512); the two
+  // softmax warpgroups grow to 216 and the third shrinks to 72:
+  // 2 x 128 x 216 + 128 x 72 = 64512, exactly the launch's total.
+  static constexpr int REG_SOFTMAX = 216, REG_OTHER = 72;
 };
 
 // p = 2^(s * c - m) for one 128-column score row, packed to bf16 pairs; returns
@@ -102,8 +112,16 @@ __device__ __forceinline__ float exp_block(const float* s, float c, float m, uin
   return sum0 + sum1;
 }
 
-// POLY_EVERY: a column pair cp (columns 2cp, 2cp+1) of each score block takes
-// the FMA-pipe cubic when cp % POLY_EVERY == POLY_EVERY - 1 (0 = never).
+// Number of key blocks the rows [row0, row0 + 128) of a tile can see (0 if the
+// tile has no valid row, or none of its rows sees a key).
+__device__ __forceinline__ int tile_blocks(int row0, int S_q, int S_k, bool causal, int BN) {
+  if (row0 >= S_q) return 0;
+  const int n_kv = (S_k + BN - 1) / BN;
+  if (!causal) return n_kv;
+  const int last_key = min(row0 + 127, S_q - 1) + (S_k - S_q);
+  return last_key < 0 ? 0 : min(n_kv, last_key / BN + 1);
+}
+
 template <int D, bool CAUSAL, int POLY_EVERY>
 __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -120,39 +138,33 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work decode: longest tiles first for causal (blocks are dispatched in index order)
+  // ---- work decode: longest units first for causal (blocks are dispatched in index order)
   const int BH = p.B * p.H_q;
-  int qt = blockIdx.x / BH;
-  const int bh = blockIdx.x - qt * BH;
-  if (CAUSAL) qt = p.n_q_tiles - 1 - qt;
+  int u = blockIdx.x / BH;
+  const int bh = blockIdx.x - u * BH;
+  if (CAUSAL) u = p.n_units - 1 - u;
   const int b = bh / p.H_q;
   const int h = bh - b * p.H_q;
   const int hkv = h / (p.H_q / p.H_kv);
-  const int q0 = qt * L::BM;
-  const int diag = p.S_k - p.S_q;  // bottom-right causal offset: key j visible to row i iff j <= i + diag
-  const int n_kv_total = (p.S_k + L::BN - 1) / L::BN;
-  int n_blocks = n_kv_total;
-  if (CAUSAL) {
-    const int last_row = min(q0 + L::BM, p.S_q) - 1;
-    const int last_key = last_row + diag;
-    n_blocks = last_key < 0 ? 0 : min(n_kv_total, last_key / L::BN + 1);
-  }
+  const int q0 = u * L::UNIT;
+  const int diag = p.S_k - p.S_q;  // bottom-right causal: key j visible to row i iff j <= i + diag
+  int nblk[2];
+  nblk[0] = tile_blocks(q0, p.S_q, p.S_k, CAUSAL, L::BN);
+  nblk[1] = tile_blocks(q0 + L::BM, p.S_q, p.S_k, CAUSAL, L::BN);
+  const int n_blocks = max(nblk[0], nblk[1]);
 
   // ---- setup
   if (threadIdx.x == 0) {
-    for (int i = 0; i < L::N_BARS; ++i) {
-      uint32_t count = 1;
-      if (i == L::B_S_FREE || i == L::B_S_FREE + 1 || i == L::B_P_FULL || i == L::B_P_FULL + 1) count = 128;
-      mbar_init(bar(i), count);
-    }
+    for (int i = 0; i < L::N_BARS; ++i)
+      mbar_init(bar(i), (i == L::B_P_FULL || i == L::B_P_FULL + 1) ? 128u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == L::WARP_MMA) {
     tmem_alloc(sbase + L::TMEM_SLOT_OFF, L::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == L::WARP_TMA && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -161,14 +173,25 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sptr + L::TMEM_SLOT_OFF);
+  static_assert(2 * 128 * L::REG_SOFTMAX + 128 * L::REG_OTHER <= L::THREADS * 168, "register split");
 
-  if (warp == 4) {
+  if (warp >= 8) {
+    // Each role's register budget is set inside its own branch, so the
+    // register allocator sees the budget that dominates the role's code.
+    setmaxnreg_dec<L::REG_OTHER>();
+  }
+  if (warp == L::WARP_TMA) {
     // ===================== TMA producer =====================
     if (lane == 0 && n_blocks > 0) {
-      mbar_arrive_expect_tx(bar(L::B_Q_FULL), L::TILE_BYTES);
 #pragma unroll
-      for (int x = 0; x < L::NBOX; ++x)
-        tma_load_4d(sbase + L::Q_OFF + x * L::BOX_BYTES, &tm_q, bar(L::B_Q_FULL), x * 64, h, q0, b);
+      for (int t = 0; t < 2; ++t) {
+        if (nblk[t] == 0) continue;
+        mbar_arrive_expect_tx(bar(L::B_Q_FULL + t), L::TILE_BYTES);
+#pragma unroll
+        for (int x = 0; x < L::NBOX; ++x)
+          tma_load_4d(sbase + L::Q_OFF + t * L::TILE_BYTES + x * L::BOX_BYTES, &tm_q, bar(L::B_Q_FULL + t),
+                      x * 64, h, q0 + t * L::BM, b);
+      }
       int issued = 0;
       for (int j = 0; j < n_blocks; ++j) {
         const int s = j % L::STAGES;
@@ -186,89 +209,111 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
         issued = j + 1;
       }
       // Drain: every load this thread issued has landed before the CTA may exit.
-      mbar_wait_drain(bar(L::B_Q_FULL), 0, 1000000000ull);
+      for (int t = 0; t < 2; ++t)
+        if (nblk[t] > 0) mbar_wait_drain(bar(L::B_Q_FULL + t), 0, 1000000000ull);
       for (int s = 0; s < L::STAGES && s < issued; ++s) {
         const int uses = (issued - 1 - s) / L::STAGES + 1;
         mbar_wait_drain(bar(L::B_K_FULL + s), (uses - 1) & 1, 1000000000ull);
         mbar_wait_drain(bar(L::B_V_FULL + s), (uses - 1) & 1, 1000000000ull);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == L::WARP_MMA) {
     // ===================== MMA issuer =====================
     if (lane == 0 && n_blocks > 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
-      bool ok = mbar_wait(bar(L::B_Q_FULL), 0, ctl);
-      for (int j = 0; ok && j <= n_blocks; ++j) {
-        if (j < n_blocks) {
-          const int s = j % L::STAGES;
-          const int buf = j & 1;
-          if (!mbar_wait(bar(L::B_K_FULL + s), (j / L::STAGES) & 1, ctl)) break;
-          if (j >= 2 && !mbar_wait(bar(L::B_S_FREE + buf), ((j - 2) >> 1) & 1, ctl)) break;
-          tc_fence_after();
-          const uint32_t d_tmem = tmem + (buf ? L::S_COL1 : L::S_COL0);
-          const uint32_t q_base = sbase + L::Q_OFF;
-          const uint32_t k_base = sbase + L::K_OFF + s * L::TILE_BYTES;
+      auto issue_s = [&](int t, int stage) {
+        const uint32_t q_base = sbase + L::Q_OFF + t * L::TILE_BYTES;
+        const uint32_t k_base = sbase + L::K_OFF + stage * L::TILE_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32;
-            umma_ss(d_tmem, sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(k_base + off, 16, 1024), IDESC_S,
-                    kk > 0 ? 1u : 0u);
-          }
-          umma_commit(bar(L::B_S_FULL + buf));
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32;
+          umma_ss(tmem + L::s_col(t), sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(k_base + off, 16, 1024),
+                  IDESC_S, kk > 0 ? 1u : 0u);
         }
-        if (j >= 1) {
-          const int jj = j - 1;
-          const int s = jj % L::STAGES;
-          const int buf = jj & 1;
-          if (!mbar_wait(bar(L::B_P_FULL + buf), (jj >> 1) & 1, ctl)) break;
-          if (!mbar_wait(bar(L::B_V_FULL + s), (jj / L::STAGES) & 1, ctl)) break;
-          tc_fence_after();
-          const uint32_t v_base = sbase + L::V_OFF + s * L::TILE_BYTES;
-          const uint32_t p_tmem = tmem + (buf ? L::P_COL1 : L::P_COL0);
+        umma_commit(bar(L::B_S_FULL + t));
+      };
+      auto issue_pv = [&](int t, int stage, bool acc) {
+        const uint32_t v_base = sbase + L::V_OFF + stage * L::TILE_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < L::BN / 16; ++kk) {
-            // 16 keys = 16 rows of 128 B = 2048 bytes; column blocks of 64 d-values are BOX_BYTES apart.
-            umma_ts(tmem + L::O_COL, p_tmem + kk * 8, sdesc_sw128(v_base + kk * 2048, L::BOX_BYTES, 1024),
-                    IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < L::BN / 16; ++kk) {
+          // 16 keys = 16 rows of 128 B = 2048 bytes; 64-wide d blocks are BOX_BYTES apart.
+          umma_ts(tmem + L::o_col(t), tmem + L::s_col(t) + kk * 8,
+                  sdesc_sw128(v_base + kk * 2048, L::BOX_BYTES, 1024), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(bar(L::B_PV_DONE + t));
+      };
+      bool ok = mbar_wait(bar(L::B_K_FULL), 0, ctl);
+      for (int t = 0; ok && t < 2; ++t) {
+        if (nblk[t] == 0) continue;
+        ok = mbar_wait(bar(L::B_Q_FULL + t), 0, ctl);
+        if (ok) {
+          tc_fence_after();
+          issue_s(t, 0);
+        }
+      }
+      for (int j = 0; ok && j < n_blocks; ++j) {
+        const int s = j % L::STAGES;
+        if (!mbar_wait(bar(L::B_V_FULL + s), (j / L::STAGES) & 1, ctl)) break;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (!ok || j >= nblk[t]) continue;
+          ok = mbar_wait(bar(L::B_P_FULL + t), j & 1, ctl);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(t, s, j > 0);
+          if (j == nblk[t] - 1) umma_commit(bar(L::B_O_FINAL + t));
+        }
+        if (!ok) break;
+        umma_commit(bar(L::B_KV_EMPTY + s));
+        if (j + 1 < n_blocks) {
+          const int s1 = (j + 1) % L::STAGES;
+          if (!mbar_wait(bar(L::B_K_FULL + s1), ((j + 1) / L::STAGES) & 1, ctl)) break;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (!ok || j + 1 >= nblk[t]) continue;
+            // P_t(j) lives in S_t's columns: PV_t(j) must be complete before S_t(j+1).
+            ok = mbar_wait(bar(L::B_PV_DONE + t), j & 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(t, s1);
           }
-          umma_commit(bar(L::B_KV_EMPTY + s));
-          umma_commit(bar(L::B_PV_DONE));
-          if (jj == n_blocks - 1) umma_commit(bar(L::B_O_FINAL));
         }
       }
       // Drain: no MMA may still be writing TMEM when it is released.
       umma_commit(bar(L::B_DRAIN));
       mbar_wait_drain(bar(L::B_DRAIN), 0, 1000000000ull);
     }
-  } else {
-    // ===================== softmax warpgroup (warps 0-3) =====================
-    const int row = threadIdx.x;  // 0..127 == TMEM lane
-    const int qi = q0 + row;
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+  } else if (warp < 8) {
+    // ===================== softmax warpgroups (warps 0-3: tile A, 4-7: tile B) =====================
+    setmaxnreg_inc<L::REG_SOFTMAX>();
+    const int t = warp >> 2;
+    const int row = threadIdx.x & 127;  // == TMEM lane
+    const int row0 = q0 + t * L::BM;
+    const int qi = row0 + row;
+    const int nb = nblk[t];
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float c = p.scale_log2;
     const int lim = min(qi + (CAUSAL ? diag : p.S_k), p.S_k - 1);  // last visible key of this row
+    const int lim_tile = CAUSAL ? row0 + diag : p.S_k - 1;         // last key every row of the tile sees
     float m_used = -INFINITY;
     float l = 0.f;
     unsigned rescales = 0;
     bool ok = true;
-    for (int j = 0; j < n_blocks; ++j) {
-      const int buf = j & 1;
-      ok = mbar_wait(bar(L::B_S_FULL + buf), (j >> 1) & 1, ctl);
+    for (int j = 0; j < nb; ++j) {
+      ok = mbar_wait(bar(L::B_S_FULL + t), j & 1, ctl);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       uint32_t sr[128];
-      const uint32_t s_addr = tmem + lane_addr + (buf ? L::S_COL1 : L::S_COL0);
+      const uint32_t s_addr = tmem + lane_addr + L::s_col(t);
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) tmem_ld32(s_addr + ch * 32, sr + ch * 32);
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) tmem_ld_wait(sr + ch * 32);
-      tc_fence_before();
-      mbar_arrive(bar(L::B_S_FREE + buf));
 
       float* s = reinterpret_cast<float*>(sr);
       const int kbase = j * L::BN;
-      const bool need_mask = (kbase + L::BN - 1 > (CAUSAL ? q0 + diag : p.S_k - 1)) || (kbase + L::BN > p.S_k);
+      const bool need_mask = (kbase + L::BN - 1 > lim_tile) || (kbase + L::BN > p.S_k);
       if (need_mask) {
         const int lim_c = lim - kbase;
 #pragma unroll
@@ -292,16 +337,11 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       // Masked blocks take MUFU ex2 only: it maps -inf to an exact 0.
       const float rowsum = need_mask ? exp_block<0>(s, c, m_eff, pk) : exp_block<POLY_EVERY>(s, c, m_eff, pk);
       l += rowsum;
-      const uint32_t p_addr = tmem + lane_addr + (buf ? L::P_COL1 : L::P_COL0);
-      tmem_st32(p_addr, pk);
-      tmem_st32(p_addr + 32, pk + 32);
-      tmem_st_wait();
+      tmem_st32(s_addr, pk);  // P_t(j) over the first 64 columns of S_t
+      tmem_st32(s_addr + 32, pk + 32);
       if (j > 0 && __any_sync(0xffffffffu, resc)) {
-        // O must hold P_{j-1} V_{j-1} before it is rescaled.
-        ok = mbar_wait(bar(L::B_PV_DONE), (j - 1) & 1, ctl);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t o_addr = tmem + lane_addr + L::O_COL;
+        // PV_t(j-1) completed before S_t(j) was issued, so O_t is final up to block j-1.
+        const uint32_t o_addr = tmem + lane_addr + L::o_col(t);
 #pragma unroll 1
         for (int ch = 0; ch < D / 32; ++ch) {
           uint32_t orr[32];
@@ -311,16 +351,16 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
           for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
           tmem_st32(o_addr + ch * 32, orr);
         }
-        tmem_st_wait();
       }
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(L::B_P_FULL + buf));
+      mbar_arrive(bar(L::B_P_FULL + t));
     }
     if (p.rescale_count != nullptr && rescales) atomicAdd(p.rescale_count, (unsigned long long)rescales);
 
     // ---- epilogue: O / l -> bf16, lse
-    if (ok && n_blocks > 0) {
-      ok = mbar_wait(bar(L::B_O_FINAL), 0, ctl);
+    if (ok && nb > 0) {
+      ok = mbar_wait(bar(L::B_O_FINAL + t), 0, ctl);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
@@ -328,11 +368,11 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const bool valid = qi < p.S_q;
       __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.S_q + qi) * p.H_q + h) * D;
-      const uint32_t o_addr = tmem + lane_addr + L::O_COL;
+      const uint32_t o_addr = tmem + lane_addr + L::o_col(t);
 #pragma unroll 1
       for (int ch = 0; ch < D / 32; ++ch) {
         uint32_t orr[32];
-        if (n_blocks > 0) {
+        if (nb > 0) {
           tmem_ld32(o_addr + ch * 32, orr);
           tmem_ld_wait(orr);
         } else {
@@ -359,7 +399,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
   // ---- teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == L::WARP_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);
   }

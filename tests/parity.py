@@ -1,11 +1,18 @@
 """Shared tolerances and comparison helpers for the GPU-vs-oracle parity tests.
 
 Tolerances (inputs ~ N(0, 1), bf16 in/out, fp32 accumulation):
-  O    : |O_gpu - O_ref| <= max(1.5e-2, ulp_bf16(O_ref)) element-wise and
-         mean |O_gpu - O_ref| <= 2e-3.  The output is bf16 (round to nearest):
-         for |O| >= 4 half an ulp alone is 2^-6 = 0.0156 > 1.5e-2, so there the
-         bound is one bf16 ulp of the exact value (half for the output rounding,
-         half for the fp32/bf16-P error before it); below 4 it is 1.5e-2.
+  O    : mean |O_gpu - O_ref| <= 2e-3, and element-wise
+           |O_gpu - O_ref| <= max(1.5e-2, ulp_bf16(O_ref))            (N(0,1) inputs)
+         The output is bf16 (round to nearest): for |O| >= 4 half an ulp alone
+         is 2^-6 = 0.0156 > 1.5e-2, so there one bf16 ulp of the exact value is
+         allowed.  Inputs that are not N(0,1) (the spiky-key workload, whose
+         softmax rows can concentrate on one or two keys) are held instead to
+         the bound derived from the arithmetic:
+           |O_gpu - O_ref| <= max(1.5e-2, ulp_bf16(O_ref)/2 + 2^-9 * max|V| + 2e-3)
+         -- P is rounded to bf16 before the PV product (relative error <= 2^-9
+         on every weight, so <= 2^-9 * max|V| on the weighted sum), the output
+         is rounded to bf16 (half an ulp), and 2e-3 covers the fp32 terms and
+         the exponentials' approximation error (each below 1e-4 relative).
   lse  : max |lse_gpu - lse_ref| <= 1e-3
   grads: max |g_gpu - g_ref| <= 3e-2 * max |g_ref|, per tensor
 and every output finite (rows that see no key: O = 0, lse = -inf exactly).
@@ -30,11 +37,15 @@ def ulp_bf16(x: np.ndarray) -> np.ndarray:
     return np.where(ax > 0, 2.0 ** (e - 7), 0.0)
 
 
-def check_o(o_gpu, o_ref, what=""):
+def check_o(o_gpu, o_ref, what="", v_absmax=None):
+    """v_absmax: max |V| of the inputs; given only for inputs that are not N(0,1)."""
     o = to_np(o_gpu) if isinstance(o_gpu, torch.Tensor) else o_gpu
     assert np.all(np.isfinite(o)), f"{what}: non-finite O"
     err = np.abs(o - o_ref)
-    bound = np.maximum(O_MAX_ABS, ulp_bf16(o_ref))
+    if v_absmax is None:
+        bound = np.maximum(O_MAX_ABS, ulp_bf16(o_ref))
+    else:
+        bound = np.maximum(O_MAX_ABS, ulp_bf16(o_ref) / 2 + 2.0 ** -9 * v_absmax + 2e-3)
     worst = np.argmax(err - bound)
     assert np.all(err <= bound), (f"{what}: O error {err.flat[worst]:.3e} at |O_ref|={abs(o_ref.flat[worst]):.3f} "
                                   f"> bound {bound.flat[worst]:.3e}")
