@@ -31,6 +31,10 @@
 
 #include "sm100_common.cuh"
 
+#ifndef ATTN_FWD_PV_WAIT
+#define ATTN_FWD_PV_WAIT 0
+#endif
+
 namespace attn {
 
 struct FwdParams {
@@ -91,13 +95,17 @@ struct FwdLayout {
 // the fp32 sum of the unrounded p.  Column pair cp (columns 2cp, 2cp+1) takes
 // the FMA-pipe cubic when cp % POLY_EVERY == POLY_EVERY - 1, MUFU ex2 otherwise.
 template <int POLY_EVERY>
-__device__ __forceinline__ float exp_block(const float* s, float c, float m, uint32_t* pk) {
-  float sum0 = 0.f, sum1 = 0.f;
+__device__ __forceinline__ float exp_block(const uint32_t* sr, float c, float m, uint32_t* pk) {
+  const uint64_t c2 = f2_pack(c, c);
+  const uint64_t nm2 = f2_pack(-m, -m);
+  uint64_t acc[4];  // 4 independent packed partial sums (8 lanes of accumulation)
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i] = 0ull;
 #pragma unroll
   for (int cp = 0; cp < 64; ++cp) {
-    const float x0 = fmaf(s[2 * cp], c, -m);
-    const float x1 = fmaf(s[2 * cp + 1], c, -m);
-    float e0, e1;
+    const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[2 * cp]), __uint_as_float(sr[2 * cp + 1])), c2, nm2);
+    float x0, x1, e0, e1;
+    f2_unpack(x2, x0, x1);
     if (POLY_EVERY > 0 && (cp % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1) {
       e0 = exp2_poly(x0);
       e1 = exp2_poly(x1);
@@ -105,11 +113,26 @@ __device__ __forceinline__ float exp_block(const float* s, float c, float m, uin
       e0 = exp2_mufu(x0);
       e1 = exp2_mufu(x1);
     }
-    sum0 += e0;
-    sum1 += e1;
+    acc[cp & 3] = f2_add(acc[cp & 3], f2_pack(e0, e1));
     pk[cp] = pack_bf16x2(e0, e1);
   }
-  return sum0 + sum1;
+  float a0, a1;
+  f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
+  return a0 + a1;
+}
+
+// Maximum of a 128-column score row: 8 independent 3-input-max chains plus a tree.
+__device__ __forceinline__ float row_max128(const uint32_t* sr) {
+  const float* s = reinterpret_cast<const float*>(sr);
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = fmaxf(s[i], s[8 + i]);
+#pragma unroll
+  for (int cc = 16; cc < 128; cc += 16) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = fmax3(m[i], s[cc + i], s[cc + 8 + i]);
+  }
+  return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
 // Number of key blocks the rows [row0, row0 + 128) of a tile can see (0 if the
@@ -241,7 +264,9 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
           umma_ts(tmem + L::o_col(t), tmem + L::s_col(t) + kk * 8,
                   sdesc_sw128(v_base + kk * 2048, L::BOX_BYTES, 1024), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
         }
+#if ATTN_FWD_PV_WAIT
         umma_commit(bar(L::B_PV_DONE + t));
+#endif
       };
       bool ok = mbar_wait(bar(L::B_K_FULL), 0, ctl);
       for (int t = 0; ok && t < 2; ++t) {
@@ -252,9 +277,15 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
           issue_s(t, 0);
         }
       }
+      // Per key block j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1).  S_t(j+1) overwrites
+      // P_t(j), which PV_t(j) reads: the MMAs of this one issuing thread execute
+      // in issue order, so PV_t(j) has read P_t(j) before S_t(j+1) writes there
+      // (ATTN_FWD_PV_WAIT=1 makes the issuer wait for PV_t(j) to complete instead).
       for (int j = 0; ok && j < n_blocks; ++j) {
         const int s = j % L::STAGES;
+        const int s1 = (j + 1) % L::STAGES;
         if (!mbar_wait(bar(L::B_V_FULL + s), (j / L::STAGES) & 1, ctl)) break;
+        bool k_next_ready = false;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           if (!ok || j >= nblk[t]) continue;
@@ -263,22 +294,22 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
           tc_fence_after();
           issue_pv(t, s, j > 0);
           if (j == nblk[t] - 1) umma_commit(bar(L::B_O_FINAL + t));
-        }
-        if (!ok) break;
-        umma_commit(bar(L::B_KV_EMPTY + s));
-        if (j + 1 < n_blocks) {
-          const int s1 = (j + 1) % L::STAGES;
-          if (!mbar_wait(bar(L::B_K_FULL + s1), ((j + 1) / L::STAGES) & 1, ctl)) break;
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (!ok || j + 1 >= nblk[t]) continue;
-            // P_t(j) lives in S_t's columns: PV_t(j) must be complete before S_t(j+1).
+          if (j + 1 < nblk[t]) {
+            if (!k_next_ready) {
+              ok = mbar_wait(bar(L::B_K_FULL + s1), ((j + 1) / L::STAGES) & 1, ctl);
+              if (!ok) break;
+              k_next_ready = true;
+            }
+#if ATTN_FWD_PV_WAIT
             ok = mbar_wait(bar(L::B_PV_DONE + t), j & 1, ctl);
             if (!ok) break;
             tc_fence_after();
+#endif
             issue_s(t, s1);
           }
         }
+        if (!ok) break;
+        umma_commit(bar(L::B_KV_EMPTY + s));
       }
       // Drain: no MMA may still be writing TMEM when it is released.
       umma_commit(bar(L::B_DRAIN));
@@ -320,9 +351,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
         for (int cc = 0; cc < 128; ++cc)
           if (cc > lim_c) s[cc] = -INFINITY;
       }
-      float mx = s[0];
-#pragma unroll
-      for (int cc = 1; cc < 128; ++cc) mx = fmaxf(mx, s[cc]);
+      const float mx = row_max128(sr);
       const float m_new = fmaxf(m_used, mx * c);
       const bool resc = (m_new - m_used) > p.tau;  // false for NaN (-inf - -inf)
       float alpha = 1.f;
@@ -335,7 +364,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
       uint32_t pk[64];
       // Masked blocks take MUFU ex2 only: it maps -inf to an exact 0.
-      const float rowsum = need_mask ? exp_block<0>(s, c, m_eff, pk) : exp_block<POLY_EVERY>(s, c, m_eff, pk);
+      const float rowsum = need_mask ? exp_block<0>(sr, c, m_eff, pk) : exp_block<POLY_EVERY>(sr, c, m_eff, pk);
       l += rowsum;
       tmem_st32(s_addr, pk);  // P_t(j) over the first 64 columns of S_t
       tmem_st32(s_addr + 32, pk + 32);
