@@ -9,6 +9,7 @@
 #include <mutex>
 
 #include "../../include/attn.h"
+#include "bwd_kernels.cuh"
 #include "fwd_kernel.cuh"
 #include "sm100_common.cuh"
 
@@ -39,15 +40,15 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 BSHD tensor viewed as (D, H, S, B); boxes of 64 x 1 x 128 x 1, 128-byte swizzle.
-bool make_bshd_map(CUtensorMap* map, const void* ptr, int B, int S, int H, int D) {
+// bf16 BSHD tensor viewed as (D, H, S, B); boxes of 64 x 1 x box_rows x 1, 128-byte swizzle.
+bool make_bshd_map(CUtensorMap* map, const void* ptr, int B, int S, int H, int D, int box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(B)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
                                  static_cast<cuuint64_t>(S) * H * D * 2};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estride[4] = {1, 1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estride,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -197,9 +198,10 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
 
 size_t attn_bwd_workspace_size(int B, int H_q, int S_q, int D) {
   if (B < 1 || H_q < 1 || S_q < 1 || (D != 64 && D != 128)) return 0;
+  const size_t s_pad = (static_cast<size_t>(S_q) + 63) / 64 * 64;
   const size_t dq_acc = static_cast<size_t>(B) * S_q * H_q * D * sizeof(float);
-  const size_t delta = static_cast<size_t>(B) * H_q * S_q * sizeof(float);
-  return ((dq_acc + 255) / 256) * 256 + ((delta + 255) / 256) * 256;
+  const size_t rows = static_cast<size_t>(B) * H_q * s_pad * sizeof(float);
+  return (dq_acc + 255) / 256 * 256 + 2 * ((rows + 255) / 256 * 256);
 }
 
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
@@ -208,8 +210,83 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
   attn_status_t st = check_common(B, H_q, H_kv, S_q, S_k, D, causal, scale);
   if (st != ATTN_OK) return st;
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
-  (void)stream;
-  return ATTN_ERR_UNSUPPORTED;
+  if (D != 128) return ATTN_ERR_UNSUPPORTED;
+  for (const void* ptr : {q, k, v, o, static_cast<const void*>(lse), dO, static_cast<const void*>(dq),
+                          static_cast<const void*>(dk), static_cast<const void*>(dv), static_cast<const void*>(workspace)})
+    if (!aligned16(ptr)) return ATTN_ERR_MISALIGNED;
+  int* status = status_ptr();
+  if (!status) return ATTN_ERR_CUDA;
+
+  const int s_pad = (S_q + 63) / 64 * 64;
+  BwdParams p{};
+  p.o = static_cast<const __nv_bfloat16*>(o);
+  p.dO = static_cast<const __nv_bfloat16*>(dO);
+  p.lse = lse;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t dq_bytes = (static_cast<size_t>(B) * S_q * H_q * D * sizeof(float) + 255) / 256 * 256;
+  const size_t row_bytes = (static_cast<size_t>(B) * H_q * s_pad * sizeof(float) + 255) / 256 * 256;
+  p.dq_acc = reinterpret_cast<float*>(ws);
+  p.nlse2 = reinterpret_cast<float*>(ws + dq_bytes);
+  p.delta = reinterpret_cast<float*>(ws + dq_bytes + row_bytes);
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.B = B;
+  p.H_q = H_q;
+  p.H_kv = H_kv;
+  p.S_q = S_q;
+  p.S_k = S_k;
+  p.S_pad = s_pad;
+  p.n_kv_tiles = (S_k + 127) / 128;
+  p.scale = scale;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.status = status;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+
+  CUtensorMap mk, mv, mq, mdo;
+  if (!make_bshd_map(&mk, k, B, S_k, H_kv, D, 128) || !make_bshd_map(&mv, v, B, S_k, H_kv, D, 128) ||
+      !make_bshd_map(&mq, q, B, S_q, H_q, D, 64) || !make_bshd_map(&mdo, dO, B, S_q, H_q, D, 64))
+    return ATTN_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  // 1. preprocess
+  {
+    const long long rows = static_cast<long long>(B) * s_pad * H_q;
+    const long long blocks = (rows * (D / 8) + 255) / 256;
+    attn_bwd_preprocess_kernel<128><<<static_cast<unsigned>(blocks < 148 * 64 ? blocks : 148 * 64), 256, 0, s>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  // 2. main pass
+  {
+    using L = BwdLayout<128>;
+    const unsigned grid = static_cast<unsigned>(p.n_kv_tiles) * B * H_kv;
+    cudaError_t err;
+    if (causal) {
+      auto kern = attn_bwd_kernel<128, true>;
+      static std::once_flag once;
+      static cudaError_t attr = cudaSuccess;
+      std::call_once(once, [&] { attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES); });
+      if (attr != cudaSuccess) return ATTN_ERR_CUDA;
+      kern<<<grid, L::THREADS, L::SMEM_BYTES, s>>>(mk, mv, mq, mdo, p);
+    } else {
+      auto kern = attn_bwd_kernel<128, false>;
+      static std::once_flag once;
+      static cudaError_t attr = cudaSuccess;
+      std::call_once(once, [&] { attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES); });
+      if (attr != cudaSuccess) return ATTN_ERR_CUDA;
+      kern<<<grid, L::THREADS, L::SMEM_BYTES, s>>>(mk, mv, mq, mdo, p);
+    }
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  // 3. dQ convert
+  {
+    const long long n8 = static_cast<long long>(B) * S_q * H_q * D / 8;
+    const long long blocks = (n8 + 255) / 256;
+    attn_bwd_convert_kernel<<<static_cast<unsigned>(blocks < 148 * 64 ? blocks : 148 * 64), 256, 0, s>>>(p, n8, D);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
 }
 
 attn_status_t attn_device_status(void* stream) {

@@ -1,0 +1,465 @@
+// Backward attention kernels for sm_100a: dQ, dK, dV of L = sum(dO * O).
+//
+// Three launches on one stream:
+//   1. attn_bwd_preprocess_kernel  delta_i = sum_d dO_id O_id (fp32), -lse_i*log2(e)
+//                                  into padded rows, and dQ_acc = 0
+//   2. attn_bwd_kernel             KV-stationary main pass (below)
+//   3. attn_bwd_convert_kernel     dQ = scale * dQ_acc -> bf16
+//
+// Main pass: one CTA owns one 128-key tile (K_j, V_j) of one (batch, kv head)
+// and visits every 64-query block (Q_i, dO_i) of every query head of the
+// group that sees it.  P is recomputed from lse rather than stored
+// ("AI Infra series ch. 6, GPU performance engineering (II)", section 5,
+// recomputation).  Per query block, all on tcgen05 with fp32 accumulation:
+//   S^T  = K_j Q_i^T      (128 x 64, TMEM X)     dP^T = V_j dO_i^T   (TMEM Y)
+//   P^T  = 2^(S^T c - lse2_i),  dS^T = P^T o (dP^T - delta_i)     (softmax warpgroup)
+//          P^T (bf16) is written over X and dS^T (bf16) over Y -- the
+//          intermediates stay in tensor memory (section 7, item 3) -- and
+//          dS^T also goes to shared memory for the dQ product
+//   dV_j += P^T dO_i     (A from TMEM X)         dK_j += dS^T Q_i    (A from TMEM Y)
+//   dQ_i^T = K_j^T dS^T  (128 x 64: both operands MN-major in shared memory)
+// dV_j, dK_j accumulate in TMEM over all query blocks; dQ_i^T goes to one of
+// two TMEM buffers and a second warpgroup adds it into the fp32 dQ
+// accumulator with coalesced atomic adds (the "atomic reductions" of
+// section 7, item 3).  Every MMA has M = 128.
+// Tensor-pipe order per block i: dV_i, dK_i, S^T_{i+1}, dP^T_{i+1}, dQ^T_i, so
+// the softmax of block i+1 overlaps dQ^T_i; S^T_{i+1} / dP^T_{i+1} overwrite
+// P^T_i / dS^T_i after dV_i / dK_i have read them (one issuing thread: the
+// MMAs execute in issue order).
+//
+// Warp roles (384 threads): warps 0-3 softmax / dS and the dK, dV epilogue
+// (thread = key row = TMEM lane); warps 4-7 dQ reduction (thread = head-dim
+// row of dQ^T); warp 8 TMA producer; warp 9 TMEM allocator and MMA issuer;
+// warps 10-11 idle.
+#pragma once
+
+#include "sm100_common.cuh"
+
+namespace attn {
+
+struct BwdParams {
+  const __nv_bfloat16* o;   // [B, S_q, H_q, D]
+  const __nv_bfloat16* dO;  // [B, S_q, H_q, D]
+  const float* lse;         // [B, H_q, S_q] natural log
+  float* dq_acc;            // [B, S_q, H_q, D] fp32 (workspace)
+  float* nlse2;             // [B, H_q, S_pad] = -lse * log2(e); -inf for padding / empty rows (workspace)
+  float* delta;             // [B, H_q, S_pad] (workspace)
+  __nv_bfloat16* dq;        // [B, S_q, H_q, D]
+  __nv_bfloat16* dk;        // [B, S_k, H_kv, D]
+  __nv_bfloat16* dv;        // [B, S_k, H_kv, D]
+  int B, H_q, H_kv, S_q, S_k, S_pad;
+  int n_kv_tiles;           // ceil(S_k / 128)
+  float scale, scale_log2;
+  int* status;
+  uint64_t wait_limit_ns;
+};
+
+// ---------------------------------------------------------------------------
+// 1. preprocess: half a warp per (b, q, h) row of D = 128 (8 bf16 per lane)
+template <int D>
+__global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(const BwdParams p) {
+  constexpr int LANES = D / 8;          // lanes per row (8 bf16 each)
+  constexpr int ROWS_PER_WARP = 32 / LANES;
+  const long long rows = static_cast<long long>(p.B) * p.S_pad * p.H_q;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane % LANES;
+  const long long warp_id = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  // whole warps iterate together (the row reduction below shuffles across the warp)
+  for (long long r0 = warp_id * ROWS_PER_WARP; r0 < rows; r0 += n_warps * ROWS_PER_WARP) {
+    const long long row = r0 + lane / LANES;
+    const bool in_range = row < rows;
+    const int h = static_cast<int>(row % p.H_q);
+    const long long bq = row / p.H_q;
+    const int q = static_cast<int>(bq % p.S_pad);
+    const int b = static_cast<int>(bq / p.S_pad);
+    float dot = 0.f;
+    if (in_range && q < p.S_q) {
+      const size_t base = ((static_cast<size_t>(b) * p.S_q + q) * p.H_q + h) * D + sub * 8;
+      const uint4 ov = *reinterpret_cast<const uint4*>(p.o + base);
+      const uint4 dv = *reinterpret_cast<const uint4*>(p.dO + base);
+      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+      const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 of = __bfloat1622float2(o2[i]);
+        const float2 df = __bfloat1622float2(d2[i]);
+        dot = fmaf(of.x, df.x, dot);
+        dot = fmaf(of.y, df.y, dot);
+      }
+      float4* acc = reinterpret_cast<float4*>(p.dq_acc + base);
+      acc[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      acc[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int off = LANES / 2; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off, LANES);
+    if (in_range && sub == 0) {
+      const size_t r = (static_cast<size_t>(b) * p.H_q + h) * p.S_pad + q;
+      float nl = -INFINITY;  // padding rows and rows that saw no key give P = 0
+      if (q < p.S_q) {
+        const float l = p.lse[(static_cast<size_t>(b) * p.H_q + h) * p.S_q + q];
+        if (l > -INFINITY) nl = -l * 1.4426950408889634f;
+      }
+      p.nlse2[r] = nl;
+      p.delta[r] = q < p.S_q ? dot : 0.f;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 3. convert: dQ = scale * dQ_acc, 8 elements per thread
+__global__ void __launch_bounds__(256) attn_bwd_convert_kernel(const BwdParams p, long long n8, int D) {
+  (void)D;
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n8;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4* src = reinterpret_cast<const float4*>(p.dq_acc) + 2 * i;
+    const float4 a = src[0], b = src[1];
+    uint4 r;
+    r.x = pack_bf16x2(a.x * p.scale, a.y * p.scale);
+    r.y = pack_bf16x2(a.z * p.scale, a.w * p.scale);
+    r.z = pack_bf16x2(b.x * p.scale, b.y * p.scale);
+    r.w = pack_bf16x2(b.z * p.scale, b.w * p.scale);
+    reinterpret_cast<uint4*>(p.dq)[i] = r;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 2. main pass
+template <int D>
+struct BwdLayout {
+  static constexpr int BN = 128;                  // keys per CTA
+  static constexpr int BQ = 64;                   // queries per block
+  static constexpr int NBOX = D / 64;
+  static constexpr int KBOX_BYTES = 128 * 128;    // 128 rows x 128 B
+  static constexpr int QBOX_BYTES = 64 * 128;     // 64 rows x 128 B
+  static constexpr int KV_TILE = 128 * D * 2;
+  static constexpr int Q_TILE = 64 * D * 2;
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = K_OFF + KV_TILE;
+  static constexpr int STAGE_OFF = V_OFF + KV_TILE;
+  // one stage: Q_i, dO_i, -lse2_i (64 fp32), delta_i (64 fp32); 1024-aligned
+  static constexpr int ST_Q = 0, ST_DO = Q_TILE, ST_L = 2 * Q_TILE, ST_DL = 2 * Q_TILE + 256;
+  static constexpr int STAGE_BYTES = ((2 * Q_TILE + 512 + 1023) / 1024) * 1024;
+  static constexpr int DS_OFF = STAGE_OFF + 2 * STAGE_BYTES;  // two dS^T buffers, 128 x 64 bf16
+  static constexpr int DS_BYTES = 128 * 64 * 2;
+  static constexpr int BAR_OFF = DS_OFF + 2 * DS_BYTES;
+  static constexpr int B_KV_FULL = 0;
+  static constexpr int B_QDO_FULL = 1;    // [2]
+  static constexpr int B_QDO_EMPTY = 3;   // [2]
+  static constexpr int B_S_FULL = 5;
+  static constexpr int B_DS_READY = 6;    // 128 arrivals
+  static constexpr int B_DQ_FULL = 7;     // [2]
+  static constexpr int B_DQ_FREE = 9;     // [2] 128 arrivals
+  static constexpr int B_D_FINAL = 11;
+  static constexpr int B_DRAIN = 12;
+  static constexpr int N_BARS = 13;
+  static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * N_BARS;
+  static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 4;
+  static constexpr int SMEM_USED = ABORT_OFF + 4;
+  static constexpr int SMEM_BYTES = (SMEM_USED + 1024) > 122880 ? (SMEM_USED + 1024) : 122880;
+  // tensor memory columns
+  static constexpr uint32_t X_COL = 0;              // S^T, then P^T (bf16) over its first 32 columns
+  static constexpr uint32_t Y_COL = 64;             // dP^T, then dS^T (bf16)
+  static constexpr uint32_t DV_COL = 128;           // D columns
+  static constexpr uint32_t DK_COL = 128 + D;       // D columns
+  __device__ static constexpr uint32_t dq_col(int b) { return 128 + 2 * D + 64 * b; }
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr int THREADS = 384;
+  static constexpr int WARP_TMA = 8, WARP_MMA = 9;
+  static constexpr int REG_MAIN = 216, REG_OTHER = 72;  // 2 x 128 x 216 + 128 x 72 = 384 x 168
+};
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
+    attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                    const BwdParams p) {
+  using L = BwdLayout<D>;
+  static_assert(D == 128, "the backward main pass is built for D = 128");
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* const sptr = smem_raw + (sbase - raw);
+  auto bar = [&](int slot) -> uint32_t { return sbase + L::BAR_OFF + 8u * slot; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + L::ABORT_OFF);
+  const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work decode: causal tiles with the most query blocks (low key index) first
+  const int BH = p.B * p.H_kv;
+  const int j = blockIdx.x / BH;
+  const int bh = blockIdx.x - j * BH;
+  const int b = bh / p.H_kv;
+  const int hkv = bh - b * p.H_kv;
+  const int G = p.H_q / p.H_kv;
+  const int k0 = j * L::BN;
+  const int diag = p.S_k - p.S_q;  // key k visible to query q iff k <= q + diag
+  const int n_qb = p.S_pad / L::BQ;
+  int qb0 = 0;
+  if (CAUSAL) {
+    const int first_q = k0 - diag;  // first query that sees key k0
+    qb0 = first_q <= 0 ? 0 : min(n_qb, first_q / L::BQ);
+  }
+  const int per_head = n_qb - qb0;
+  const int m = G * per_head;  // query blocks this CTA visits
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::N_BARS; ++i)
+      mbar_init(bar(i), (i == L::B_DS_READY || i == L::B_DQ_FREE || i == L::B_DQ_FREE + 1) ? 128u : 1u);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == L::WARP_MMA) {
+    tmem_alloc(sbase + L::TMEM_SLOT_OFF, L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == L::WARP_TMA && lane == 0) {
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_do);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sptr + L::TMEM_SLOT_OFF);
+
+  if (warp >= 8) setmaxnreg_dec<L::REG_OTHER>();
+
+  if (warp == L::WARP_TMA) {
+    // ===================== TMA producer =====================
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar(L::B_KV_FULL), 2 * L::KV_TILE);
+#pragma unroll
+      for (int x = 0; x < L::NBOX; ++x) {
+        tma_load_4d(sbase + L::K_OFF + x * L::KBOX_BYTES, &tm_k, bar(L::B_KV_FULL), x * 64, hkv, k0, b);
+        tma_load_4d(sbase + L::V_OFF + x * L::KBOX_BYTES, &tm_v, bar(L::B_KV_FULL), x * 64, hkv, k0, b);
+      }
+      int issued = 0;
+      for (int i = 0; i < m; ++i) {
+        const int st = i & 1;
+        if (i >= 2 && !mbar_wait(bar(L::B_QDO_EMPTY + st), ((i >> 1) - 1) & 1, ctl)) break;
+        const int h = hkv * G + i / per_head;
+        const int q0 = (qb0 + i % per_head) * L::BQ;
+        const uint32_t sb = sbase + L::STAGE_OFF + st * L::STAGE_BYTES;
+        const uint32_t fb = bar(L::B_QDO_FULL + st);
+        mbar_arrive_expect_tx(fb, 2 * L::Q_TILE + 512);
+#pragma unroll
+        for (int x = 0; x < L::NBOX; ++x) {
+          tma_load_4d(sb + L::ST_Q + x * L::QBOX_BYTES, &tm_q, fb, x * 64, h, q0, b);
+          tma_load_4d(sb + L::ST_DO + x * L::QBOX_BYTES, &tm_do, fb, x * 64, h, q0, b);
+        }
+        const size_t r = (static_cast<size_t>(b) * p.H_q + h) * p.S_pad + q0;
+        bulk_load(sb + L::ST_L, p.nlse2 + r, 256, fb);
+        bulk_load(sb + L::ST_DL, p.delta + r, 256, fb);
+        issued = i + 1;
+      }
+      mbar_wait_drain(bar(L::B_KV_FULL), 0, 1000000000ull);
+      for (int st = 0; st < 2 && st < issued; ++st) {
+        const int uses = (issued - 1 - st) / 2 + 1;
+        mbar_wait_drain(bar(L::B_QDO_FULL + st), (uses - 1) & 1, 1000000000ull);
+      }
+    }
+  } else if (warp == L::WARP_MMA) {
+    // ===================== MMA issuer =====================
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_bf16_f32(128, L::BQ, false, false);   // S^T, dP^T
+      constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, false, true);        // dV, dK (A in TMEM)
+      constexpr uint32_t IDESC_Q = idesc_bf16_f32(D, L::BQ, true, true);       // dQ^T
+      const uint32_t k_base = sbase + L::K_OFF, v_base = sbase + L::V_OFF;
+      auto issue_s_dp = [&](int st) {
+        const uint32_t sb = sbase + L::STAGE_OFF + st * L::STAGE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ao = (kk >> 2) * L::KBOX_BYTES + (kk & 3) * 32;
+          const uint32_t bo = (kk >> 2) * L::QBOX_BYTES + (kk & 3) * 32;
+          umma_ss(tmem + L::X_COL, sdesc_sw128(k_base + ao, 16, 1024), sdesc_sw128(sb + L::ST_Q + bo, 16, 1024),
+                  IDESC_S, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ao = (kk >> 2) * L::KBOX_BYTES + (kk & 3) * 32;
+          const uint32_t bo = (kk >> 2) * L::QBOX_BYTES + (kk & 3) * 32;
+          umma_ss(tmem + L::Y_COL, sdesc_sw128(v_base + ao, 16, 1024), sdesc_sw128(sb + L::ST_DO + bo, 16, 1024),
+                  IDESC_S, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(bar(L::B_S_FULL));
+      };
+      bool ok = mbar_wait(bar(L::B_KV_FULL), 0, ctl);
+      if (ok && m > 0) {
+        ok = mbar_wait(bar(L::B_QDO_FULL), 0, ctl);
+        if (ok) {
+          tc_fence_after();
+          issue_s_dp(0);
+        }
+      }
+      for (int i = 0; ok && i < m; ++i) {
+        const int st = i & 1;
+        const uint32_t sb = sbase + L::STAGE_OFF + st * L::STAGE_BYTES;
+        if (!mbar_wait(bar(L::B_DS_READY), i & 1, ctl)) break;
+        tc_fence_after();
+        // dV += P^T dO_i ; dK += dS^T Q_i   (16 queries per MMA: 8 TMEM columns, 2048 B of the stage)
+#pragma unroll
+        for (int kk = 0; kk < L::BQ / 16; ++kk)
+          umma_ts(tmem + L::DV_COL, tmem + L::X_COL + kk * 8, sdesc_sw128(sb + L::ST_DO + kk * 2048, L::QBOX_BYTES, 1024),
+                  IDESC_G, (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < L::BQ / 16; ++kk)
+          umma_ts(tmem + L::DK_COL, tmem + L::Y_COL + kk * 8, sdesc_sw128(sb + L::ST_Q + kk * 2048, L::QBOX_BYTES, 1024),
+                  IDESC_G, (i > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(L::B_QDO_EMPTY + st));
+        if (i + 1 < m) {
+          if (!mbar_wait(bar(L::B_QDO_FULL + (st ^ 1)), ((i + 1) >> 1) & 1, ctl)) break;
+          tc_fence_after();
+          issue_s_dp(st ^ 1);
+        }
+        if (i >= 2) {
+          if (!mbar_wait(bar(L::B_DQ_FREE + st), ((i - 2) >> 1) & 1, ctl)) break;
+          tc_fence_after();
+        }
+        // dQ_i^T = K_j^T dS_i^T : 16 keys per MMA = 2048 B of K_j and of dS^T
+        const uint32_t ds = sbase + L::DS_OFF + st * L::DS_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < L::BN / 16; ++kk)
+          umma_ss(tmem + L::dq_col(st), sdesc_sw128(k_base + kk * 2048, L::KBOX_BYTES, 1024),
+                  sdesc_sw128(ds + kk * 2048, L::DS_BYTES, 1024), IDESC_Q, kk > 0 ? 1u : 0u);
+        umma_commit(bar(L::B_DQ_FULL + st));
+      }
+      if (ok) umma_commit(bar(L::B_D_FINAL));
+      umma_commit(bar(L::B_DRAIN));
+      mbar_wait_drain(bar(L::B_DRAIN), 0, 1000000000ull);
+    }
+  } else if (warp < 4) {
+    // ===================== softmax / dS warpgroup: thread = key row =====================
+    setmaxnreg_inc<L::REG_MAIN>();
+    const int r = threadIdx.x;
+    const int key = k0 + r;
+    const bool valid_key = key < p.S_k;
+    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+    bool ok = true;
+    for (int i = 0; i < m; ++i) {
+      const int st = i & 1;
+      const int q0 = (qb0 + i % per_head) * L::BQ;
+      ok = mbar_wait(bar(L::B_S_FULL), i & 1, ctl);
+      if (ok && i >= 2) ok = mbar_wait(bar(L::B_DQ_FULL + st), ((i - 2) >> 1) & 1, ctl);  // dS^T buffer free
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t sv[64], dp[64];
+      tmem_ld32(tmem + lane_addr + L::X_COL, sv);
+      tmem_ld32(tmem + lane_addr + L::X_COL + 32, sv + 32);
+      tmem_ld32(tmem + lane_addr + L::Y_COL, dp);
+      tmem_ld32(tmem + lane_addr + L::Y_COL + 32, dp + 32);
+      tmem_ld_wait(sv);
+      tmem_ld_wait(sv + 32);
+      tmem_ld_wait(dp);
+      tmem_ld_wait(dp + 32);
+      const float* nl = reinterpret_cast<const float*>(sptr + L::STAGE_OFF + st * L::STAGE_BYTES + L::ST_L);
+      const float* dl = reinterpret_cast<const float*>(sptr + L::STAGE_OFF + st * L::STAGE_BYTES + L::ST_DL);
+      // causal: key visible to query q0 + c iff c >= key - diag - q0; keys past S_k see nothing
+      const int c_first = !valid_key ? L::BQ : (CAUSAL ? key - diag - q0 : 0);
+      uint32_t pp[32], pd[32];
+#pragma unroll
+      for (int cp = 0; cp < 32; ++cp) {
+        const float2 nlv = *reinterpret_cast<const float2*>(nl + 2 * cp);
+        const float2 dlv = *reinterpret_cast<const float2*>(dl + 2 * cp);
+        const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[2 * cp]), __uint_as_float(sv[2 * cp + 1])), c2,
+                                   f2_pack(nlv.x, nlv.y));
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        float p0 = exp2_mufu(x0), p1 = exp2_mufu(x1);
+        if (2 * cp < c_first) p0 = 0.f;
+        if (2 * cp + 1 < c_first) p1 = 0.f;
+        const uint64_t g2 = f2_sub(f2_pack(__uint_as_float(dp[2 * cp]), __uint_as_float(dp[2 * cp + 1])),
+                                   f2_pack(dlv.x, dlv.y));
+        float d0, d1;
+        f2_unpack(f2_mul(f2_pack(p0, p1), g2), d0, d1);
+        pp[cp] = pack_bf16x2(p0, p1);
+        pd[cp] = pack_bf16x2(d0, d1);
+      }
+      tmem_st32(tmem + lane_addr + L::X_COL, pp);  // P^T (bf16 pairs)
+      tmem_st32(tmem + lane_addr + L::Y_COL, pd);  // dS^T
+      // dS^T row r into the 128B-swizzled MN-major operand: 16-byte chunk c goes to chunk c ^ (r % 8)
+      uint8_t* dsrow = sptr + L::DS_OFF + st * L::DS_BYTES + r * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(dsrow + ((c ^ (r & 7)) << 4)) =
+            make_uint4(pd[4 * c], pd[4 * c + 1], pd[4 * c + 2], pd[4 * c + 3]);
+      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar(L::B_DS_READY));
+    }
+    // ---- epilogue: dV, dK (scaled) -> bf16
+    if (ok && m > 0) {
+      ok = mbar_wait(bar(L::B_D_FINAL), 0, ctl);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const size_t rowoff = ((static_cast<size_t>(b) * p.S_k + key) * p.H_kv + hkv) * D;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t col = which == 0 ? L::DV_COL : L::DK_COL;
+        const float sc = which == 0 ? 1.f : p.scale;
+        __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + rowoff;
+#pragma unroll 1
+        for (int ch = 0; ch < D / 32; ++ch) {
+          uint32_t v[32];
+          if (m > 0) {
+            tmem_ld32(tmem + lane_addr + col + ch * 32, v);
+            tmem_ld_wait(v);
+          } else {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) v[t] = 0u;
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t)
+            pk[t] = pack_bf16x2(__uint_as_float(v[2 * t]) * sc, __uint_as_float(v[2 * t + 1]) * sc);
+          if (valid_key) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 32);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) d4[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+          }
+        }
+      }
+    }
+  } else if (warp < 8) {
+    // ===================== dQ reduction warpgroup: thread = head-dim index =====================
+    setmaxnreg_inc<L::REG_MAIN>();
+    const int d = threadIdx.x - 128;
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const size_t qstride = static_cast<size_t>(p.H_q) * D;
+    for (int i = 0; i < m; ++i) {
+      const int st = i & 1;
+      bool ok = mbar_wait(bar(L::B_DQ_FULL + st), (i >> 1) & 1, ctl);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      uint32_t v[64];
+      tmem_ld32(tmem + lane_addr + L::dq_col(st), v);
+      tmem_ld32(tmem + lane_addr + L::dq_col(st) + 32, v + 32);
+      tmem_ld_wait(v);
+      tmem_ld_wait(v + 32);
+      tc_fence_before();
+      mbar_arrive(bar(L::B_DQ_FREE + st));
+      const int h = hkv * G + i / per_head;
+      const int q0 = (qb0 + i % per_head) * L::BQ;
+      float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.S_q + q0) * p.H_q + h) * D + d;
+      const int nq = min(L::BQ, p.S_q - q0);
+#pragma unroll
+      for (int c = 0; c < L::BQ; ++c)
+        if (c < nq) atomicAdd(dst + c * qstride, __uint_as_float(v[c]));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == L::WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+}  // namespace attn

@@ -1,0 +1,90 @@
+"""GPU backward vs the fp64 oracle, through the C ABI.  The GPU backward consumes
+the GPU forward's O and lse; the oracle recomputes its own fp64 P."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import reference as ref
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _attn():
+    import attention_attn_fwd_10_b200 as attn
+
+    return attn
+
+
+def _gpu_fwd_bwd(x, causal, scale):
+    attn = _attn()
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = attn.fwd(q, k, v, causal=causal, scale=scale)
+    dq, dk, dv = attn.bwd(q, k, v, o, lse, do, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    assert attn.device_status() == 0
+    return dq, dk, dv
+
+
+def _check(w, x, grads, groups=None, batches=None):
+    ref_g = ref.backward(x["q"], x["k"], x["v"], x["do"], w.causal, w.scale, groups=groups, batches=batches)
+    G = w.H_q // w.H_kv
+    for name, g, gr in zip(("dq", "dk", "dv"), grads, ref_g):
+        g = parity.to_np(g)
+        if groups is not None:
+            bs = batches if batches is not None else range(w.B)
+            sel_q = [h for grp in groups for h in range(grp * G, (grp + 1) * G)]
+            idx = (list(bs), slice(None), sel_q if name == "dq" else list(groups), slice(None))
+            g = g[np.ix_(idx[0], range(g.shape[1]), idx[2], range(g.shape[3]))]
+            gr = gr[np.ix_(idx[0], range(gr.shape[1]), idx[2], range(gr.shape[3]))]
+        parity.check_grad(g, gr, f"{w.name} {name}")
+
+
+@pytest.mark.parametrize("S_q,S_k", [(1, 1), (17, 17), (64, 64), (127, 127), (128, 128), (129, 129),
+                                     (200, 200), (300, 300), (100, 260), (260, 100)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_small_shapes(S_q, S_k, causal):
+    w = workloads.small(B=2, H_q=2, S_q=S_q, S_k=S_k, D=128, causal=causal, seed=S_q * 7 + S_k, backward=True)
+    x = workloads.make_inputs(w)
+    _check(w, x, _gpu_fwd_bwd(x, causal, w.scale))
+
+
+@pytest.mark.parametrize("H_q,H_kv", [(4, 1), (8, 2), (6, 3)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa(H_q, H_kv, causal):
+    w = workloads.small(B=1, H_q=H_q, H_kv=H_kv, S_q=384, S_k=384, D=128, causal=causal, seed=21, backward=True)
+    x = workloads.make_inputs(w)
+    _check(w, x, _gpu_fwd_bwd(x, causal, w.scale))
+
+
+def test_medium_causal():
+    w = workloads.small(B=1, H_q=2, S_q=1536, S_k=1536, D=128, causal=True, seed=33, backward=True)
+    x = workloads.make_inputs(w)
+    _check(w, x, _gpu_fwd_bwd(x, True, w.scale))
+
+
+def test_backward_config_sampled_heads_and_invariants():
+    w = workloads.BWD_CAUSAL
+    x = workloads.make_inputs(w)
+    dq, dk, dv = _gpu_fwd_bwd(x, w.causal, w.scale)
+    # whole (b, kv head) groups checked against the oracle: first and last
+    _check(w, x, (dq, dk, dv), groups=[0], batches=[0])
+    _check(w, x, (dq, dk, dv), groups=[w.H_kv - 1], batches=[w.B - 1])
+    # properties at full size: sum over keys of dK is 0; sum over keys of dV = sum over queries of dO
+    dk64 = dk.double()
+    assert torch.isfinite(dq.float()).all() and torch.isfinite(dk.float()).all() and torch.isfinite(dv.float()).all()
+    assert dk64.sum(dim=1).abs().max() <= 3e-2 * dk64.abs().max() * w.S_k ** 0.5
+    sum_dv = dv.double().sum(dim=1)
+    sum_do = x["do"].double().sum(dim=1).cuda()
+    assert (sum_dv - sum_do).abs().max() <= 3e-2 * sum_do.abs().max()
+
+
+def test_unsupported_head_dim_is_rejected():
+    attn = _attn()
+    w = workloads.small(B=1, H_q=1, S_q=64, S_k=64, D=64, causal=False, seed=1, backward=True)
+    x = workloads.make_inputs(w)
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = attn.fwd(q, k, v)
+    with pytest.raises(RuntimeError, match="UNSUPPORTED"):
+        attn.bwd(q, k, v, o, lse, do)
