@@ -14,7 +14,10 @@ Tolerances (inputs ~ N(0, 1), bf16 in/out, fp32 accumulation):
          is rounded to bf16 (half an ulp), and 2e-3 covers the fp32 terms and
          the exponentials' approximation error (each below 1e-4 relative).
   lse  : max |lse_gpu - lse_ref| <= 1e-3
-  grads: max |g_gpu - g_ref| <= 3e-2 * max |g_ref|, per tensor
+  grads: max |g_gpu - g_ref| <= 3e-2 * max(max |g_ref|, 1e-3), per tensor.  The
+         1e-3 floor only matters where the exact gradient vanishes identically
+         (e.g. a single key: P = 1 and dS = P (dP - delta) = 0), so that the
+         GPU's rounding noise (~1e-7) is compared with an absolute bound.
 and every output finite (rows that see no key: O = 0, lse = -inf exactly).
 """
 import numpy as np
@@ -67,7 +70,7 @@ def check_lse(l_gpu, l_ref, what=""):
 def check_grad(g_gpu, g_ref, what=""):
     g = to_np(g_gpu) if isinstance(g_gpu, torch.Tensor) else g_gpu
     assert np.all(np.isfinite(g)), f"{what}: non-finite gradient"
-    scale = max(np.abs(g_ref).max(), 1e-30)
+    scale = max(np.abs(g_ref).max(), 1e-3)
     err = np.abs(g - g_ref).max()
     assert err <= GRAD_REL_MAX * scale, f"{what}: max-abs {err:.3e} > {GRAD_REL_MAX} * {scale:.3e}"
     return float(err / scale)
