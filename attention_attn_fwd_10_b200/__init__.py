@@ -90,8 +90,11 @@ def bwd_workspace_size(B, H_q, S_q, D) -> int:
 
 
 def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, dq=None, dk=None, dv=None,
-        workspace=None, stream=None):
-    """Backward attention.  Returns (dq, dk, dv) bf16 with the shapes of q, k, v."""
+        workspace=None, stream=None, main_pass_events=None):
+    """Backward attention.  Returns (dq, dk, dv) bf16 with the shapes of q, k, v.
+
+    ``main_pass_events``: optional (start, stop) torch.cuda.Event pair recorded
+    around the main-pass kernel (diagnostic timing)."""
     on_host = not q.is_cuda
     if on_host:
         dev = torch.device("cuda", torch.cuda.current_device())
@@ -114,9 +117,12 @@ def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, d
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     if workspace.numel() * workspace.element_size() < need or not workspace.is_cuda:
         raise ValueError(f"workspace must be a CUDA buffer of at least {need} bytes")
-    code = load().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
-                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
-                           B, H_q, H_kv, S_q, S_k, D, int(bool(causal)), scale, _stream_ptr(stream))
+    opt = None
+    if main_pass_events is not None:
+        opt = ctypes.byref(_abi.BwdOptions(main_pass_events[0].cuda_event, main_pass_events[1].cuda_event))
+    code = load().attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                              dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                              B, H_q, H_kv, S_q, S_k, D, int(bool(causal)), scale, opt, _stream_ptr(stream))
     _abi.check(code, "attn_bwd")
     if on_host:
         return dq.cpu(), dk.cpu(), dv.cpu()

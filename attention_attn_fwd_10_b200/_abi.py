@@ -30,6 +30,7 @@ EXPORTED = (
     "attn_fwd_ex",
     "attn_bwd_workspace_size",
     "attn_bwd",
+    "attn_bwd_ex",
     "attn_device_status",
     "attn_set_wait_limit_ns",
     "attn_exp2_poly_eval",
@@ -46,6 +47,12 @@ class FwdOptions(ctypes.Structure):
     ]
 
 
+class BwdOptions(ctypes.Structure):
+    """attn_bwd_options_t"""
+
+    _fields_ = [("main_pass_start", ctypes.c_void_p), ("main_pass_stop", ctypes.c_void_p)]
+
+
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
 _f = ctypes.c_float
@@ -59,6 +66,7 @@ _SIGNATURES = {
                          ctypes.POINTER(FwdOptions), _vp]),
     "attn_bwd_workspace_size": (ctypes.c_size_t, [_i, _i, _i, _i]),
     "attn_bwd": (_i, [_vp] * 10 + [_i, _i, _i, _i, _i, _i, _i, _f, _vp]),
+    "attn_bwd_ex": (_i, [_vp] * 10 + [_i, _i, _i, _i, _i, _i, _i, _f, ctypes.POINTER(BwdOptions), _vp]),
     "attn_device_status": (_i, [_vp]),
     "attn_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
     "attn_exp2_poly_eval": (_i, [_vp, _vp, ctypes.c_longlong, _vp]),

@@ -204,9 +204,10 @@ size_t attn_bwd_workspace_size(int B, int H_q, int S_q, int D) {
   return (dq_acc + 255) / 256 * 256 + 2 * ((rows + 255) / 256 * 256);
 }
 
-attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
-                       void* dq, void* dk, void* dv, void* workspace, int B, int H_q, int H_kv, int S_q, int S_k,
-                       int D, int causal, float scale, void* stream) {
+attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                          const void* dO, void* dq, void* dk, void* dv, void* workspace, int B, int H_q, int H_kv,
+                          int S_q, int S_k, int D, int causal, float scale, const attn_bwd_options_t* opt,
+                          void* stream) {
   attn_status_t st = check_common(B, H_q, H_kv, S_q, S_k, D, causal, scale);
   if (st != ATTN_OK) return st;
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
@@ -257,6 +258,8 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   // 2. main pass
+  if (opt && opt->main_pass_start && cudaEventRecord(static_cast<cudaEvent_t>(opt->main_pass_start), s) != cudaSuccess)
+    return ATTN_ERR_CUDA;
   {
     using L = BwdLayout<128>;
     const unsigned grid = static_cast<unsigned>(p.n_kv_tiles) * B * H_kv;
@@ -279,6 +282,8 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
     err = cudaGetLastError();
     if (err != cudaSuccess) return ATTN_ERR_CUDA;
   }
+  if (opt && opt->main_pass_stop && cudaEventRecord(static_cast<cudaEvent_t>(opt->main_pass_stop), s) != cudaSuccess)
+    return ATTN_ERR_CUDA;
   // 3. dQ convert
   {
     const long long n8 = static_cast<long long>(B) * S_q * H_q * D / 8;
@@ -287,6 +292,13 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
+}
+
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                       void* dq, void* dk, void* dv, void* workspace, int B, int H_q, int H_kv, int S_q, int S_k,
+                       int D, int causal, float scale, void* stream) {
+  return attn_bwd_ex(q, k, v, o, lse, dO, dq, dk, dv, workspace, B, H_q, H_kv, S_q, S_k, D, causal, scale, nullptr,
+                     stream);
 }
 
 attn_status_t attn_device_status(void* stream) {

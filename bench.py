@@ -210,8 +210,9 @@ def run_ours(args):
     def fwd():
         attn.fwd(q, k, v, causal=wf.causal, scale=wf.scale, out=o, lse=lse)
 
-    def bwd():
-        attn.bwd(q, k, v, o, lse, do, causal=wb.causal, scale=wb.scale, dq=dq, dk=dk, dv=dv, workspace=ws)
+    def bwd(events=None):
+        attn.bwd(q, k, v, o, lse, do, causal=wb.causal, scale=wb.scale, dq=dq, dk=dk, dv=dv, workspace=ws,
+                 main_pass_events=events)
 
     for _ in range(args.warmup):
         fwd()
@@ -222,23 +223,25 @@ def run_ours(args):
         raise RuntimeError("device status not OK after warm-up")
 
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    f_ms, b_ms, s_ms = [], [], []
+    f_ms, b_ms, s_ms, m_ms = [], [], [], []
     with ClockSampler(dev.index) as clk:
         for _ in range(args.steps):
             flush.fill_(1)
             barrier(world)
             torch.cuda.synchronize()
-            e0, e1, e2 = ev(), ev(), ev()
+            e0, e1, e2, m0, m1 = ev(), ev(), ev(), ev(), ev()
             e0.record(stream)
             fwd()
             e1.record(stream)
             if have_bwd:
-                bwd()
+                bwd((m0, m1))
             e2.record(stream)
             torch.cuda.synchronize()
             f_ms.append(e0.elapsed_time(e1))
             b_ms.append(e1.elapsed_time(e2))
             s_ms.append(e0.elapsed_time(e2))
+            if have_bwd:
+                m_ms.append(m0.elapsed_time(m1))
         barrier(world)
     clocks = clk.summary()
     if attn.device_status() != 0:
@@ -247,6 +250,7 @@ def run_ours(args):
     step_ms = max_over_ranks(world, sum(s_ms) / len(s_ms))
     fwd_ms = sum(f_ms) / len(f_ms)
     bwd_ms = sum(b_ms) / len(b_ms) if have_bwd else 0.0
+    main_ms = sum(m_ms) / len(m_ms) if have_bwd else 0.0
     flops_step = wf.fwd_flops() + (wb.bwd_flops() if have_bwd else 0.0)
     value = world * flops_step / (step_ms * 1e-3) / 1e12
 
@@ -257,8 +261,8 @@ def run_ours(args):
     fwd_tf = wf.fwd_flops() / (fwd_ms * 1e-3) / 1e12
     bwd_tf = wb.bwd_flops() / (bwd_ms * 1e-3) / 1e12 if have_bwd else None
     # dominant kernel: the one with the larger share of the step
-    if have_bwd and bwd_ms > fwd_ms:
-        dom, dom_flops, dom_ms = "attn_bwd (3 kernels)", wb.bwd_flops(), bwd_ms
+    if have_bwd and main_ms > fwd_ms:
+        dom, dom_flops, dom_ms = "attn_bwd_kernel (main pass)", wb.bwd_flops(), main_ms
     else:
         dom, dom_flops, dom_ms = "attn_fwd_kernel", wf.fwd_flops(), fwd_ms
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
@@ -286,7 +290,7 @@ def run_ours(args):
         "fwd": {"ms": round(fwd_ms, 4), "tflops": round(fwd_tf, 1),
                 "frac_of_spec_2250": round(fwd_tf / SPEC_PEAK_TFLOPS, 4),
                 "frac_of_measured": round(fwd_tf / peak, 4)},
-        "bwd": ({"ms": round(bwd_ms, 4), "tflops": round(bwd_tf, 1),
+        "bwd": ({"ms": round(bwd_ms, 4), "main_pass_ms": round(main_ms, 4), "tflops": round(bwd_tf, 1),
                  "frac_of_spec_2250": round(bwd_tf / SPEC_PEAK_TFLOPS, 4),
                  "frac_of_measured": round(bwd_tf / peak, 4)} if have_bwd else None),
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1),

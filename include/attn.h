@@ -92,7 +92,8 @@ attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, 
 
 /*
  * Bytes of device workspace attn_bwd needs: an fp32 dQ accumulator
- * [B, S_q, H_q, D] and the fp32 row terms delta_i = sum_d dO_id O_id [B, H_q, S_q].
+ * [B, S_q, H_q, D] and two fp32 row-term arrays [B, H_q, S_pad] (S_pad =
+ * S_q rounded up to 64): -lse_i * log2(e) and delta_i = sum_d dO_id O_id.
  * Returns 0 for invalid sizes.
  */
 size_t attn_bwd_workspace_size(int B, int H_q, int S_q, int D);
@@ -103,10 +104,28 @@ size_t attn_bwd_workspace_size(int B, int H_q, int S_q, int D);
  * (bf16).  `workspace` must hold attn_bwd_workspace_size(...) bytes, 16-byte
  * aligned; its contents on entry are ignored.  The dQ accumulation uses atomic
  * fp32 additions, so results may differ in the last bits from run to run.
+ * This build serves D = 128 (other head dims: ATTN_ERR_UNSUPPORTED).
  */
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                        const void* dO, void* dq, void* dk, void* dv, void* workspace, int B, int H_q,
                        int H_kv, int S_q, int S_k, int D, int causal, float scale, void* stream);
+
+/*
+ * Diagnostics of the backward.  main_pass_start / main_pass_stop: optional
+ * cudaEvent_t handles (created by the caller) that the library records on
+ * `stream` immediately before and after the main-pass kernel, so the caller
+ * can time that kernel alone.  NULL = not recorded.
+ */
+typedef struct {
+  void* main_pass_start;
+  void* main_pass_stop;
+} attn_bwd_options_t;
+
+/* attn_bwd with explicit options (`opt` NULL = none). */
+attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                          const void* dO, void* dq, void* dk, void* dv, void* workspace, int B, int H_q,
+                          int H_kv, int S_q, int S_k, int D, int causal, float scale,
+                          const attn_bwd_options_t* opt, void* stream);
 
 /*
  * Synchronises `stream`, then returns and clears the device status word:
