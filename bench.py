@@ -389,6 +389,31 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile(args):
+    """Launch only one pass (--profile fwd|bwd) W + K times on the workload, no
+    timing: the driver for ncu captures of a single kernel."""
+    import torch
+
+    import attention_attn_fwd_10_b200 as attn
+
+    wf, wb = WORKLOADS[args.workload]
+    torch.cuda.set_device(0)
+    x = workloads.make_inputs(wb)
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = attn.fwd(q, k, v, causal=wf.causal, scale=wf.scale)
+    ws = torch.empty(attn.bwd_workspace_size(wb.B, wb.H_q, wb.S_q, wb.D), dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup + args.steps):
+        if args.profile == "fwd":
+            attn.fwd(q, k, v, causal=wf.causal, scale=wf.scale, out=o, lse=lse)
+        else:
+            attn.bwd(q, k, v, o, lse, do, causal=wb.causal, scale=wb.scale, workspace=ws)
+    torch.cuda.synchronize()
+    st = attn.device_status()
+    print(f"profile {args.profile}: {args.warmup + args.steps} launches, device status {st}")
+    if st != 0:
+        sys.exit(1)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -398,7 +423,12 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="causal8k")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU time to sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=("fwd", "bwd"), default=None,
+                    help="only launch one pass W+K times (driver for ncu captures); prints no JSON")
     args = ap.parse_args()
+    if args.profile:
+        run_profile(args)
+        return
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
