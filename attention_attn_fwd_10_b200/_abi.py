@@ -19,6 +19,7 @@ STATUS_NAMES = {
     3: "ATTN_ERR_MISALIGNED",
     4: "ATTN_ERR_CUDA",
     5: "ATTN_ERR_DEVICE_TIMEOUT",
+    6: "ATTN_ERR_SCRATCH_TOO_SMALL",
 }
 
 # Every symbol include/attn.h declares (tests check the library exports all of them).
@@ -31,6 +32,7 @@ EXPORTED = (
     "attn_bwd_workspace_size",
     "attn_bwd",
     "attn_bwd_ex",
+    "attn_bwd_noalloc",
     "attn_device_status",
     "attn_set_wait_limit_ns",
     "attn_exp2_poly_eval",
@@ -67,6 +69,7 @@ _SIGNATURES = {
     "attn_bwd_workspace_size": (ctypes.c_size_t, [_i, _i, _i, _i]),
     "attn_bwd": (_i, [_vp] * 10 + [_i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "attn_bwd_ex": (_i, [_vp] * 10 + [_i, _i, _i, _i, _i, _i, _i, _f, ctypes.POINTER(BwdOptions), _vp]),
+    "attn_bwd_noalloc": (_i, [_vp] * 9 + [_i, _i, _i, _i, _i, _i, _i, _f, _vp]),
     "attn_device_status": (_i, [_vp]),
     "attn_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
     "attn_exp2_poly_eval": (_i, [_vp, _vp, ctypes.c_longlong, _vp]),

@@ -18,6 +18,13 @@ namespace attn {
 // Device status word: kernels record kDevWaitTimeout here when they abandon a wait.
 __device__ int g_status = 0;
 
+// Fixed scratch for attn_bwd_noalloc: every device that loads this library
+// holds these bytes until the process exits.  Host code must not pass the
+// symbol itself to a kernel (on the host it is only a stand-in); it looks up
+// the device address with cudaGetSymbolAddress, once per device.
+constexpr size_t kNoAllocScratchBytes = 32ull << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_bwd_scratch[kNoAllocScratchBytes];
+
 namespace {
 
 constexpr unsigned long long kDefaultWaitLimitNs = 4000000000ull;
@@ -71,6 +78,22 @@ int* status_ptr() {
     ptr_dev = dev;
   }
   return ptr;
+}
+
+// Device address of g_bwd_scratch on the current device (looked up once per device).
+void* noalloc_scratch_ptr() {
+  constexpr int kMaxDevices = 64;
+  static void* ptrs[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) != cudaSuccess) return nullptr;
+    ptrs[dev] = ptr;
+  }
+  return ptrs[dev];
 }
 
 attn_status_t check_common(int B, int H_q, int H_kv, int S_q, int S_k, int D, int causal, float scale) {
@@ -134,6 +157,8 @@ const char* attn_status_string(attn_status_t s) {
     case ATTN_ERR_MISALIGNED: return "ATTN_ERR_MISALIGNED: tensor pointers must be 16-byte aligned";
     case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA: a CUDA call failed";
     case ATTN_ERR_DEVICE_TIMEOUT: return "ATTN_ERR_DEVICE_TIMEOUT: a kernel abandoned a bounded wait";
+    case ATTN_ERR_SCRATCH_TOO_SMALL:
+      return "ATTN_ERR_SCRATCH_TOO_SMALL: the problem needs more scratch than attn_bwd_noalloc's fixed 32 MiB buffer";
   }
   return "ATTN_ERR_UNKNOWN";
 }
@@ -299,6 +324,19 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
                        int D, int causal, float scale, void* stream) {
   return attn_bwd_ex(q, k, v, o, lse, dO, dq, dk, dv, workspace, B, H_q, H_kv, S_q, S_k, D, causal, scale, nullptr,
                      stream);
+}
+
+attn_status_t attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                               const void* dO, void* dq, void* dk, void* dv, int B, int H_q, int H_kv, int S_q,
+                               int S_k, int D, int causal, float scale, void* stream) {
+  attn_status_t st = check_common(B, H_q, H_kv, S_q, S_k, D, causal, scale);
+  if (st != ATTN_OK) return st;
+  const size_t need = attn_bwd_workspace_size(B, H_q, S_q, D);
+  if (need == 0) return ATTN_ERR_INVALID_ARG;
+  if (need > kNoAllocScratchBytes) return ATTN_ERR_SCRATCH_TOO_SMALL;
+  void* scratch = noalloc_scratch_ptr();
+  if (scratch == nullptr) return ATTN_ERR_CUDA;
+  return attn_bwd(q, k, v, o, lse, dO, dq, dk, dv, scratch, B, H_q, H_kv, S_q, S_k, D, causal, scale, stream);
 }
 
 attn_status_t attn_device_status(void* stream) {

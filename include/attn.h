@@ -43,7 +43,8 @@ typedef enum {
   ATTN_ERR_UNSUPPORTED = 2,    /* a valid request this build does not serve (e.g. D not in {64,128}) */
   ATTN_ERR_MISALIGNED = 3,     /* a tensor pointer is not 16-byte aligned */
   ATTN_ERR_CUDA = 4,           /* a CUDA runtime/driver call failed (no device, launch failure ...) */
-  ATTN_ERR_DEVICE_TIMEOUT = 5  /* a kernel abandoned a bounded internal wait (see attn_device_status) */
+  ATTN_ERR_DEVICE_TIMEOUT = 5, /* a kernel abandoned a bounded internal wait (see attn_device_status) */
+  ATTN_ERR_SCRATCH_TOO_SMALL = 6 /* attn_bwd_noalloc: the problem needs more than its fixed scratch */
 } attn_status_t;
 
 /* Version of this ABI (bumped on any incompatible change). */
@@ -126,6 +127,29 @@ attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const voi
                           const void* dO, void* dq, void* dk, void* dv, void* workspace, int B, int H_q,
                           int H_kv, int S_q, int S_k, int D, int causal, float scale,
                           const attn_bwd_options_t* opt, void* stream);
+
+/*
+ * attn_bwd for callers that cannot allocate device memory: the same backward,
+ * with its scratch taken from a buffer built into the library instead of a
+ * caller-provided workspace.  (The pages describe no such variant; it serves
+ * integrations where allocation is not available at the call site -- code that
+ * runs under a framework's memory pool it may not grow, inside a plug-in or a
+ * callback with no allocator handle, or in a latency path that must never
+ * reach cudaMalloc.)
+ *
+ * The buffer is a file-scope device array of 32 MiB (33554432 bytes) that
+ * every GPU which loads the library holds until the process exits.  Problems whose attn_bwd_workspace_size() exceeds it return
+ * ATTN_ERR_SCRATCH_TOO_SMALL before anything is launched.  The first call on a
+ * device looks up the buffer's device address (cudaGetSymbolAddress); make that
+ * first call before any stream capture.  No call allocates or frees device
+ * memory.  All calls share the one buffer and it keeps the last call's
+ * contents (each call clears what must start at zero): calls that may overlap
+ * on the GPU -- on different streams, or from different host threads -- race
+ * on it and must be serialised by the caller.  Arguments and results as attn_bwd.
+ */
+attn_status_t attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                               const void* dO, void* dq, void* dk, void* dv, int B, int H_q, int H_kv,
+                               int S_q, int S_k, int D, int causal, float scale, void* stream);
 
 /*
  * Synchronises `stream`, then returns and clears the device status word:
