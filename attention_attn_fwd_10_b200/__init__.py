@@ -119,6 +119,10 @@ def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, d
         raise ValueError(f"workspace must be a CUDA buffer of at least {need} bytes")
     opt = None
     if main_pass_events is not None:
+        s = torch.cuda.current_stream() if stream is None else stream
+        for e in main_pass_events:
+            if e.cuda_event == 0:  # torch creates the CUDA event lazily, on its first record
+                e.record(s)
         opt = ctypes.byref(_abi.BwdOptions(main_pass_events[0].cuda_event, main_pass_events[1].cuda_event))
     code = load().attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
                               dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
