@@ -62,6 +62,22 @@ bool make_bshd_map(CUtensorMap* map, const void* ptr, int B, int S, int H, int D
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// fp32 [B, S, H, D] dQ accumulator viewed as (D, H, S, B); boxes of D x 1 x 64 x 1
+// (whole 64-query blocks), no swizzle: the target of the backward's TMA reduce-adds.
+bool make_dqacc_map(CUtensorMap* map, void* ptr, int B, int S, int H, int D) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(H) * D * 4,
+                                 static_cast<cuuint64_t>(S) * H * D * 4};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(D), 1, 64, 1};
+  const cuuint32_t estride[4] = {1, 1, 1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ptr, dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int* status_ptr() {
@@ -269,9 +285,10 @@ attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const voi
   p.status = status;
   p.wait_limit_ns = g_wait_limit_ns.load();
 
-  CUtensorMap mk, mv, mq, mdo;
+  CUtensorMap mk, mv, mq, mdo, mdq;
   if (!make_bshd_map(&mk, k, B, S_k, H_kv, D, 128) || !make_bshd_map(&mv, v, B, S_k, H_kv, D, 128) ||
-      !make_bshd_map(&mq, q, B, S_q, H_q, D, 64) || !make_bshd_map(&mdo, dO, B, S_q, H_q, D, 64))
+      !make_bshd_map(&mq, q, B, S_q, H_q, D, 64) || !make_bshd_map(&mdo, dO, B, S_q, H_q, D, 64) ||
+      !make_dqacc_map(&mdq, p.dq_acc, B, S_q, H_q, D))
     return ATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
@@ -295,14 +312,14 @@ attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const voi
       static cudaError_t attr = cudaSuccess;
       std::call_once(once, [&] { attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES); });
       if (attr != cudaSuccess) return ATTN_ERR_CUDA;
-      kern<<<grid, L::THREADS, L::SMEM_BYTES, s>>>(mk, mv, mq, mdo, p);
+      kern<<<grid, L::THREADS, L::SMEM_BYTES, s>>>(mk, mv, mq, mdo, mdq, p);
     } else {
       auto kern = attn_bwd_kernel<128, false>;
       static std::once_flag once;
       static cudaError_t attr = cudaSuccess;
       std::call_once(once, [&] { attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES); });
       if (attr != cudaSuccess) return ATTN_ERR_CUDA;
-      kern<<<grid, L::THREADS, L::SMEM_BYTES, s>>>(mk, mv, mq, mdo, p);
+      kern<<<grid, L::THREADS, L::SMEM_BYTES, s>>>(mk, mv, mq, mdo, mdq, p);
     }
     err = cudaGetLastError();
     if (err != cudaSuccess) return ATTN_ERR_CUDA;

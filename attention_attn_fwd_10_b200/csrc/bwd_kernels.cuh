@@ -13,19 +13,19 @@
 // recomputation).  Per query block, all on tcgen05 with fp32 accumulation:
 //   S^T  = K_j Q_i^T      (128 x 64, TMEM X)     dP^T = V_j dO_i^T   (TMEM Y)
 //   P^T  = 2^(S^T c - lse2_i),  dS^T = P^T o (dP^T - delta_i)     (softmax warpgroup)
-//          P^T (bf16) is written over X and dS^T (bf16) over Y -- the
+//          P^T and dS^T (bf16) are written to their own TMEM columns -- the
 //          intermediates stay in tensor memory (section 7, item 3) -- and
 //          dS^T also goes to shared memory for the dQ product
 //   dV_j += P^T dO_i     (A from TMEM X)         dK_j += dS^T Q_i    (A from TMEM Y)
 //   dQ_i^T = K_j^T dS^T  (128 x 64: both operands MN-major in shared memory)
 // dV_j, dK_j accumulate in TMEM over all query blocks; dQ_i^T goes to one of
-// two TMEM buffers and a second warpgroup adds it into the fp32 dQ
-// accumulator with coalesced atomic adds (the "atomic reductions" of
-// section 7, item 3).  Every MMA has M = 128.
-// Tensor-pipe order per block i: dV_i, dK_i, S^T_{i+1}, dP^T_{i+1}, dQ^T_i, so
-// the softmax of block i+1 overlaps dQ^T_i; S^T_{i+1} / dP^T_{i+1} overwrite
-// P^T_i / dS^T_i after dV_i / dK_i have read them (one issuing thread: the
-// MMAs execute in issue order).
+// two TMEM buffers and a second warpgroup stages it in shared memory and adds
+// it into the fp32 dQ accumulator with one TMA reduce-add per block (the
+// "atomic reductions" of section 7, item 3).  Every MMA has M = 128.
+// Tensor-pipe order per block i: S^T_{i+1}, dP^T_{i+1}, dV_i, dK_i, dQ^T_i, so
+// the softmax of block i+1 overlaps dV_i, dK_i and dQ^T_i.  Barriers: the
+// softmax writes P^T_{i+1}, dS^T_{i+1} only after dV_i, dK_i completed
+// (PD_FREE); dQ^T_{i+1} waits for the dQ warpgroup to have read dQ^T_i.
 //
 // Warp roles (384 threads): warps 0-3 softmax / dS and the dK, dV epilogue
 // (thread = key row = TMEM lane); warps 4-7 dQ reduction (thread = head-dim
@@ -142,27 +142,32 @@ struct BwdLayout {
   static constexpr int STAGE_BYTES = ((2 * Q_TILE + 512 + 1023) / 1024) * 1024;
   static constexpr int DS_OFF = STAGE_OFF + 2 * STAGE_BYTES;  // two dS^T buffers, 128 x 64 bf16
   static constexpr int DS_BYTES = 128 * 64 * 2;
-  static constexpr int BAR_OFF = DS_OFF + 2 * DS_BYTES;
+  static constexpr int DQ_STAGE_OFF = DS_OFF + 2 * DS_BYTES;  // dQ_i staging, fp32 [64 q][D]
+  static constexpr int DQ_STAGE_BYTES = 64 * D * 4;
+  static constexpr int BAR_OFF = DQ_STAGE_OFF + DQ_STAGE_BYTES;
   static constexpr int B_KV_FULL = 0;
   static constexpr int B_QDO_FULL = 1;    // [2]
   static constexpr int B_QDO_EMPTY = 3;   // [2]
-  static constexpr int B_S_FULL = 5;
-  static constexpr int B_DS_READY = 6;    // 128 arrivals
-  static constexpr int B_DQ_FULL = 7;     // [2]
-  static constexpr int B_DQ_FREE = 9;     // [2] 128 arrivals
-  static constexpr int B_D_FINAL = 11;
-  static constexpr int B_DRAIN = 12;
-  static constexpr int N_BARS = 13;
+  static constexpr int B_S_FULL = 5;      // S^T_i and dP^T_i in TMEM
+  static constexpr int B_DS_READY = 6;    // 128 arrivals: P^T_i, dS^T_i written
+  static constexpr int B_PD_FREE = 7;     // dV_i, dK_i have read P^T_i, dS^T_i
+  static constexpr int B_DQ_FULL = 8;     // dQ^T_i in TMEM
+  static constexpr int B_DQ_FREE = 9;     // 128 arrivals: dQ^T_i read out
+  static constexpr int B_D_FINAL = 10;
+  static constexpr int B_DRAIN = 11;
+  static constexpr int N_BARS = 12;
   static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * N_BARS;
   static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 4;
   static constexpr int SMEM_USED = ABORT_OFF + 4;
   static constexpr int SMEM_BYTES = (SMEM_USED + 1024) > 122880 ? (SMEM_USED + 1024) : 122880;
-  // tensor memory columns
-  static constexpr uint32_t X_COL = 0;              // S^T, then P^T (bf16) over its first 32 columns
-  static constexpr uint32_t Y_COL = 64;             // dP^T, then dS^T (bf16)
-  static constexpr uint32_t DV_COL = 128;           // D columns
-  static constexpr uint32_t DK_COL = 128 + D;       // D columns
-  __device__ static constexpr uint32_t dq_col(int b) { return 128 + 2 * D + 64 * b; }
+  // tensor memory columns (512): S^T 64 | dP^T 64 | P^T 32 | dS^T 32 | dV D | dK D | dQ^T 64
+  static constexpr uint32_t X_COL = 0;              // S^T (fp32, 64 query columns)
+  static constexpr uint32_t Y_COL = 64;             // dP^T (fp32)
+  static constexpr uint32_t P_COL = 128;            // P^T (bf16 pairs)
+  static constexpr uint32_t DS_COL = 160;           // dS^T (bf16 pairs)
+  static constexpr uint32_t DV_COL = 192;           // D columns
+  static constexpr uint32_t DK_COL = 192 + D;       // D columns
+  static constexpr uint32_t DQ_COL = 192 + 2 * D;   // 64 columns
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int THREADS = 384;
   static constexpr int WARP_TMA = 8, WARP_MMA = 9;
@@ -173,7 +178,7 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
-                    const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams p) {
   using L = BwdLayout<D>;
   static_assert(D == 128, "the backward main pass is built for D = 128");
   extern __shared__ uint8_t smem_raw[];
@@ -206,7 +211,7 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::N_BARS; ++i)
-      mbar_init(bar(i), (i == L::B_DS_READY || i == L::B_DQ_FREE || i == L::B_DQ_FREE + 1) ? 128u : 1u);
+      mbar_init(bar(i), (i == L::B_DS_READY || i == L::B_DQ_FREE) ? 128u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -299,32 +304,35 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
         const uint32_t sb = sbase + L::STAGE_OFF + st * L::STAGE_BYTES;
         if (!mbar_wait(bar(L::B_DS_READY), i & 1, ctl)) break;
         tc_fence_after();
-        // dV += P^T dO_i ; dK += dS^T Q_i   (16 queries per MMA: 8 TMEM columns, 2048 B of the stage)
-#pragma unroll
-        for (int kk = 0; kk < L::BQ / 16; ++kk)
-          umma_ts(tmem + L::DV_COL, tmem + L::X_COL + kk * 8, sdesc_sw128(sb + L::ST_DO + kk * 2048, L::QBOX_BYTES, 1024),
-                  IDESC_G, (i > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < L::BQ / 16; ++kk)
-          umma_ts(tmem + L::DK_COL, tmem + L::Y_COL + kk * 8, sdesc_sw128(sb + L::ST_Q + kk * 2048, L::QBOX_BYTES, 1024),
-                  IDESC_G, (i > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar(L::B_QDO_EMPTY + st));
+        // the next block's S^T, dP^T first: the softmax warpgroup starts on them while
+        // the tensor pipe runs dV_i, dK_i, dQ^T_i
         if (i + 1 < m) {
           if (!mbar_wait(bar(L::B_QDO_FULL + (st ^ 1)), ((i + 1) >> 1) & 1, ctl)) break;
           tc_fence_after();
           issue_s_dp(st ^ 1);
         }
-        if (i >= 2) {
-          if (!mbar_wait(bar(L::B_DQ_FREE + st), ((i - 2) >> 1) & 1, ctl)) break;
+        // dV += P^T dO_i ; dK += dS^T Q_i   (16 queries per MMA: 8 TMEM columns, 2048 B of the stage)
+#pragma unroll
+        for (int kk = 0; kk < L::BQ / 16; ++kk)
+          umma_ts(tmem + L::DV_COL, tmem + L::P_COL + kk * 8, sdesc_sw128(sb + L::ST_DO + kk * 2048, L::QBOX_BYTES, 1024),
+                  IDESC_G, (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < L::BQ / 16; ++kk)
+          umma_ts(tmem + L::DK_COL, tmem + L::DS_COL + kk * 8, sdesc_sw128(sb + L::ST_Q + kk * 2048, L::QBOX_BYTES, 1024),
+                  IDESC_G, (i > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(L::B_PD_FREE));
+        umma_commit(bar(L::B_QDO_EMPTY + st));
+        if (i >= 1) {
+          if (!mbar_wait(bar(L::B_DQ_FREE), (i - 1) & 1, ctl)) break;
           tc_fence_after();
         }
         // dQ_i^T = K_j^T dS_i^T : 16 keys per MMA = 2048 B of K_j and of dS^T
         const uint32_t ds = sbase + L::DS_OFF + st * L::DS_BYTES;
 #pragma unroll
         for (int kk = 0; kk < L::BN / 16; ++kk)
-          umma_ss(tmem + L::dq_col(st), sdesc_sw128(k_base + kk * 2048, L::KBOX_BYTES, 1024),
+          umma_ss(tmem + L::DQ_COL, sdesc_sw128(k_base + kk * 2048, L::KBOX_BYTES, 1024),
                   sdesc_sw128(ds + kk * 2048, L::DS_BYTES, 1024), IDESC_Q, kk > 0 ? 1u : 0u);
-        umma_commit(bar(L::B_DQ_FULL + st));
+        umma_commit(bar(L::B_DQ_FULL));
       }
       if (ok) umma_commit(bar(L::B_D_FINAL));
       umma_commit(bar(L::B_DRAIN));
@@ -342,8 +350,8 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
     for (int i = 0; i < m; ++i) {
       const int st = i & 1;
       const int q0 = (qb0 + i % per_head) * L::BQ;
+      // S_FULL(i) is committed after dQ^T_{i-2}, so dS^T buffer `st` is free as well.
       ok = mbar_wait(bar(L::B_S_FULL), i & 1, ctl);
-      if (ok && i >= 2) ok = mbar_wait(bar(L::B_DQ_FULL + st), ((i - 2) >> 1) & 1, ctl);  // dS^T buffer free
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       uint32_t sv[64], dp[64];
@@ -355,31 +363,39 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
       tmem_ld_wait(sv + 32);
       tmem_ld_wait(dp);
       tmem_ld_wait(dp + 32);
-      const float* nl = reinterpret_cast<const float*>(sptr + L::STAGE_OFF + st * L::STAGE_BYTES + L::ST_L);
-      const float* dl = reinterpret_cast<const float*>(sptr + L::STAGE_OFF + st * L::STAGE_BYTES + L::ST_DL);
+      const uint8_t* stg = sptr + L::STAGE_OFF + st * L::STAGE_BYTES;
+      const float4* nl4 = reinterpret_cast<const float4*>(stg + L::ST_L);
+      const float4* dl4 = reinterpret_cast<const float4*>(stg + L::ST_DL);
       // causal: key visible to query q0 + c iff c >= key - diag - q0; keys past S_k see nothing
       const int c_first = !valid_key ? L::BQ : (CAUSAL ? key - diag - q0 : 0);
+      const bool masked = __any_sync(0xffffffffu, c_first > 0);
       uint32_t pp[32], pd[32];
 #pragma unroll
-      for (int cp = 0; cp < 32; ++cp) {
-        const float2 nlv = *reinterpret_cast<const float2*>(nl + 2 * cp);
-        const float2 dlv = *reinterpret_cast<const float2*>(dl + 2 * cp);
-        const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[2 * cp]), __uint_as_float(sv[2 * cp + 1])), c2,
-                                   f2_pack(nlv.x, nlv.y));
-        float x0, x1;
-        f2_unpack(x2, x0, x1);
-        float p0 = exp2_mufu(x0), p1 = exp2_mufu(x1);
-        if (2 * cp < c_first) p0 = 0.f;
-        if (2 * cp + 1 < c_first) p1 = 0.f;
-        const uint64_t g2 = f2_sub(f2_pack(__uint_as_float(dp[2 * cp]), __uint_as_float(dp[2 * cp + 1])),
-                                   f2_pack(dlv.x, dlv.y));
-        float d0, d1;
-        f2_unpack(f2_mul(f2_pack(p0, p1), g2), d0, d1);
-        pp[cp] = pack_bf16x2(p0, p1);
-        pd[cp] = pack_bf16x2(d0, d1);
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 nlv = nl4[c4];
+        const float4 dlv = dl4[c4];
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int cp = 2 * c4 + h2;
+          const float na = h2 ? nlv.z : nlv.x, nb = h2 ? nlv.w : nlv.y;
+          const float da = h2 ? dlv.z : dlv.x, db = h2 ? dlv.w : dlv.y;
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[2 * cp]), __uint_as_float(sv[2 * cp + 1])), c2,
+                                     f2_pack(na, nb));
+          float x0, x1;
+          f2_unpack(x2, x0, x1);
+          float p0 = exp2_mufu(x0), p1 = exp2_mufu(x1);
+          if (masked) {
+            if (2 * cp < c_first) p0 = 0.f;
+            if (2 * cp + 1 < c_first) p1 = 0.f;
+          }
+          const uint64_t g2 = f2_sub(f2_pack(__uint_as_float(dp[2 * cp]), __uint_as_float(dp[2 * cp + 1])),
+                                     f2_pack(da, db));
+          float d0, d1;
+          f2_unpack(f2_mul(f2_pack(p0, p1), g2), d0, d1);
+          pp[cp] = pack_bf16x2(p0, p1);
+          pd[cp] = pack_bf16x2(d0, d1);
+        }
       }
-      tmem_st32(tmem + lane_addr + L::X_COL, pp);  // P^T (bf16 pairs)
-      tmem_st32(tmem + lane_addr + L::Y_COL, pd);  // dS^T
       // dS^T row r into the 128B-swizzled MN-major operand: 16-byte chunk c goes to chunk c ^ (r % 8)
       uint8_t* dsrow = sptr + L::DS_OFF + st * L::DS_BYTES + r * 128;
 #pragma unroll
@@ -387,6 +403,13 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
         *reinterpret_cast<uint4*>(dsrow + ((c ^ (r & 7)) << 4)) =
             make_uint4(pd[4 * c], pd[4 * c + 1], pd[4 * c + 2], pd[4 * c + 3]);
       fence_proxy_async_smem();
+      if (i >= 1) {  // dV_{i-1}, dK_{i-1} have read the previous P^T, dS^T
+        ok = mbar_wait(bar(L::B_PD_FREE), (i - 1) & 1, ctl);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+      }
+      tmem_st32(tmem + lane_addr + L::P_COL, pp);
+      tmem_st32(tmem + lane_addr + L::DS_COL, pd);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(L::B_DS_READY));
@@ -428,30 +451,37 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
     }
   } else if (warp < 8) {
     // ===================== dQ reduction warpgroup: thread = head-dim index =====================
+    // dQ_i^T (TMEM) -> fp32 [64 q][D] tile in shared memory -> one TMA reduce-add
+    // into the dQ accumulator (rows past S_q are clipped by the tensor map).
     setmaxnreg_inc<L::REG_MAIN>();
     const int d = threadIdx.x - 128;
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const size_t qstride = static_cast<size_t>(p.H_q) * D;
+    float* stage = reinterpret_cast<float*>(sptr + L::DQ_STAGE_OFF);
     for (int i = 0; i < m; ++i) {
-      const int st = i & 1;
-      bool ok = mbar_wait(bar(L::B_DQ_FULL + st), (i >> 1) & 1, ctl);
+      bool ok = mbar_wait(bar(L::B_DQ_FULL), i & 1, ctl);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       uint32_t v[64];
-      tmem_ld32(tmem + lane_addr + L::dq_col(st), v);
-      tmem_ld32(tmem + lane_addr + L::dq_col(st) + 32, v + 32);
+      tmem_ld32(tmem + lane_addr + L::DQ_COL, v);
+      tmem_ld32(tmem + lane_addr + L::DQ_COL + 32, v + 32);
       tmem_ld_wait(v);
       tmem_ld_wait(v + 32);
       tc_fence_before();
-      mbar_arrive(bar(L::B_DQ_FREE + st));
-      const int h = hkv * G + i / per_head;
-      const int q0 = (qb0 + i % per_head) * L::BQ;
-      float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.S_q + q0) * p.H_q + h) * D + d;
-      const int nq = min(L::BQ, p.S_q - q0);
+      mbar_arrive(bar(L::B_DQ_FREE));
+      if (d == 0) bulk_wait_read_all();  // the previous reduce has read the staging tile
+      named_barrier_sync(1, 128);
 #pragma unroll
-      for (int c = 0; c < L::BQ; ++c)
-        if (c < nq) atomicAdd(dst + c * qstride, __uint_as_float(v[c]));
+      for (int c = 0; c < L::BQ; ++c) stage[c * D + d] = __uint_as_float(v[c]);
+      fence_proxy_async_smem();
+      named_barrier_sync(1, 128);
+      if (d == 0) {
+        const int h = hkv * G + i / per_head;
+        const int q0 = (qb0 + i % per_head) * L::BQ;
+        tma_reduce_add_4d(&tm_dqacc, sbase + L::DQ_STAGE_OFF, 0, h, q0, b);
+        bulk_commit_group();
+      }
     }
+    if (d == 0) bulk_wait_all();
   }
 
   tc_fence_before();
