@@ -136,30 +136,33 @@ struct BwdLayout {
   static constexpr int Q_TILE = 64 * D * 2;
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + KV_TILE;
+  static constexpr int NST = 3;                   // Q/dO ring depth
   static constexpr int STAGE_OFF = V_OFF + KV_TILE;
-  // one stage: Q_i, dO_i, -lse2_i (64 fp32), delta_i (64 fp32); 1024-aligned
-  static constexpr int ST_Q = 0, ST_DO = Q_TILE, ST_L = 2 * Q_TILE, ST_DL = 2 * Q_TILE + 256;
-  static constexpr int STAGE_BYTES = ((2 * Q_TILE + 512 + 1023) / 1024) * 1024;
-  static constexpr int DS_OFF = STAGE_OFF + 2 * STAGE_BYTES;  // two dS^T buffers, 128 x 64 bf16
+  // one stage: Q_i, dO_i (1024-aligned); their -lse2_i and delta_i (64 fp32 each) sit in LD_OFF
+  static constexpr int ST_Q = 0, ST_DO = Q_TILE;
+  static constexpr int STAGE_BYTES = 2 * Q_TILE;
+  static constexpr int DS_OFF = STAGE_OFF + NST * STAGE_BYTES;  // two dS^T buffers, 128 x 64 bf16
   static constexpr int DS_BYTES = 128 * 64 * 2;
   static constexpr int DQ_STAGE_OFF = DS_OFF + 2 * DS_BYTES;  // dQ_i staging, fp32 [64 q][D]
   static constexpr int DQ_STAGE_BYTES = 64 * D * 4;
-  static constexpr int BAR_OFF = DQ_STAGE_OFF + DQ_STAGE_BYTES;
+  static constexpr int LD_OFF = DQ_STAGE_OFF + DQ_STAGE_BYTES;  // per stage: -lse2 (256 B), delta (256 B)
+  static constexpr int BAR_OFF = LD_OFF + NST * 512;
   static constexpr int B_KV_FULL = 0;
-  static constexpr int B_QDO_FULL = 1;    // [2]
-  static constexpr int B_QDO_EMPTY = 3;   // [2]
-  static constexpr int B_S_FULL = 5;      // S^T_i and dP^T_i in TMEM
-  static constexpr int B_DS_READY = 6;    // 128 arrivals: P^T_i, dS^T_i written
-  static constexpr int B_PD_FREE = 7;     // dV_i, dK_i have read P^T_i, dS^T_i
-  static constexpr int B_DQ_FULL = 8;     // dQ^T_i in TMEM
-  static constexpr int B_DQ_FREE = 9;     // 128 arrivals: dQ^T_i read out
-  static constexpr int B_D_FINAL = 10;
-  static constexpr int B_DRAIN = 11;
-  static constexpr int N_BARS = 12;
+  static constexpr int B_QDO_FULL = 1;            // [NST]
+  static constexpr int B_QDO_EMPTY = 1 + NST;     // [NST]
+  static constexpr int B_S_FULL = 1 + 2 * NST;    // S^T_i and dP^T_i in TMEM
+  static constexpr int B_DS_READY = B_S_FULL + 1; // 128 arrivals: P^T_i, dS^T_i written
+  static constexpr int B_PD_FREE = B_S_FULL + 2;  // dV_i, dK_i have read P^T_i, dS^T_i
+  static constexpr int B_DQ_FULL = B_S_FULL + 3;  // dQ^T_i in TMEM
+  static constexpr int B_DQ_FREE = B_S_FULL + 4;  // 128 arrivals: dQ^T_i read out
+  static constexpr int B_D_FINAL = B_S_FULL + 5;
+  static constexpr int B_DRAIN = B_S_FULL + 6;
+  static constexpr int N_BARS = B_S_FULL + 7;
   static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * N_BARS;
   static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 4;
   static constexpr int SMEM_USED = ABORT_OFF + 4;
   static constexpr int SMEM_BYTES = (SMEM_USED + 1024) > 122880 ? (SMEM_USED + 1024) : 122880;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   // tensor memory columns (512): S^T 64 | dP^T 64 | P^T 32 | dS^T 32 | dV D | dK D | dQ^T 64
   static constexpr uint32_t X_COL = 0;              // S^T (fp32, 64 query columns)
   static constexpr uint32_t Y_COL = 64;             // dP^T (fp32)
@@ -243,8 +246,8 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
       }
       int issued = 0;
       for (int i = 0; i < m; ++i) {
-        const int st = i & 1;
-        if (i >= 2 && !mbar_wait(bar(L::B_QDO_EMPTY + st), ((i >> 1) - 1) & 1, ctl)) break;
+        const int st = i % L::NST;
+        if (i >= L::NST && !mbar_wait(bar(L::B_QDO_EMPTY + st), ((i / L::NST) - 1) & 1, ctl)) break;
         const int h = hkv * G + i / per_head;
         const int q0 = (qb0 + i % per_head) * L::BQ;
         const uint32_t sb = sbase + L::STAGE_OFF + st * L::STAGE_BYTES;
@@ -256,13 +259,13 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
           tma_load_4d(sb + L::ST_DO + x * L::QBOX_BYTES, &tm_do, fb, x * 64, h, q0, b);
         }
         const size_t r = (static_cast<size_t>(b) * p.H_q + h) * p.S_pad + q0;
-        bulk_load(sb + L::ST_L, p.nlse2 + r, 256, fb);
-        bulk_load(sb + L::ST_DL, p.delta + r, 256, fb);
+        bulk_load(sbase + L::LD_OFF + st * 512, p.nlse2 + r, 256, fb);
+        bulk_load(sbase + L::LD_OFF + st * 512 + 256, p.delta + r, 256, fb);
         issued = i + 1;
       }
       mbar_wait_drain(bar(L::B_KV_FULL), 0, 1000000000ull);
-      for (int st = 0; st < 2 && st < issued; ++st) {
-        const int uses = (issued - 1 - st) / 2 + 1;
+      for (int st = 0; st < L::NST && st < issued; ++st) {
+        const int uses = (issued - 1 - st) / L::NST + 1;
         mbar_wait_drain(bar(L::B_QDO_FULL + st), (uses - 1) & 1, 1000000000ull);
       }
     }
@@ -300,16 +303,18 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
         }
       }
       for (int i = 0; ok && i < m; ++i) {
-        const int st = i & 1;
+        const int st = i % L::NST;        // Q/dO stage of block i
+        const int st1 = (i + 1) % L::NST;
+        const int db = i & 1;             // dS^T buffer of block i
         const uint32_t sb = sbase + L::STAGE_OFF + st * L::STAGE_BYTES;
         if (!mbar_wait(bar(L::B_DS_READY), i & 1, ctl)) break;
         tc_fence_after();
         // the next block's S^T, dP^T first: the softmax warpgroup starts on them while
         // the tensor pipe runs dV_i, dK_i, dQ^T_i
         if (i + 1 < m) {
-          if (!mbar_wait(bar(L::B_QDO_FULL + (st ^ 1)), ((i + 1) >> 1) & 1, ctl)) break;
+          if (!mbar_wait(bar(L::B_QDO_FULL + st1), ((i + 1) / L::NST) & 1, ctl)) break;
           tc_fence_after();
-          issue_s_dp(st ^ 1);
+          issue_s_dp(st1);
         }
         // dV += P^T dO_i ; dK += dS^T Q_i   (16 queries per MMA: 8 TMEM columns, 2048 B of the stage)
 #pragma unroll
@@ -327,7 +332,7 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
           tc_fence_after();
         }
         // dQ_i^T = K_j^T dS_i^T : 16 keys per MMA = 2048 B of K_j and of dS^T
-        const uint32_t ds = sbase + L::DS_OFF + st * L::DS_BYTES;
+        const uint32_t ds = sbase + L::DS_OFF + db * L::DS_BYTES;
 #pragma unroll
         for (int kk = 0; kk < L::BN / 16; ++kk)
           umma_ss(tmem + L::DQ_COL, sdesc_sw128(k_base + kk * 2048, L::KBOX_BYTES, 1024),
@@ -348,9 +353,10 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
     const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int i = 0; i < m; ++i) {
-      const int st = i & 1;
+      const int st = i % L::NST;  // Q/dO stage (its -lse2, delta)
+      const int db = i & 1;       // dS^T buffer
       const int q0 = (qb0 + i % per_head) * L::BQ;
-      // S_FULL(i) is committed after dQ^T_{i-2}, so dS^T buffer `st` is free as well.
+      // S_FULL(i) is committed after dQ^T_{i-2}, so dS^T buffer `db` is free as well.
       ok = mbar_wait(bar(L::B_S_FULL), i & 1, ctl);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
@@ -363,9 +369,8 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
       tmem_ld_wait(sv + 32);
       tmem_ld_wait(dp);
       tmem_ld_wait(dp + 32);
-      const uint8_t* stg = sptr + L::STAGE_OFF + st * L::STAGE_BYTES;
-      const float4* nl4 = reinterpret_cast<const float4*>(stg + L::ST_L);
-      const float4* dl4 = reinterpret_cast<const float4*>(stg + L::ST_DL);
+      const float4* nl4 = reinterpret_cast<const float4*>(sptr + L::LD_OFF + st * 512);
+      const float4* dl4 = reinterpret_cast<const float4*>(sptr + L::LD_OFF + st * 512 + 256);
       // causal: key visible to query q0 + c iff c >= key - diag - q0; keys past S_k see nothing
       const int c_first = !valid_key ? L::BQ : (CAUSAL ? key - diag - q0 : 0);
       const bool masked = __any_sync(0xffffffffu, c_first > 0);
@@ -397,7 +402,7 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
         }
       }
       // dS^T row r into the 128B-swizzled MN-major operand: 16-byte chunk c goes to chunk c ^ (r % 8)
-      uint8_t* dsrow = sptr + L::DS_OFF + st * L::DS_BYTES + r * 128;
+      uint8_t* dsrow = sptr + L::DS_OFF + db * L::DS_BYTES + r * 128;
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         *reinterpret_cast<uint4*>(dsrow + ((c ^ (r & 7)) << 4)) =
