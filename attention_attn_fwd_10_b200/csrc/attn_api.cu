@@ -150,10 +150,19 @@ cudaError_t launch_fwd_poly(int poly, const CUtensorMap& mq, const CUtensorMap& 
   }
 }
 
+// Evaluates the kernels' packed-pair cubic on x[2i], x[2i+1] (the last element of
+// an odd-length array is paired with itself).
 __global__ void exp2_poly_eval_kernel(const float* x, float* y, long long n) {
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<long long>(gridDim.x) * blockDim.x)
-    y[i] = exp2_poly(x[i]);
+  const long long pairs = (n + 1) / 2;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < pairs;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float a = x[2 * i];
+    const float b = 2 * i + 1 < n ? x[2 * i + 1] : a;
+    float ea, eb;
+    exp2_poly_x2(f2_pack(a, b), ea, eb);
+    y[2 * i] = ea;
+    if (2 * i + 1 < n) y[2 * i + 1] = eb;
+  }
 }
 
 }  // namespace

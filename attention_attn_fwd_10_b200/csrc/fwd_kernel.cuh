@@ -5,9 +5,13 @@
 // each K_j / V_j block is loaded once and used by both tiles.  Warp roles:
 //   warps 0-3   softmax warpgroup of tile A (thread t owns row t: TMEM lane t)
 //   warps 4-7   softmax warpgroup of tile B
-//   warp  8     TMA producer: Q_A, Q_B once, then K_j / V_j into a 2-stage ring
+//   warp  8     TMA producer: Q_A, Q_B once, then K_j into a 3-stage ring
 //   warp  9     TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 10-11 idle (they complete the third warpgroup)
+//   warp  10    TMA producer: V_j into a 2-stage ring
+//   warp  11    idle (it completes the third warpgroup)
+// K_j is released as soon as both tiles' S(j) have completed and V_j once both
+// PV(j) have, so the next loads start a full MMA group earlier than with a
+// shared K/V stage.
 // Tensor memory (32-bit columns): S_A, S_B (128 x 128 fp32 scores each),
 // O_A, O_B (128 x D fp32).  The softmax writes P_t (bf16, two per column)
 // over the first 64 columns of S_t, and the PV MMA reads it from there.
@@ -54,20 +58,22 @@ struct FwdLayout {
   static constexpr int BM = 128;                 // query rows per tile
   static constexpr int UNIT = 256;               // query rows per work unit (two tiles)
   static constexpr int BN = 128;                 // keys per block
-  static constexpr int STAGES = 2;               // K/V ring depth
+  static constexpr int KST = 3;                  // K ring depth (released after the last S MMA of a block)
+  static constexpr int VST = 2;                  // V ring depth (released after the last PV MMA of a block)
   static constexpr int NBOX = D / 64;            // 64-element (128 B) TMA boxes per row block
   static constexpr int BOX_BYTES = 128 * 128;    // one 128 x 64 bf16 box
   static constexpr int TILE_BYTES = 128 * D * 2; // one 128 x D bf16 tile
   static constexpr int Q_OFF = 0;                // two Q tiles
   static constexpr int K_OFF = Q_OFF + 2 * TILE_BYTES;
-  static constexpr int V_OFF = K_OFF + STAGES * TILE_BYTES;
-  static constexpr int BAR_OFF = V_OFF + STAGES * TILE_BYTES;
+  static constexpr int V_OFF = K_OFF + KST * TILE_BYTES;
+  static constexpr int BAR_OFF = V_OFF + VST * TILE_BYTES;
   // barrier slots (8 bytes each); [t] = per Q tile, [s] = per ring stage
   static constexpr int B_Q_FULL = 0;                    // [t]
-  static constexpr int B_K_FULL = B_Q_FULL + 2;         // [s]
-  static constexpr int B_V_FULL = B_K_FULL + STAGES;    // [s]
-  static constexpr int B_KV_EMPTY = B_V_FULL + STAGES;  // [s]
-  static constexpr int B_S_FULL = B_KV_EMPTY + STAGES;  // [t]
+  static constexpr int B_K_FULL = B_Q_FULL + 2;        // [ks]
+  static constexpr int B_K_EMPTY = B_K_FULL + KST;     // [ks]
+  static constexpr int B_V_FULL = B_K_EMPTY + KST;     // [vs]
+  static constexpr int B_V_EMPTY = B_V_FULL + VST;     // [vs]
+  static constexpr int B_S_FULL = B_V_EMPTY + VST;     // [t]
   static constexpr int B_P_FULL = B_S_FULL + 2;         // [t]  (128 arrivals)
   static constexpr int B_PV_DONE = B_P_FULL + 2;        // [t]
   static constexpr int B_O_FINAL = B_PV_DONE + 2;       // [t]
@@ -79,12 +85,13 @@ struct FwdLayout {
   // 1 KiB of slack to align the base to 1024 bytes (128-byte swizzle atoms);
   // at least 120 KiB so a single CTA occupies an SM (its TMEM request is 512 columns).
   static constexpr int SMEM_BYTES = (SMEM_USED + 1024) > 122880 ? (SMEM_USED + 1024) : 122880;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   // tensor memory columns
   __device__ static constexpr uint32_t s_col(int t) { return static_cast<uint32_t>(t) * 128u; }
   __device__ static constexpr uint32_t o_col(int t) { return 256u + static_cast<uint32_t>(t) * D; }
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int THREADS = 384;
-  static constexpr int WARP_TMA = 8, WARP_MMA = 9;
+  static constexpr int WARP_TMA = 8, WARP_MMA = 9, WARP_TMA_V = 10;
   // Register split: launched at 168 per thread (384 x 168 = 64512); the two
   // softmax warpgroups grow to 216 and the third shrinks to 72:
   // 2 x 128 x 216 + 128 x 72 = 64512, exactly the launch's total.
@@ -104,12 +111,12 @@ __device__ __forceinline__ float exp_block(const uint32_t* sr, float c, float m,
 #pragma unroll
   for (int cp = 0; cp < 64; ++cp) {
     const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[2 * cp]), __uint_as_float(sr[2 * cp + 1])), c2, nm2);
-    float x0, x1, e0, e1;
-    f2_unpack(x2, x0, x1);
+    float e0, e1;
     if (POLY_EVERY > 0 && (cp % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1) {
-      e0 = exp2_poly(x0);
-      e1 = exp2_poly(x1);
+      exp2_poly_x2(x2, e0, e1);
     } else {
+      float x0, x1;
+      f2_unpack(x2, x0, x1);
       e0 = exp2_mufu(x0);
       e1 = exp2_mufu(x1);
     }
@@ -204,7 +211,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
     setmaxnreg_dec<L::REG_OTHER>();
   }
   if (warp == L::WARP_TMA) {
-    // ===================== TMA producer =====================
+    // ===================== TMA producer: Q, K =====================
     if (lane == 0 && n_blocks > 0) {
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
@@ -217,13 +224,28 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       }
       int issued = 0;
       for (int j = 0; j < n_blocks; ++j) {
-        const int s = j % L::STAGES;
-        if (j >= L::STAGES && !mbar_wait(bar(L::B_KV_EMPTY + s), ((j / L::STAGES) - 1) & 1, ctl)) break;
+        const int s = j % L::KST;
+        if (j >= L::KST && !mbar_wait(bar(L::B_K_EMPTY + s), ((j / L::KST) - 1) & 1, ctl)) break;
         mbar_arrive_expect_tx(bar(L::B_K_FULL + s), L::TILE_BYTES);
 #pragma unroll
         for (int x = 0; x < L::NBOX; ++x)
           tma_load_4d(sbase + L::K_OFF + s * L::TILE_BYTES + x * L::BOX_BYTES, &tm_k, bar(L::B_K_FULL + s),
                       x * 64, hkv, j * L::BN, b);
+        issued = j + 1;
+      }
+      // Drain: every load this thread issued has landed before the CTA may exit.
+      for (int t = 0; t < 2; ++t)
+        if (nblk[t] > 0) mbar_wait_drain(bar(L::B_Q_FULL + t), 0, 1000000000ull);
+      for (int s = 0; s < L::KST && s < issued; ++s)
+        mbar_wait_drain(bar(L::B_K_FULL + s), ((issued - 1 - s) / L::KST) & 1, 1000000000ull);
+    }
+  } else if (warp == L::WARP_TMA_V) {
+    // ===================== TMA producer: V =====================
+    if (lane == 0 && n_blocks > 0) {
+      int issued = 0;
+      for (int j = 0; j < n_blocks; ++j) {
+        const int s = j % L::VST;
+        if (j >= L::VST && !mbar_wait(bar(L::B_V_EMPTY + s), ((j / L::VST) - 1) & 1, ctl)) break;
         mbar_arrive_expect_tx(bar(L::B_V_FULL + s), L::TILE_BYTES);
 #pragma unroll
         for (int x = 0; x < L::NBOX; ++x)
@@ -231,14 +253,8 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
                       x * 64, hkv, j * L::BN, b);
         issued = j + 1;
       }
-      // Drain: every load this thread issued has landed before the CTA may exit.
-      for (int t = 0; t < 2; ++t)
-        if (nblk[t] > 0) mbar_wait_drain(bar(L::B_Q_FULL + t), 0, 1000000000ull);
-      for (int s = 0; s < L::STAGES && s < issued; ++s) {
-        const int uses = (issued - 1 - s) / L::STAGES + 1;
-        mbar_wait_drain(bar(L::B_K_FULL + s), (uses - 1) & 1, 1000000000ull);
-        mbar_wait_drain(bar(L::B_V_FULL + s), (uses - 1) & 1, 1000000000ull);
-      }
+      for (int s = 0; s < L::VST && s < issued; ++s)
+        mbar_wait_drain(bar(L::B_V_FULL + s), ((issued - 1 - s) / L::VST) & 1, 1000000000ull);
     }
   } else if (warp == L::WARP_MMA) {
     // ===================== MMA issuer =====================
@@ -277,14 +293,15 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
           issue_s(t, 0);
         }
       }
+      if (ok) umma_commit(bar(L::B_K_EMPTY));  // K_0 released once both S(0) complete
       // Per key block j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1).  S_t(j+1) overwrites
       // P_t(j), which PV_t(j) reads: the MMAs of this one issuing thread execute
       // in issue order, so PV_t(j) has read P_t(j) before S_t(j+1) writes there
       // (ATTN_FWD_PV_WAIT=1 makes the issuer wait for PV_t(j) to complete instead).
       for (int j = 0; ok && j < n_blocks; ++j) {
-        const int s = j % L::STAGES;
-        const int s1 = (j + 1) % L::STAGES;
-        if (!mbar_wait(bar(L::B_V_FULL + s), (j / L::STAGES) & 1, ctl)) break;
+        const int vs = j % L::VST;
+        const int ks1 = (j + 1) % L::KST;
+        if (!mbar_wait(bar(L::B_V_FULL + vs), (j / L::VST) & 1, ctl)) break;
         bool k_next_ready = false;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
@@ -292,11 +309,11 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
           ok = mbar_wait(bar(L::B_P_FULL + t), j & 1, ctl);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(t, s, j > 0);
+          issue_pv(t, vs, j > 0);
           if (j == nblk[t] - 1) umma_commit(bar(L::B_O_FINAL + t));
           if (j + 1 < nblk[t]) {
             if (!k_next_ready) {
-              ok = mbar_wait(bar(L::B_K_FULL + s1), ((j + 1) / L::STAGES) & 1, ctl);
+              ok = mbar_wait(bar(L::B_K_FULL + ks1), ((j + 1) / L::KST) & 1, ctl);
               if (!ok) break;
               k_next_ready = true;
             }
@@ -305,11 +322,12 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
             if (!ok) break;
             tc_fence_after();
 #endif
-            issue_s(t, s1);
+            issue_s(t, ks1);
           }
         }
         if (!ok) break;
-        umma_commit(bar(L::B_KV_EMPTY + s));
+        umma_commit(bar(L::B_V_EMPTY + vs));
+        if (k_next_ready) umma_commit(bar(L::B_K_EMPTY + ks1));
       }
       // Drain: no MMA may still be writing TMEM when it is released.
       umma_commit(bar(L::B_DRAIN));

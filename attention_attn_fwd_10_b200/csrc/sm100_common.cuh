@@ -365,6 +365,27 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
+// The same cubic on a packed pair (two lanes of work per f32x2 instruction):
+// clamp (two scalar max), floor via add.rm against 1.5*2^23, exact reduction,
+// Horner in fma.f32x2, then the exponent-field add per lane.
+__device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float& e0, float& e1) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  const uint64_t xc = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
+  uint64_t t;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(t) : "l"(xc), "l"(magic));
+  const uint64_t f = f2_sub(xc, f2_sub(t, magic));
+  uint64_t p = f2_fma(f2_pack(kExp2C3, kExp2C3), f, f2_pack(kExp2C2, kExp2C2));
+  p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
+  p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  e0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  e1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 // Pack two floats into bf16x2 (round to nearest even): lo -> bits [0,16).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
