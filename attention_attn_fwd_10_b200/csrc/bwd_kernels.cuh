@@ -157,7 +157,8 @@ struct BwdLayout {
   static constexpr int B_DQ_FREE = B_S_FULL + 4;  // 128 arrivals: dQ^T_i read out
   static constexpr int B_D_FINAL = B_S_FULL + 5;
   static constexpr int B_DRAIN = B_S_FULL + 6;
-  static constexpr int N_BARS = B_S_FULL + 7;
+  static constexpr int B_DQ_WG = B_S_FULL + 7;    // 128 arrivals: barrier among the dQ warpgroup
+  static constexpr int N_BARS = B_S_FULL + 8;
   static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * N_BARS;
   static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 4;
   static constexpr int SMEM_USED = ABORT_OFF + 4;
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::N_BARS; ++i)
-      mbar_init(bar(i), (i == L::B_DS_READY || i == L::B_DQ_FREE) ? 128u : 1u);
+      mbar_init(bar(i), (i == L::B_DS_READY || i == L::B_DQ_FREE || i == L::B_DQ_WG) ? 128u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -462,6 +463,15 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
     const int d = threadIdx.x - 128;
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     float* stage = reinterpret_cast<float*>(sptr + L::DQ_STAGE_OFF);
+    // Barrier among the 128 threads of this warpgroup built on an mbarrier, so
+    // that every wait is bounded (a warp that gave up cannot strand the others).
+    uint32_t wg_phase = 0;
+    auto wg_sync = [&]() -> bool {
+      mbar_arrive(bar(L::B_DQ_WG));
+      const bool r = mbar_wait(bar(L::B_DQ_WG), wg_phase & 1, ctl);
+      ++wg_phase;
+      return __all_sync(0xffffffffu, r);
+    };
     for (int i = 0; i < m; ++i) {
       bool ok = mbar_wait(bar(L::B_DQ_FULL), i & 1, ctl);
       if (!__all_sync(0xffffffffu, ok)) break;
@@ -474,11 +484,11 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
       tc_fence_before();
       mbar_arrive(bar(L::B_DQ_FREE));
       if (d == 0) bulk_wait_read_all();  // the previous reduce has read the staging tile
-      named_barrier_sync(1, 128);
+      if (!wg_sync()) break;
 #pragma unroll
       for (int c = 0; c < L::BQ; ++c) stage[c * D + d] = __uint_as_float(v[c]);
       fence_proxy_async_smem();
-      named_barrier_sync(1, 128);
+      if (!wg_sync()) break;
       if (d == 0) {
         const int h = hkv * G + i / per_head;
         const int q0 = (qb0 + i % per_head) * L::BQ;
