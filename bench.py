@@ -142,15 +142,21 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(world, x: float) -> float:
+def max_over_ranks(world, x: float, device: str = "cuda") -> float:
+    """The slowest rank's value (every rank takes part; NCCL on GPUs, gloo on CPU)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_throughput(world: int, flops_per_rank_step: float, step_ms_max: float) -> float:
+    """Whole-job TFLOPS of N independent replicas: all ranks' work / slowest rank's time."""
+    return world * flops_per_rank_step / (step_ms_max * 1e-3) / 1e12
 
 
 # --------------------------------------------------------------------------- oracle (CPU) timing
@@ -252,7 +258,7 @@ def run_ours(args):
     bwd_ms = sum(b_ms) / len(b_ms) if have_bwd else 0.0
     main_ms = sum(m_ms) / len(m_ms) if have_bwd else 0.0
     flops_step = wf.fwd_flops() + (wb.bwd_flops() if have_bwd else 0.0)
-    value = world * flops_step / (step_ms * 1e-3) / 1e12
+    value = replica_throughput(world, flops_step, step_ms)
 
     # end to end through the public API with pinned host buffers
     e2e = run_e2e(args, attn, x, wf, wb, have_bwd, dev, world)
