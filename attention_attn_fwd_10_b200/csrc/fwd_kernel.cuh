@@ -6,20 +6,20 @@
 //   warps 0-3   softmax warpgroup of tile A (thread t owns row t: TMEM lane t)
 //   warps 4-7   softmax warpgroup of tile B
 //   warp  8     TMA producer: Q_A, Q_B once, then K_j into a 3-stage ring
-//   warp  9     TMEM allocator; its lane 0 issues tile A's tcgen05.mma
+//   warp  9     TMEM allocator and single-thread tcgen05.mma issuer
 //   warp  10    TMA producer: V_j into a 2-stage ring
-//   warp  11    lane 0 issues tile B's tcgen05.mma
+//   warp  11    idle (it completes the third warpgroup)
 // K_j is released as soon as both tiles' S(j) have completed and V_j once both
 // PV(j) have, so the next loads start a full MMA group earlier than with a
 // shared K/V stage.
 // Tensor memory (32-bit columns): S_A, S_B (128 x 128 fp32 scores each),
 // O_A, O_B (128 x D fp32).  The softmax writes P_t (bf16, two per column)
 // over the first 64 columns of S_t, and the PV MMA reads it from there.
-// Each tile's issuer sends, per key block j, PV_t(j) then S_t(j+1) (which
-// overwrites P_t(j) after PV_t(j) has read it: one thread's MMAs execute in
-// issue order).  While one tile's softmax runs, the tensor pipe works on the
-// other tile's MMAs: the fully asynchronous MMA pipeline with softmax/MMA
-// overlap of FlashAttention-4 ("AI Infra series ch. 6, GPU performance engineering (II)",
+// Tensor-pipe issue order per key block j:  PV_A(j), PV_B(j), S_A(j+1),
+// S_B(j+1); S_t(j+1) is issued only once PV_t(j) has completed (it overwrites
+// P_t(j)).  While one tile's softmax runs, the tensor pipe works on the other
+// tile's MMAs: the fully asynchronous MMA pipeline with softmax/MMA overlap of
+// FlashAttention-4 ("AI Infra series ch. 6, GPU performance engineering (II)",
 // section 7; "NVIDIA's strongest B200 wastes 60%", second move).
 //
 // Softmax (per row, base-2 units t = s * scale * log2 e):
@@ -70,10 +70,10 @@ struct FwdLayout {
   // barrier slots (8 bytes each); [t] = per Q tile, [s] = per ring stage
   static constexpr int B_Q_FULL = 0;                    // [t]
   static constexpr int B_K_FULL = B_Q_FULL + 2;        // [ks]
-  static constexpr int B_K_EMPTY = B_K_FULL + KST;     // [t][ks]: tile t is done with the slot
-  static constexpr int B_V_FULL = B_K_EMPTY + 2 * KST; // [vs]
-  static constexpr int B_V_EMPTY = B_V_FULL + VST;     // [t][vs]
-  static constexpr int B_S_FULL = B_V_EMPTY + 2 * VST; // [t]
+  static constexpr int B_K_EMPTY = B_K_FULL + KST;     // [ks]
+  static constexpr int B_V_FULL = B_K_EMPTY + KST;     // [vs]
+  static constexpr int B_V_EMPTY = B_V_FULL + VST;     // [vs]
+  static constexpr int B_S_FULL = B_V_EMPTY + VST;     // [t]
   static constexpr int B_P_FULL = B_S_FULL + 2;         // [t]  (128 arrivals)
   static constexpr int B_PV_DONE = B_P_FULL + 2;        // [t]
   static constexpr int B_O_FINAL = B_PV_DONE + 2;       // [t]
@@ -91,7 +91,7 @@ struct FwdLayout {
   __device__ static constexpr uint32_t o_col(int t) { return 256u + static_cast<uint32_t>(t) * D; }
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int THREADS = 384;
-  static constexpr int WARP_TMA = 8, WARP_MMA = 9, WARP_TMA_V = 10, WARP_MMA_B = 11;
+  static constexpr int WARP_TMA = 8, WARP_MMA = 9, WARP_TMA_V = 10;
   // Register split: launched at 168 per thread (384 x 168 = 64512); the two
   // softmax warpgroups grow to 216 and the third shrinks to 72:
   // 2 x 128 x 216 + 128 x 72 = 64512, exactly the launch's total.
@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
   // ---- setup
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::N_BARS; ++i)
-      mbar_init(bar(i), (i == L::B_P_FULL || i == L::B_P_FULL + 1) ? 128u : (i == L::B_DRAIN ? 2u : 1u));
+      mbar_init(bar(i), (i == L::B_P_FULL || i == L::B_P_FULL + 1) ? 128u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -225,12 +225,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       int issued = 0;
       for (int j = 0; j < n_blocks; ++j) {
         const int s = j % L::KST;
-        bool free_ok = true;
-#pragma unroll
-        for (int t = 0; t < 2; ++t)  // every tile that used the slot's previous block has released it
-          if (free_ok && j >= L::KST && j - L::KST < nblk[t])
-            free_ok = mbar_wait(bar(L::B_K_EMPTY + t * L::KST + s), ((j / L::KST) - 1) & 1, ctl);
-        if (!free_ok) break;
+        if (j >= L::KST && !mbar_wait(bar(L::B_K_EMPTY + s), ((j / L::KST) - 1) & 1, ctl)) break;
         mbar_arrive_expect_tx(bar(L::B_K_FULL + s), L::TILE_BYTES);
 #pragma unroll
         for (int x = 0; x < L::NBOX; ++x)
@@ -250,12 +245,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       int issued = 0;
       for (int j = 0; j < n_blocks; ++j) {
         const int s = j % L::VST;
-        bool free_ok = true;
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-          if (free_ok && j >= L::VST && j - L::VST < nblk[t])
-            free_ok = mbar_wait(bar(L::B_V_EMPTY + t * L::VST + s), ((j / L::VST) - 1) & 1, ctl);
-        if (!free_ok) break;
+        if (j >= L::VST && !mbar_wait(bar(L::B_V_EMPTY + s), ((j / L::VST) - 1) & 1, ctl)) break;
         mbar_arrive_expect_tx(bar(L::B_V_FULL + s), L::TILE_BYTES);
 #pragma unroll
         for (int x = 0; x < L::NBOX; ++x)
@@ -266,20 +256,13 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       for (int s = 0; s < L::VST && s < issued; ++s)
         mbar_wait_drain(bar(L::B_V_FULL + s), ((issued - 1 - s) / L::VST) & 1, 1000000000ull);
     }
-  } else if (warp == L::WARP_MMA || warp == L::WARP_MMA_B) {
-    // ===================== MMA issuers: one thread per Q tile =====================
-    // Tile A's MMAs are issued by warp 9, tile B's by warp 11.  An issuing thread
-    // blocks in tcgen05.mma while the tensor pipe works, so with one issuer per
-    // tile one tile's waits overlap the other tile's issue and the pipe stays fed.
-    // Each thread releases the K and V slots its own tile used (per-tile empty
-    // barriers); the producers wait for every tile that used a slot's previous block.
-    const int t = warp == L::WARP_MMA ? 0 : 1;
+  } else if (warp == L::WARP_MMA) {
+    // ===================== MMA issuer =====================
     if (lane == 0 && n_blocks > 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
-      const int nb = nblk[t];
-      const uint32_t q_base = sbase + L::Q_OFF + t * L::TILE_BYTES;
-      auto issue_s = [&](int stage) {
+      auto issue_s = [&](int t, int stage) {
+        const uint32_t q_base = sbase + L::Q_OFF + t * L::TILE_BYTES;
         const uint32_t k_base = sbase + L::K_OFF + stage * L::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -289,7 +272,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
         }
         umma_commit(bar(L::B_S_FULL + t));
       };
-      auto issue_pv = [&](int stage, bool acc) {
+      auto issue_pv = [&](int t, int stage, bool acc) {
         const uint32_t v_base = sbase + L::V_OFF + stage * L::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < L::BN / 16; ++kk) {
@@ -301,39 +284,50 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
         umma_commit(bar(L::B_PV_DONE + t));
 #endif
       };
-      bool ok = true;
-      if (nb > 0) {
-        ok = mbar_wait(bar(L::B_K_FULL), 0, ctl) && mbar_wait(bar(L::B_Q_FULL + t), 0, ctl);
+      bool ok = mbar_wait(bar(L::B_K_FULL), 0, ctl);
+      for (int t = 0; ok && t < 2; ++t) {
+        if (nblk[t] == 0) continue;
+        ok = mbar_wait(bar(L::B_Q_FULL + t), 0, ctl);
         if (ok) {
           tc_fence_after();
-          issue_s(0);
+          issue_s(t, 0);
         }
       }
-      if (ok && nb > 0) umma_commit(bar(L::B_K_EMPTY + t * L::KST));  // done with K_0 once S_t(0) completes
-      // Per key block j: PV_t(j), then S_t(j+1).  S_t(j+1) overwrites P_t(j),
-      // which PV_t(j) reads: the MMAs of one issuing thread execute in issue
-      // order, so PV_t(j) has read P_t(j) before S_t(j+1) writes there
+      if (ok) umma_commit(bar(L::B_K_EMPTY));  // K_0 released once both S(0) complete
+      // Per key block j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1).  S_t(j+1) overwrites
+      // P_t(j), which PV_t(j) reads: the MMAs of this one issuing thread execute
+      // in issue order, so PV_t(j) has read P_t(j) before S_t(j+1) writes there
       // (ATTN_FWD_PV_WAIT=1 makes the issuer wait for PV_t(j) to complete instead).
       for (int j = 0; ok && j < n_blocks; ++j) {
         const int vs = j % L::VST;
         const int ks1 = (j + 1) % L::KST;
-        if (j < nb) {
-          if (!mbar_wait(bar(L::B_V_FULL + vs), (j / L::VST) & 1, ctl)) break;
-          if (!mbar_wait(bar(L::B_P_FULL + t), j & 1, ctl)) break;
+        if (!mbar_wait(bar(L::B_V_FULL + vs), (j / L::VST) & 1, ctl)) break;
+        bool k_next_ready = false;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (!ok || j >= nblk[t]) continue;
+          ok = mbar_wait(bar(L::B_P_FULL + t), j & 1, ctl);
+          if (!ok) break;
           tc_fence_after();
-          issue_pv(vs, j > 0);
-          if (j == nb - 1) umma_commit(bar(L::B_O_FINAL + t));
-          if (j + 1 < nb) {
-            if (!mbar_wait(bar(L::B_K_FULL + ks1), ((j + 1) / L::KST) & 1, ctl)) break;
+          issue_pv(t, vs, j > 0);
+          if (j == nblk[t] - 1) umma_commit(bar(L::B_O_FINAL + t));
+          if (j + 1 < nblk[t]) {
+            if (!k_next_ready) {
+              ok = mbar_wait(bar(L::B_K_FULL + ks1), ((j + 1) / L::KST) & 1, ctl);
+              if (!ok) break;
+              k_next_ready = true;
+            }
 #if ATTN_FWD_PV_WAIT
-            if (!mbar_wait(bar(L::B_PV_DONE + t), j & 1, ctl)) break;
+            ok = mbar_wait(bar(L::B_PV_DONE + t), j & 1, ctl);
+            if (!ok) break;
             tc_fence_after();
 #endif
-            issue_s(ks1);
-            umma_commit(bar(L::B_K_EMPTY + t * L::KST + ks1));
+            issue_s(t, ks1);
           }
-          umma_commit(bar(L::B_V_EMPTY + t * L::VST + vs));
         }
+        if (!ok) break;
+        umma_commit(bar(L::B_V_EMPTY + vs));
+        if (k_next_ready) umma_commit(bar(L::B_K_EMPTY + ks1));
       }
       // Drain: no MMA may still be writing TMEM when it is released.
       umma_commit(bar(L::B_DRAIN));
