@@ -74,8 +74,8 @@ struct FwdLayout {
   static constexpr int B_V_FULL = B_K_EMPTY + KST;     // [vs]
   static constexpr int B_V_EMPTY = B_V_FULL + VST;     // [vs]
   static constexpr int B_S_FULL = B_V_EMPTY + VST;     // [t]
-  static constexpr int B_P_FULL = B_S_FULL + 2;         // [t]  (128 arrivals)
-  static constexpr int B_PV_DONE = B_P_FULL + 2;        // [t]
+  static constexpr int B_P_FULL = B_S_FULL + 2;         // [t][half]  (128 arrivals)
+  static constexpr int B_PV_DONE = B_P_FULL + 4;        // [t]
   static constexpr int B_O_FINAL = B_PV_DONE + 2;       // [t]
   static constexpr int B_DRAIN = B_O_FINAL + 2;
   static constexpr int N_BARS = B_DRAIN + 1;
@@ -102,26 +102,26 @@ struct FwdLayout {
 // the fp32 sum of the unrounded p.  Column pair cp (columns 2cp, 2cp+1) takes
 // the FMA-pipe cubic when cp % POLY_EVERY == POLY_EVERY - 1, MUFU ex2 otherwise.
 template <int POLY_EVERY>
-__device__ __forceinline__ float exp_block(const uint32_t* sr, float c, float m, uint32_t* pk) {
+__device__ __forceinline__ float exp_half(const uint32_t* sr, float c, float m, uint32_t* pk, int half) {
   const uint64_t c2 = f2_pack(c, c);
   const uint64_t nm2 = f2_pack(-m, -m);
   uint64_t acc[4];  // 4 independent packed partial sums (8 lanes of accumulation)
 #pragma unroll
   for (int i = 0; i < 4; ++i) acc[i] = 0ull;
 #pragma unroll
-  for (int cp = 0; cp < 64; ++cp) {
+  for (int q = 0; q < 32; ++q) {
+    const int cp = 32 * half + q;
     const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sr[2 * cp]), __uint_as_float(sr[2 * cp + 1])), c2, nm2);
-    float e0, e1;
+    float x0, x1, e0, e1;
+    f2_unpack(x2, x0, x1);
     if (POLY_EVERY > 0 && (cp % (POLY_EVERY > 0 ? POLY_EVERY : 1)) == POLY_EVERY - 1) {
       exp2_poly_x2(x2, e0, e1);
     } else {
-      float x0, x1;
-      f2_unpack(x2, x0, x1);
       e0 = exp2_mufu(x0);
       e1 = exp2_mufu(x1);
     }
-    acc[cp & 3] = f2_add(acc[cp & 3], f2_pack(e0, e1));
-    pk[cp] = pack_bf16x2(e0, e1);
+    acc[q & 3] = f2_add(acc[q & 3], f2_pack(e0, e1));
+    pk[q] = pack_bf16x2(e0, e1);
   }
   float a0, a1;
   f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
   // ---- setup
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::N_BARS; ++i)
-      mbar_init(bar(i), (i == L::B_P_FULL || i == L::B_P_FULL + 1) ? 128u : 1u);
+      mbar_init(bar(i), (i >= L::B_P_FULL && i < L::B_P_FULL + 4) ? 128u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -272,16 +272,18 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
         }
         umma_commit(bar(L::B_S_FULL + t));
       };
-      auto issue_pv = [&](int t, int stage, bool acc) {
+      // PV_t(j) in two halves of 64 keys, each issued once its half of P_t(j) is in TMEM
+      auto issue_pv_half = [&](int t, int stage, bool acc, int hf) {
         const uint32_t v_base = sbase + L::V_OFF + stage * L::TILE_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < L::BN / 16; ++kk) {
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int kk = 4 * hf + k4;
           // 16 keys = 16 rows of 128 B = 2048 bytes; 64-wide d blocks are BOX_BYTES apart.
           umma_ts(tmem + L::o_col(t), tmem + L::s_col(t) + kk * 8,
                   sdesc_sw128(v_base + kk * 2048, L::BOX_BYTES, 1024), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
         }
 #if ATTN_FWD_PV_WAIT
-        umma_commit(bar(L::B_PV_DONE + t));
+        if (hf == 1) umma_commit(bar(L::B_PV_DONE + t));
 #endif
       };
       bool ok = mbar_wait(bar(L::B_K_FULL), 0, ctl);
@@ -306,10 +308,14 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           if (!ok || j >= nblk[t]) continue;
-          ok = mbar_wait(bar(L::B_P_FULL + t), j & 1, ctl);
+          ok = mbar_wait(bar(L::B_P_FULL + 2 * t), j & 1, ctl);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(t, vs, j > 0);
+          issue_pv_half(t, vs, j > 0, 0);
+          ok = mbar_wait(bar(L::B_P_FULL + 2 * t + 1), j & 1, ctl);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv_half(t, vs, j > 0, 1);
           if (j == nblk[t] - 1) umma_commit(bar(L::B_O_FINAL + t));
           if (j + 1 < nblk[t]) {
             if (!k_next_ready) {
@@ -380,14 +386,9 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
         if (j > 0) ++rescales;
       }
       const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-      uint32_t pk[64];
-      // Masked blocks take MUFU ex2 only: it maps -inf to an exact 0.
-      const float rowsum = need_mask ? exp_block<0>(sr, c, m_eff, pk) : exp_block<POLY_EVERY>(sr, c, m_eff, pk);
-      l += rowsum;
-      tmem_st32(s_addr, pk);  // P_t(j) over the first 64 columns of S_t
-      tmem_st32(s_addr + 32, pk + 32);
       if (j > 0 && __any_sync(0xffffffffu, resc)) {
-        // PV_t(j-1) completed before S_t(j) was issued, so O_t is final up to block j-1.
+        // PV_t(j-1) completed before S_t(j) was issued, so O_t is final up to block
+        // j-1; it is rescaled before any part of P_t(j) is published.
         const uint32_t o_addr = tmem + lane_addr + L::o_col(t);
 #pragma unroll 1
         for (int ch = 0; ch < D / 32; ++ch) {
@@ -399,9 +400,18 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
           tmem_st32(o_addr + ch * 32, orr);
         }
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(bar(L::B_P_FULL + t));
+      // P_t(j) over the first 64 columns of S_t, published in two halves (keys 0-63,
+      // then 64-127) so the PV MMA starts on the first while the second is computed.
+      // Masked blocks take MUFU ex2 only: it maps -inf to an exact 0.
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t pk[32];
+        l += need_mask ? exp_half<0>(sr, c, m_eff, pk, hf) : exp_half<POLY_EVERY>(sr, c, m_eff, pk, hf);
+        tmem_st32(s_addr + 32 * hf, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(L::B_P_FULL + 2 * t + hf));
+      }
     }
     if (p.rescale_count != nullptr && rescales) atomicAdd(p.rescale_count, (unsigned long long)rescales);
 
