@@ -27,10 +27,11 @@
 // softmax writes P^T_{i+1}, dS^T_{i+1} only after dV_i, dK_i completed
 // (PD_FREE); dQ^T_{i+1} waits for the dQ warpgroup to have read dQ^T_i.
 //
-// Warp roles (384 threads): warps 0-3 softmax / dS and the dK, dV epilogue
-// (thread = key row = TMEM lane); warps 4-7 dQ reduction (thread = head-dim
-// row of dQ^T); warp 8 TMA producer; warp 9 TMEM allocator and MMA issuer;
-// warps 10-11 idle.
+// Warp roles (512 threads): warps 0-7 softmax / dS and the dK, dV epilogue
+// (thread = key row = TMEM lane, two warps per row, 32 queries each: P^T and dS^T
+// need no row reduction, so the row splits freely); warps 8-11 dQ reduction
+// (thread = head-dim row of dQ^T); warp 12 TMA producer; warp 13 TMEM allocator
+// and MMA issuer; warps 14-15 idle.
 #pragma once
 
 #include "sm100_common.cuh"
@@ -151,7 +152,7 @@ struct BwdLayout {
   static constexpr int B_QDO_FULL = 1;            // [NST]
   static constexpr int B_QDO_EMPTY = 1 + NST;     // [NST]
   static constexpr int B_S_FULL = 1 + 2 * NST;    // S^T_i and dP^T_i in TMEM
-  static constexpr int B_DS_READY = B_S_FULL + 1; // 128 arrivals: P^T_i, dS^T_i written
+  static constexpr int B_DS_READY = B_S_FULL + 1; // 256 arrivals: P^T_i, dS^T_i written
   static constexpr int B_PD_FREE = B_S_FULL + 2;  // dV_i, dK_i have read P^T_i, dS^T_i
   static constexpr int B_DQ_FULL = B_S_FULL + 3;  // dQ^T_i in TMEM
   static constexpr int B_DQ_FREE = B_S_FULL + 4;  // 128 arrivals: dQ^T_i read out
@@ -173,9 +174,10 @@ struct BwdLayout {
   static constexpr uint32_t DK_COL = 192 + D;       // D columns
   static constexpr uint32_t DQ_COL = 192 + 2 * D;   // 64 columns
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr int THREADS = 384;
-  static constexpr int WARP_TMA = 8, WARP_MMA = 9;
-  static constexpr int REG_MAIN = 216, REG_OTHER = 72;  // 2 x 128 x 216 + 128 x 72 = 384 x 168
+  // warps 0-7 softmax / dS (two warps per key row, 32 queries each), 8-11 dQ
+  // reduction, 12 TMA, 13 TMEM + MMA, 14-15 idle; 128 registers per thread.
+  static constexpr int THREADS = 512;
+  static constexpr int WARP_TMA = 12, WARP_MMA = 13;
 };
 
 template <int D, bool CAUSAL>
@@ -215,7 +217,7 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::N_BARS; ++i)
-      mbar_init(bar(i), (i == L::B_DS_READY || i == L::B_DQ_FREE || i == L::B_DQ_WG) ? 128u : 1u);
+      mbar_init(bar(i), i == L::B_DS_READY ? 256u : ((i == L::B_DQ_FREE || i == L::B_DQ_WG) ? 128u : 1u));
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -234,7 +236,6 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sptr + L::TMEM_SLOT_OFF);
 
-  if (warp >= 8) setmaxnreg_dec<L::REG_OTHER>();
 
   if (warp == L::WARP_TMA) {
     // ===================== TMA producer =====================
@@ -344,13 +345,13 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
       umma_commit(bar(L::B_DRAIN));
       mbar_wait_drain(bar(L::B_DRAIN), 0, 1000000000ull);
     }
-  } else if (warp < 4) {
-    // ===================== softmax / dS warpgroup: thread = key row =====================
-    setmaxnreg_inc<L::REG_MAIN>();
-    const int r = threadIdx.x;
+  } else if (warp < 8) {
+    // ===================== softmax / dS: thread = (key row, half of the 64 queries) =====================
+    const int r = threadIdx.x & 127;   // key row == TMEM lane
+    const int hc = threadIdx.x >> 7;   // query half: columns [32 hc, 32 hc + 32)
     const int key = k0 + r;
     const bool valid_key = key < p.S_k;
-    const uint32_t lane_addr = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int i = 0; i < m; ++i) {
@@ -361,30 +362,26 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
       ok = mbar_wait(bar(L::B_S_FULL), i & 1, ctl);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sv[64], dp[64];
-      tmem_ld32(tmem + lane_addr + L::X_COL, sv);
-      tmem_ld32(tmem + lane_addr + L::X_COL + 32, sv + 32);
-      tmem_ld32(tmem + lane_addr + L::Y_COL, dp);
-      tmem_ld32(tmem + lane_addr + L::Y_COL + 32, dp + 32);
+      uint32_t sv[32], dp[32];
+      tmem_ld32(tmem + lane_addr + L::X_COL + 32 * hc, sv);
+      tmem_ld32(tmem + lane_addr + L::Y_COL + 32 * hc, dp);
       tmem_ld_wait(sv);
-      tmem_ld_wait(sv + 32);
       tmem_ld_wait(dp);
-      tmem_ld_wait(dp + 32);
-      const float4* nl4 = reinterpret_cast<const float4*>(sptr + L::LD_OFF + st * 512);
-      const float4* dl4 = reinterpret_cast<const float4*>(sptr + L::LD_OFF + st * 512 + 256);
+      const float4* nl4 = reinterpret_cast<const float4*>(sptr + L::LD_OFF + st * 512) + 8 * hc;
+      const float4* dl4 = reinterpret_cast<const float4*>(sptr + L::LD_OFF + st * 512 + 256) + 8 * hc;
       // causal: key visible to query q0 + c iff c >= key - diag - q0; keys past S_k see nothing
-      const int c_first = !valid_key ? L::BQ : (CAUSAL ? key - diag - q0 : 0);
+      const int c_first = (!valid_key ? L::BQ : (CAUSAL ? key - diag - q0 : 0)) - 32 * hc;
       const bool masked = __any_sync(0xffffffffu, c_first > 0);
-      uint32_t pp[32], pd[32];
+      uint32_t pp[16], pd[16];
 #pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
+      for (int c4 = 0; c4 < 8; ++c4) {
         const float4 nlv = nl4[c4];
         const float4 dlv = dl4[c4];
 #pragma unroll
         for (int h2 = 0; h2 < 2; ++h2) {
           const int cp = 2 * c4 + h2;
           const float na = h2 ? nlv.z : nlv.x, nb = h2 ? nlv.w : nlv.y;
-          const float da = h2 ? dlv.z : dlv.x, db = h2 ? dlv.w : dlv.y;
+          const float da = h2 ? dlv.z : dlv.x, dbv = h2 ? dlv.w : dlv.y;
           const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[2 * cp]), __uint_as_float(sv[2 * cp + 1])), c2,
                                      f2_pack(na, nb));
           float x0, x1;
@@ -395,7 +392,7 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
             if (2 * cp + 1 < c_first) p1 = 0.f;
           }
           const uint64_t g2 = f2_sub(f2_pack(__uint_as_float(dp[2 * cp]), __uint_as_float(dp[2 * cp + 1])),
-                                     f2_pack(da, db));
+                                     f2_pack(da, dbv));
           float d0, d1;
           f2_unpack(f2_mul(f2_pack(p0, p1), g2), d0, d1);
           pp[cp] = pack_bf16x2(p0, p1);
@@ -405,8 +402,8 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
       // dS^T row r into the 128B-swizzled MN-major operand: 16-byte chunk c goes to chunk c ^ (r % 8)
       uint8_t* dsrow = sptr + L::DS_OFF + db * L::DS_BYTES + r * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(dsrow + ((c ^ (r & 7)) << 4)) =
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<uint4*>(dsrow + (((4 * hc + c) ^ (r & 7)) << 4)) =
             make_uint4(pd[4 * c], pd[4 * c + 1], pd[4 * c + 2], pd[4 * c + 3]);
       fence_proxy_async_smem();
       if (i >= 1) {  // dV_{i-1}, dK_{i-1} have read the previous P^T, dS^T
@@ -414,13 +411,13 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
       }
-      tmem_st32(tmem + lane_addr + L::P_COL, pp);
-      tmem_st32(tmem + lane_addr + L::DS_COL, pd);
+      tmem_st16(tmem + lane_addr + L::P_COL + 16 * hc, pp);  // P^T (bf16 pairs)
+      tmem_st16(tmem + lane_addr + L::DS_COL + 16 * hc, pd);  // dS^T
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar(L::B_DS_READY));
     }
-    // ---- epilogue: dV, dK (scaled) -> bf16
+    // ---- epilogue: dV, dK (scaled) -> bf16; this thread writes head dims [64 hc, 64 hc + 64)
     if (ok && m > 0) {
       ok = mbar_wait(bar(L::B_D_FINAL), 0, ctl);
       ok = __all_sync(0xffffffffu, ok);
@@ -434,7 +431,7 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
         const float sc = which == 0 ? 1.f : p.scale;
         __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + rowoff;
 #pragma unroll 1
-        for (int ch = 0; ch < D / 32; ++ch) {
+        for (int ch = 2 * hc; ch < 2 * hc + 2; ++ch) {
           uint32_t v[32];
           if (m > 0) {
             tmem_ld32(tmem + lane_addr + col + ch * 32, v);
@@ -455,12 +452,11 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
         }
       }
     }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ===================== dQ reduction warpgroup: thread = head-dim index =====================
     // dQ_i^T (TMEM) -> fp32 [64 q][D] tile in shared memory -> one TMA reduce-add
     // into the dQ accumulator (rows past S_q are clipped by the tensor map).
-    setmaxnreg_inc<L::REG_MAIN>();
-    const int d = threadIdx.x - 128;
+    const int d = threadIdx.x - 256;
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     float* stage = reinterpret_cast<float*>(sptr + L::DQ_STAGE_OFF);
     // Barrier among the 128 threads of this warpgroup built on an mbarrier, so
