@@ -46,6 +46,27 @@ WORKLOADS = {
 }
 
 
+def captured_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from profiles/roofline_traffic.txt, or None
+    when the kernel sources changed since that capture (sha1 mismatch)."""
+    import glob
+    import hashlib
+
+    h = hashlib.sha1()
+    for f in sorted(glob.glob(os.path.join(ROOT, "attention_attn_fwd_10_b200", "csrc", "*.cuh"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    try:
+        with open(os.path.join(ROOT, "profiles", "roofline_traffic.txt")) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) == 3 and not line.startswith("#") and parts[0] == kernel:
+                    return int(parts[1]) if parts[2] == h.hexdigest() else None
+    except OSError:
+        pass
+    return None
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -303,7 +324,8 @@ def run_ours(args):
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json bf16_tflops)"
                      if peaks_src == "measured" else "fallback 1.59 PFLOP/s burst",
-                     "traffic": None},
+                     "traffic": captured_traffic("attn_bwd_kernel" if dom.startswith("attn_bwd") else "attn_fwd_kernel"),
+                     "traffic_unit": "bytes per launch (ncu dram read + write)"},
         "e2e": e2e,
         "gpu_launches": args.steps * (1 + (3 if have_bwd else 0)),
         "clocks": clocks,
