@@ -152,6 +152,21 @@ cudaError_t launch_fwd_poly(int poly, const CUtensorMap& mq, const CUtensorMap& 
 
 // Evaluates the kernels' packed-pair cubic on x[2i], x[2i+1] (the last element of
 // an odd-length array is paired with itself).
+template <int D, bool CAUSAL>
+cudaError_t launch_bwd(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mq, const CUtensorMap& mdo,
+                       const CUtensorMap& mdq, const BwdParams& p, unsigned grid, cudaStream_t st) {
+  using L = BwdLayout<D>;
+  auto kern = attn_bwd_kernel<D, CAUSAL>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [&] {
+    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  kern<<<grid, L::THREADS, L::SMEM_BYTES, st>>>(mk, mv, mq, mdo, mdq, p);
+  return cudaGetLastError();
+}
+
 __global__ void exp2_poly_eval_kernel(const float* x, float* y, long long n) {
   const long long pairs = (n + 1) / 2;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < pairs;
@@ -261,7 +276,6 @@ attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const voi
   attn_status_t st = check_common(B, H_q, H_kv, S_q, S_k, D, causal, scale);
   if (st != ATTN_OK) return st;
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID_ARG;
-  if (D != 128) return ATTN_ERR_UNSUPPORTED;
   for (const void* ptr : {q, k, v, o, static_cast<const void*>(lse), dO, static_cast<const void*>(dq),
                           static_cast<const void*>(dk), static_cast<const void*>(dv), static_cast<const void*>(workspace)})
     if (!aligned16(ptr)) return ATTN_ERR_MISALIGNED;
@@ -305,32 +319,25 @@ attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const voi
   {
     const long long rows = static_cast<long long>(B) * s_pad * H_q;
     const long long blocks = (rows * (D / 8) + 255) / 256;
-    attn_bwd_preprocess_kernel<128><<<static_cast<unsigned>(blocks < 148 * 64 ? blocks : 148 * 64), 256, 0, s>>>(p);
+    const unsigned g = static_cast<unsigned>(blocks < 148 * 64 ? blocks : 148 * 64);
+    if (D == 128)
+      attn_bwd_preprocess_kernel<128><<<g, 256, 0, s>>>(p);
+    else
+      attn_bwd_preprocess_kernel<64><<<g, 256, 0, s>>>(p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   // 2. main pass
   if (opt && opt->main_pass_start && cudaEventRecord(static_cast<cudaEvent_t>(opt->main_pass_start), s) != cudaSuccess)
     return ATTN_ERR_CUDA;
   {
-    using L = BwdLayout<128>;
     const unsigned grid = static_cast<unsigned>(p.n_kv_tiles) * B * H_kv;
     cudaError_t err;
-    if (causal) {
-      auto kern = attn_bwd_kernel<128, true>;
-      static std::once_flag once;
-      static cudaError_t attr = cudaSuccess;
-      std::call_once(once, [&] { attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES); });
-      if (attr != cudaSuccess) return ATTN_ERR_CUDA;
-      kern<<<grid, L::THREADS, L::SMEM_BYTES, s>>>(mk, mv, mq, mdo, mdq, p);
-    } else {
-      auto kern = attn_bwd_kernel<128, false>;
-      static std::once_flag once;
-      static cudaError_t attr = cudaSuccess;
-      std::call_once(once, [&] { attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES); });
-      if (attr != cudaSuccess) return ATTN_ERR_CUDA;
-      kern<<<grid, L::THREADS, L::SMEM_BYTES, s>>>(mk, mv, mq, mdo, mdq, p);
-    }
-    err = cudaGetLastError();
+    if (D == 128)
+      err = causal ? launch_bwd<128, true>(mk, mv, mq, mdo, mdq, p, grid, s)
+                   : launch_bwd<128, false>(mk, mv, mq, mdo, mdq, p, grid, s);
+    else
+      err = causal ? launch_bwd<64, true>(mk, mv, mq, mdo, mdq, p, grid, s)
+                   : launch_bwd<64, false>(mk, mv, mq, mdo, mdq, p, grid, s);
     if (err != cudaSuccess) return ATTN_ERR_CUDA;
   }
   if (opt && opt->main_pass_stop && cudaEventRecord(static_cast<cudaEvent_t>(opt->main_pass_stop), s) != cudaSuccess)

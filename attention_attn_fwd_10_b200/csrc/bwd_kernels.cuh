@@ -30,8 +30,10 @@
 // Warp roles (512 threads): warps 0-7 softmax / dS and the dK, dV epilogue
 // (thread = key row = TMEM lane, two warps per row, 32 queries each: P^T and dS^T
 // need no row reduction, so the row splits freely); warps 8-11 dQ reduction
-// (thread = head-dim row of dQ^T); warp 12 TMA producer; warp 13 TMEM allocator
-// and MMA issuer; warps 14-15 idle.
+// (thread = head-dim row of dQ^T; at D = 64 dQ^T is an M = 64 accumulator whose
+// rows 16w..16w+15 sit in lanes 32w..32w+15, so half of each warp is idle);
+// warp 12 TMA producer; warp 13 TMEM allocator and MMA issuer; warps 14-15 idle.
+// Head dims 64 and 128.
 #pragma once
 
 #include "sm100_common.cuh"
@@ -56,7 +58,7 @@ struct BwdParams {
 };
 
 // ---------------------------------------------------------------------------
-// 1. preprocess: half a warp per (b, q, h) row of D = 128 (8 bf16 per lane)
+// 1. preprocess: D / 8 lanes per (b, q, h) row (8 bf16 per lane)
 template <int D>
 __global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(const BwdParams p) {
   constexpr int LANES = D / 8;          // lanes per row (8 bf16 each)
@@ -186,7 +188,7 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
                     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams p) {
   using L = BwdLayout<D>;
-  static_assert(D == 128, "the backward main pass is built for D = 128");
+  static_assert(D == 64 || D == 128, "head dim 64 or 128");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -417,7 +419,7 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
       tc_fence_before();
       mbar_arrive(bar(L::B_DS_READY));
     }
-    // ---- epilogue: dV, dK (scaled) -> bf16; this thread writes head dims [64 hc, 64 hc + 64)
+    // ---- epilogue: dV, dK (scaled) -> bf16; this thread writes head dims [D/2 hc, D/2 (hc + 1))
     if (ok && m > 0) {
       ok = mbar_wait(bar(L::B_D_FINAL), 0, ctl);
       ok = __all_sync(0xffffffffu, ok);
@@ -431,7 +433,7 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
         const float sc = which == 0 ? 1.f : p.scale;
         __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + rowoff;
 #pragma unroll 1
-        for (int ch = 2 * hc; ch < 2 * hc + 2; ++ch) {
+        for (int ch = (D / 64) * hc; ch < (D / 64) * (hc + 1); ++ch) {
           uint32_t v[32];
           if (m > 0) {
             tmem_ld32(tmem + lane_addr + col + ch * 32, v);
@@ -456,7 +458,11 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
     // ===================== dQ reduction warpgroup: thread = head-dim index =====================
     // dQ_i^T (TMEM) -> fp32 [64 q][D] tile in shared memory -> one TMA reduce-add
     // into the dQ accumulator (rows past S_q are clipped by the tensor map).
-    const int d = threadIdx.x - 256;
+    // dQ^T has M = D rows.  For D = 128 row d is TMEM lane d.  For D = 64 (an M = 64
+    // accumulator) rows 16g..16g+15 sit in lanes 32g..32g+15: only the low 16 lanes
+    // of each warp hold a row.
+    const int wl = (warp & 3) * 32 + lane;  // this thread's TMEM lane
+    const int d = D == 128 ? wl : ((lane < 16) ? (warp & 3) * 16 + lane : -1);
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     float* stage = reinterpret_cast<float*>(sptr + L::DQ_STAGE_OFF);
     // Barrier among the 128 threads of this warpgroup built on an mbarrier, so
@@ -479,20 +485,21 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
       tmem_ld_wait(v + 32);
       tc_fence_before();
       mbar_arrive(bar(L::B_DQ_FREE));
-      if (d == 0) bulk_wait_read_all();  // the previous reduce has read the staging tile
+      if (wl == 0) bulk_wait_read_all();  // the previous reduce has read the staging tile
       if (!wg_sync()) break;
 #pragma unroll
-      for (int c = 0; c < L::BQ; ++c) stage[c * D + d] = __uint_as_float(v[c]);
+      for (int c = 0; c < L::BQ; ++c)
+        if (d >= 0) stage[c * D + d] = __uint_as_float(v[c]);
       fence_proxy_async_smem();
       if (!wg_sync()) break;
-      if (d == 0) {
+      if (wl == 0) {
         const int h = hkv * G + i / per_head;
         const int q0 = (qb0 + i % per_head) * L::BQ;
         tma_reduce_add_4d(&tm_dqacc, sbase + L::DQ_STAGE_OFF, 0, h, q0, b);
         bulk_commit_group();
       }
     }
-    if (d == 0) bulk_wait_all();
+    if (wl == 0) bulk_wait_all();
   }
 
   tc_fence_before();

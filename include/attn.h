@@ -105,7 +105,6 @@ size_t attn_bwd_workspace_size(int B, int H_q, int S_q, int D);
  * (bf16).  `workspace` must hold attn_bwd_workspace_size(...) bytes, 16-byte
  * aligned; its contents on entry are ignored.  The dQ accumulation uses atomic
  * fp32 additions, so results may differ in the last bits from run to run.
- * This build serves D = 128 (other head dims: ATTN_ERR_UNSUPPORTED).
  */
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                        const void* dO, void* dq, void* dk, void* dv, void* workspace, int B, int H_q,

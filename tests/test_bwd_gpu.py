@@ -80,11 +80,17 @@ def test_backward_config_sampled_heads_and_invariants():
     assert (sum_dv - sum_do).abs().max() <= 3e-2 * sum_do.abs().max()
 
 
+@pytest.mark.parametrize("S_q,S_k", [(1, 1), (64, 64), (129, 129), (300, 300), (100, 260)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_head_dim_64(S_q, S_k, causal):
+    w = workloads.small(B=2, H_q=4, H_kv=2, S_q=S_q, S_k=S_k, D=64, causal=causal, seed=S_q + 3 * S_k,
+                        backward=True)
+    x = workloads.make_inputs(w)
+    _check(w, x, _gpu_fwd_bwd(x, causal, w.scale))
+
+
 def test_unsupported_head_dim_is_rejected():
     attn = _attn()
-    w = workloads.small(B=1, H_q=1, S_q=64, S_k=64, D=64, causal=False, seed=1, backward=True)
-    x = workloads.make_inputs(w)
-    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
-    o, lse = attn.fwd(q, k, v)
+    q = torch.zeros(1, 8, 1, 96, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(RuntimeError, match="UNSUPPORTED"):
-        attn.bwd(q, k, v, o, lse, do)
+        attn.bwd(q, q, q, q, torch.zeros(1, 1, 8, device="cuda"), q)
