@@ -30,6 +30,17 @@ namespace {
 constexpr unsigned long long kDefaultWaitLimitNs = 4000000000ull;
 std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
 
+// Grid order of the forward and of the backward main pass: (batch, head) pairs
+// per group of CTAs that run together and share L2.
+#ifndef ATTN_FWD_BH_GROUP
+#define ATTN_FWD_BH_GROUP 8
+#endif
+#ifndef ATTN_BWD_BH_GROUP
+#define ATTN_BWD_BH_GROUP 8
+#endif
+constexpr int kFwdBhGroup = ATTN_FWD_BH_GROUP;
+constexpr int kBwdBhGroup = ATTN_BWD_BH_GROUP;
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -239,6 +250,7 @@ attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, 
   p.S_q = S_q;
   p.S_k = S_k;
   p.n_units = (S_q + 255) / 256;
+  p.bh_group = kFwdBhGroup < B * H_q ? kFwdBhGroup : B * H_q;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.tau = opt.rescale_threshold;
   p.status = status;
@@ -303,6 +315,7 @@ attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const voi
   p.S_k = S_k;
   p.S_pad = s_pad;
   p.n_kv_tiles = (S_k + 127) / 128;
+  p.bh_group = kBwdBhGroup < B * H_kv ? kBwdBhGroup : B * H_kv;
   p.scale = scale;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.status = status;

@@ -52,6 +52,7 @@ struct BwdParams {
   __nv_bfloat16* dv;        // [B, S_k, H_kv, D]
   int B, H_q, H_kv, S_q, S_k, S_pad;
   int n_kv_tiles;           // ceil(S_k / 128)
+  int bh_group;             // main-pass grid order: (batch, kv head) pairs per group
   float scale, scale_log2;
   int* status;
   uint64_t wait_limit_ns;
@@ -154,13 +155,13 @@ struct BwdLayout {
   static constexpr int B_QDO_FULL = 1;            // [NST]
   static constexpr int B_QDO_EMPTY = 1 + NST;     // [NST]
   static constexpr int B_S_FULL = 1 + 2 * NST;    // S^T_i and dP^T_i in TMEM
-  static constexpr int B_DS_READY = B_S_FULL + 1; // 256 arrivals: P^T_i, dS^T_i written
+  static constexpr int B_DS_READY = B_S_FULL + 1; // 8 warp arrivals: P^T_i, dS^T_i written
   static constexpr int B_PD_FREE = B_S_FULL + 2;  // dV_i, dK_i have read P^T_i, dS^T_i
   static constexpr int B_DQ_FULL = B_S_FULL + 3;  // dQ^T_i in TMEM
-  static constexpr int B_DQ_FREE = B_S_FULL + 4;  // 128 arrivals: dQ^T_i read out
+  static constexpr int B_DQ_FREE = B_S_FULL + 4;  // 4 warp arrivals: dQ^T_i read out
   static constexpr int B_D_FINAL = B_S_FULL + 5;
   static constexpr int B_DRAIN = B_S_FULL + 6;
-  static constexpr int B_DQ_WG = B_S_FULL + 7;    // 128 arrivals: barrier among the dQ warpgroup
+  static constexpr int B_DQ_WG = B_S_FULL + 7;    // 4 warp arrivals: barrier among the dQ warpgroup
   static constexpr int N_BARS = B_S_FULL + 8;
   static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * N_BARS;
   static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 4;
@@ -199,10 +200,16 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work decode: causal tiles with the most query blocks (low key index) first
+  // ---- work decode: groups of bh_group (batch, kv head) pairs run together, so
+  // the dQ accumulator rows and Q / dO tiles they share stay in L2; inside a
+  // group, causal tiles with the most query blocks (low key index) come first
   const int BH = p.B * p.H_kv;
-  const int j = blockIdx.x / BH;
-  const int bh = blockIdx.x - j * BH;
+  const int per_group = p.bh_group * p.n_kv_tiles;
+  const int grp = blockIdx.x / per_group;
+  const int within = blockIdx.x - grp * per_group;
+  const int gs = min(p.bh_group, BH - grp * p.bh_group);
+  const int j = within / gs;
+  const int bh = grp * p.bh_group + (within - j * gs);
   const int b = bh / p.H_kv;
   const int hkv = bh - b * p.H_kv;
   const int G = p.H_q / p.H_kv;
@@ -219,7 +226,7 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::N_BARS; ++i)
-      mbar_init(bar(i), i == L::B_DS_READY ? 256u : ((i == L::B_DQ_FREE || i == L::B_DQ_WG) ? 128u : 1u));
+      mbar_init(bar(i), i == L::B_DS_READY ? 8u : ((i == L::B_DQ_FREE || i == L::B_DQ_WG) ? 4u : 1u));
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -417,7 +424,7 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
       tmem_st16(tmem + lane_addr + L::DS_COL + 16 * hc, pd);  // dS^T
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(L::B_DS_READY));
+      mbar_arrive_warp(bar(L::B_DS_READY));
     }
     // ---- epilogue: dV, dK (scaled) -> bf16; this thread writes head dims [D/2 hc, D/2 (hc + 1))
     if (ok && m > 0) {
@@ -469,7 +476,7 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
     // that every wait is bounded (a warp that gave up cannot strand the others).
     uint32_t wg_phase = 0;
     auto wg_sync = [&]() -> bool {
-      mbar_arrive(bar(L::B_DQ_WG));
+      mbar_arrive_warp(bar(L::B_DQ_WG));
       const bool r = mbar_wait(bar(L::B_DQ_WG), wg_phase & 1, ctl);
       ++wg_phase;
       return __all_sync(0xffffffffu, r);
@@ -484,7 +491,7 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
       tmem_ld_wait(v);
       tmem_ld_wait(v + 32);
       tc_fence_before();
-      mbar_arrive(bar(L::B_DQ_FREE));
+      mbar_arrive_warp(bar(L::B_DQ_FREE));
       if (wl == 0) bulk_wait_read_all();  // the previous reduce has read the staging tile
       if (!wg_sync()) break;
 #pragma unroll

@@ -46,6 +46,7 @@ struct FwdParams {
   float* lse;        // [B, H_q, S_q]
   int B, H_q, H_kv, S_q, S_k;
   int n_units;       // ceil(S_q / 256) work units per (batch, head)
+  int bh_group;      // grid order: (batch, head) pairs per group
   float scale_log2;  // scale * log2(e)
   float tau;         // rescale threshold (base-2 units); 0 = rescale on every increase
   int* status;       // device status word
@@ -74,7 +75,7 @@ struct FwdLayout {
   static constexpr int B_V_FULL = B_K_EMPTY + KST;     // [vs]
   static constexpr int B_V_EMPTY = B_V_FULL + VST;     // [vs]
   static constexpr int B_S_FULL = B_V_EMPTY + VST;     // [t]
-  static constexpr int B_P_FULL = B_S_FULL + 2;         // [t][half]  (128 arrivals)
+  static constexpr int B_P_FULL = B_S_FULL + 2;         // [t][half]  (one arrival per softmax warp)
   static constexpr int B_PV_DONE = B_P_FULL + 4;        // [t]
   static constexpr int B_O_FINAL = B_PV_DONE + 2;       // [t]
   static constexpr int B_DRAIN = B_O_FINAL + 2;
@@ -168,10 +169,16 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work decode: longest units first for causal (blocks are dispatched in index order)
+  // ---- work decode: groups of bh_group (batch, head) pairs run together, so the
+  // K / V rows they read stay in L2 (heads of one kv group are adjacent); inside a
+  // group, longest units first for causal (blocks are dispatched in index order)
   const int BH = p.B * p.H_q;
-  int u = blockIdx.x / BH;
-  const int bh = blockIdx.x - u * BH;
+  const int per_group = p.bh_group * p.n_units;
+  const int grp = blockIdx.x / per_group;
+  const int within = blockIdx.x - grp * per_group;
+  const int gs = min(p.bh_group, BH - grp * p.bh_group);
+  int u = within / gs;
+  const int bh = grp * p.bh_group + (within - u * gs);
   if (CAUSAL) u = p.n_units - 1 - u;
   const int b = bh / p.H_q;
   const int h = bh - b * p.H_q;
@@ -186,7 +193,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
   // ---- setup
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::N_BARS; ++i)
-      mbar_init(bar(i), (i >= L::B_P_FULL && i < L::B_P_FULL + 4) ? 128u : 1u);
+      mbar_init(bar(i), (i >= L::B_P_FULL && i < L::B_P_FULL + 4) ? 4u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -410,7 +417,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
         tmem_st32(s_addr + 32 * hf, pk);
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar(L::B_P_FULL + 2 * t + hf));
+        mbar_arrive_warp(bar(L::B_P_FULL + 2 * t + hf));
       }
     }
     if (p.rescale_count != nullptr && rescales) atomicAdd(p.rescale_count, (unsigned long long)rescales);
