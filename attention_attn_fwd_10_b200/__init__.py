@@ -7,6 +7,7 @@ machine without the built library or without a CUDA device these functions
 raise.
 
     o, lse = fwd(q, k, v, causal=True)            # q [B,S_q,H_q,D], k/v [B,S_k,H_kv,D] bf16
+    o, lse = fwd_split(q, k, v)                   # same result, key range split across CTAs (S_q << S_k)
     dq, dk, dv = bwd(q, k, v, o, lse, do, causal=True)
 
 Inputs may also be CPU tensors: they are copied to the current device, the
@@ -23,7 +24,7 @@ import torch
 from . import _abi
 from ._abi import FwdOptions, load, status_string  # noqa: F401
 
-__all__ = ["fwd", "bwd", "fwd_bwd", "device_status", "set_wait_limit_ns", "exp2_poly_eval", "bwd_workspace_size",
+__all__ = ["fwd", "fwd_split", "fwd_split_count", "bwd", "fwd_bwd", "device_status", "set_wait_limit_ns", "exp2_poly_eval", "bwd_workspace_size",
            "load", "status_string"]
 
 
@@ -82,6 +83,41 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse
     _abi.check(code, "attn_fwd")
     if on_host:
         return out.cpu(), lse.cpu()
+    return out, lse
+
+
+def fwd_split_count(B, H_q, S_q, S_k, causal: bool = False) -> int:
+    """Number of key ranges fwd_split uses by default (attn_fwd_split_count)."""
+    return int(load().attn_fwd_split_count(B, H_q, S_q, S_k, int(bool(causal))))
+
+
+def fwd_split(q, k, v, causal: bool = False, scale: float | None = None, num_splits: int = 0, out=None, lse=None,
+              workspace=None, stream=None):
+    """Split-KV forward (attn_fwd_split): the same (o, lse) as fwd, with the key
+    blocks divided among ``num_splits`` ranges (0 = library default) whose partial
+    results are merged by the log-sum-exp identity.  Device tensors only."""
+    B, S_q, H_q, S_k, H_kv, D = _shapes(q, k)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    _check_tensor("q", q, (B, S_q, H_q, D))
+    _check_tensor("k", k, (B, S_k, H_kv, D))
+    _check_tensor("v", v, (B, S_k, H_kv, D))
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H_q, S_q), dtype=torch.float32, device=q.device)
+    _check_tensor("out", out, (B, S_q, H_q, D))
+    _check_tensor("lse", lse, (B, H_q, S_q), torch.float32)
+    lib = load()
+    n = int(num_splits) if num_splits else fwd_split_count(B, H_q, S_q, S_k, causal)
+    need = int(lib.attn_fwd_split_workspace_size(B, H_q, S_q, D, n)) if n > 1 else 0
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is not None and workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace holds {workspace.numel() * workspace.element_size()} bytes, needs {need}")
+    code = lib.attn_fwd_split(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                              workspace.data_ptr() if workspace is not None else None, B, H_q, H_kv, S_q, S_k, D,
+                              int(bool(causal)), scale, n, _stream_ptr(stream))
+    _abi.check(code, "attn_fwd_split")
     return out, lse
 
 

@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -40,6 +41,9 @@ std::atomic<unsigned long long> g_wait_limit_ns{kDefaultWaitLimitNs};
 #endif
 constexpr int kFwdBhGroup = ATTN_FWD_BH_GROUP;
 constexpr int kBwdBhGroup = ATTN_BWD_BH_GROUP;
+
+constexpr int kNumSms = 148;     // B200
+constexpr int kMaxSplits = 128;  // key splits of the split-KV forward
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -191,6 +195,78 @@ __global__ void exp2_poly_eval_kernel(const float* x, float* y, long long n) {
   }
 }
 
+// Forward (unsplit when n_splits == 1); with n_splits > 1 the kernel writes
+// per-split partial results into `workspace` and a combine kernel merges them.
+attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace, int B,
+                      int H_q, int H_kv, int S_q, int S_k, int D, int causal, float scale,
+                      const attn_fwd_options_t* opt_in, int n_splits, void* stream) {
+  attn_fwd_options_t opt;
+  attn_fwd_default_options(&opt);
+  if (opt_in) opt = *opt_in;
+  attn_status_t st = check_common(B, H_q, H_kv, S_q, S_k, D, causal, scale);
+  if (st != ATTN_OK) return st;
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  // split ranges: split_blocks key blocks each; trailing splits that would be empty are dropped
+  const int n_kv = (S_k + 127) / 128;
+  const int split_blocks = (n_kv + n_splits - 1) / n_splits;
+  n_splits = (n_kv + split_blocks - 1) / split_blocks;
+  if (n_splits > 1 && (!workspace || !aligned16(workspace))) return workspace ? ATTN_ERR_MISALIGNED : ATTN_ERR_INVALID_ARG;
+  if (!(opt.rescale_threshold >= 0.f && opt.rescale_threshold <= 16.f)) return ATTN_ERR_INVALID_ARG;
+  if (opt.poly_exp_every != 0 && opt.poly_exp_every != 4 && opt.poly_exp_every != 8) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_MISALIGNED;
+
+  CUtensorMap mq, mk, mv;
+  if (!make_bshd_map(&mq, q, B, S_q, H_q, D) || !make_bshd_map(&mk, k, B, S_k, H_kv, D) ||
+      !make_bshd_map(&mv, v, B, S_k, H_kv, D))
+    return ATTN_ERR_CUDA;
+  int* status = status_ptr();
+  if (!status) return ATTN_ERR_CUDA;
+
+  FwdParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.B = B;
+  p.H_q = H_q;
+  p.H_kv = H_kv;
+  p.S_q = S_q;
+  p.S_k = S_k;
+  p.n_units = (S_q + 255) / 256;
+  p.bh_group = kFwdBhGroup < B * H_q ? kFwdBhGroup : B * H_q;
+  p.n_splits = n_splits;
+  p.split_blocks = split_blocks;
+  if (n_splits > 1) {
+    const size_t rows = static_cast<size_t>(n_splits) * B * H_q * S_q;
+    p.o_part = static_cast<float*>(workspace);
+    p.lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + (rows * D * sizeof(float) + 255) / 256 * 256);
+  }
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.tau = opt.rescale_threshold;
+  p.status = status;
+  p.rescale_count = opt.rescale_count;
+  p.wait_limit_ns = g_wait_limit_ns.load();
+  const unsigned grid = static_cast<unsigned>(p.n_units) * B * H_q * n_splits;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t err;
+  if (D == 128)
+    err = causal ? launch_fwd_poly<128, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s)
+                 : launch_fwd_poly<128, false>(opt.poly_exp_every, mq, mk, mv, p, grid, s);
+  else
+    err = causal ? launch_fwd_poly<64, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s)
+                 : launch_fwd_poly<64, false>(opt.poly_exp_every, mq, mk, mv, p, grid, s);
+  if (err != cudaSuccess) return ATTN_ERR_CUDA;
+  if (n_splits > 1) {
+    const long long warps = static_cast<long long>(B) * S_q * H_q;
+    const long long blocks = (warps + 7) / 8;
+    const unsigned g = static_cast<unsigned>(blocks < kNumSms * 16 ? blocks : kNumSms * 16);
+    if (D == 128)
+      attn_fwd_combine_kernel<128><<<g, 256, 0, s>>>(p);
+    else
+      attn_fwd_combine_kernel<64><<<g, 256, 0, s>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
 }  // namespace
 }  // namespace attn
 
@@ -224,54 +300,52 @@ void attn_fwd_default_options(attn_fwd_options_t* opt) {
 attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H_q,
                           int H_kv, int S_q, int S_k, int D, int causal, float scale,
                           const attn_fwd_options_t* opt_in, void* stream) {
-  attn_fwd_options_t opt;
-  attn_fwd_default_options(&opt);
-  if (opt_in) opt = *opt_in;
-  attn_status_t st = check_common(B, H_q, H_kv, S_q, S_k, D, causal, scale);
-  if (st != ATTN_OK) return st;
-  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
-  if (!(opt.rescale_threshold >= 0.f && opt.rescale_threshold <= 16.f)) return ATTN_ERR_INVALID_ARG;
-  if (opt.poly_exp_every != 0 && opt.poly_exp_every != 4 && opt.poly_exp_every != 8) return ATTN_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_MISALIGNED;
-
-  CUtensorMap mq, mk, mv;
-  if (!make_bshd_map(&mq, q, B, S_q, H_q, D) || !make_bshd_map(&mk, k, B, S_k, H_kv, D) ||
-      !make_bshd_map(&mv, v, B, S_k, H_kv, D))
-    return ATTN_ERR_CUDA;
-  int* status = status_ptr();
-  if (!status) return ATTN_ERR_CUDA;
-
-  FwdParams p{};
-  p.o = static_cast<__nv_bfloat16*>(o);
-  p.lse = lse;
-  p.B = B;
-  p.H_q = H_q;
-  p.H_kv = H_kv;
-  p.S_q = S_q;
-  p.S_k = S_k;
-  p.n_units = (S_q + 255) / 256;
-  p.bh_group = kFwdBhGroup < B * H_q ? kFwdBhGroup : B * H_q;
-  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  p.tau = opt.rescale_threshold;
-  p.status = status;
-  p.rescale_count = opt.rescale_count;
-  p.wait_limit_ns = g_wait_limit_ns.load();
-  const unsigned grid = static_cast<unsigned>(p.n_units) * B * H_q;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t err;
-  if (D == 128)
-    err = causal ? launch_fwd_poly<128, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s)
-                 : launch_fwd_poly<128, false>(opt.poly_exp_every, mq, mk, mv, p, grid, s);
-  else
-    err = causal ? launch_fwd_poly<64, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s)
-                 : launch_fwd_poly<64, false>(opt.poly_exp_every, mq, mk, mv, p, grid, s);
-  return err == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return run_fwd(q, k, v, o, lse, nullptr, B, H_q, H_kv, S_q, S_k, D, causal, scale, opt_in, 1, stream);
 }
 
 attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H_q, int H_kv,
                        int S_q, int S_k, int D, int causal, float scale, void* stream) {
   return attn_fwd_ex(q, k, v, o, lse, B, H_q, H_kv, S_q, S_k, D, causal, scale, nullptr, stream);
 }
+
+int attn_fwd_split_count(int B, int H_q, int S_q, int S_k, int causal) {
+  (void)causal;
+  if (B < 1 || H_q < 1 || S_q < 1 || S_k < 1) return 1;
+  const long long ctas = static_cast<long long>((S_q + 255) / 256) * B * H_q;
+  const int n_kv = (S_k + 127) / 128;
+  if (ctas >= kNumSms) return 1;
+  // time ~ waves of CTAs x (key blocks per range + ~2 blocks of per-CTA fixed cost)
+  int best = 1;
+  long long best_cost = -1;
+  for (int n = 1; n <= std::min(kMaxSplits, n_kv); ++n) {
+    const long long per = (n_kv + n - 1) / n;
+    const long long ranges = (n_kv + per - 1) / per;
+    const long long waves = (ctas * ranges + kNumSms - 1) / kNumSms;
+    const long long cost = waves * (per + 2);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = static_cast<int>(ranges);
+    }
+  }
+  return best;
+}
+
+size_t attn_fwd_split_workspace_size(int B, int H_q, int S_q, int D, int n_splits) {
+  if (B < 1 || H_q < 1 || S_q < 1 || (D != 64 && D != 128) || n_splits < 1 || n_splits > kMaxSplits) return 0;
+  if (n_splits == 1) return 0;
+  const size_t rows = static_cast<size_t>(n_splits) * B * H_q * S_q;
+  return (rows * D * sizeof(float) + 255) / 256 * 256 + (rows * sizeof(float) + 255) / 256 * 256;
+}
+
+attn_status_t attn_fwd_split(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace,
+                             int B, int H_q, int H_kv, int S_q, int S_k, int D, int causal, float scale,
+                             int n_splits, void* stream) {
+  if (n_splits < 0 || n_splits > kMaxSplits) return ATTN_ERR_INVALID_ARG;
+  if (n_splits == 0) n_splits = attn_fwd_split_count(B, H_q, S_q, S_k, causal);
+  return run_fwd(q, k, v, o, lse, workspace, B, H_q, H_kv, S_q, S_k, D, causal, scale, nullptr, n_splits, stream);
+}
+
+
 
 size_t attn_bwd_workspace_size(int B, int H_q, int S_q, int D) {
   if (B < 1 || H_q < 1 || S_q < 1 || (D != 64 && D != 128)) return 0;

@@ -47,6 +47,14 @@ struct FwdParams {
   int B, H_q, H_kv, S_q, S_k;
   int n_units;       // ceil(S_q / 256) work units per (batch, head)
   int bh_group;      // grid order: (batch, head) pairs per group
+  // Split-KV: each (unit, batch, head) is processed by n_splits CTAs, split s
+  // taking key blocks [s * split_blocks, (s + 1) * split_blocks).  With
+  // n_splits > 1 the kernel writes O_s (normalized within the split, fp32,
+  // [n_splits, B, S_q, H_q, D]) and lse_s ([n_splits, B, H_q, S_q]) for
+  // attn_fwd_combine_kernel instead of o and lse.
+  int n_splits, split_blocks;
+  float* o_part;
+  float* lse_part;
   float scale_log2;  // scale * log2(e)
   float tau;         // rescale threshold (base-2 units); 0 = rescale on every increase
   int* status;       // device status word
@@ -173,9 +181,11 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
   // K / V rows they read stay in L2 (heads of one kv group are adjacent); inside a
   // group, longest units first for causal (blocks are dispatched in index order)
   const int BH = p.B * p.H_q;
+  const int split = static_cast<int>(blockIdx.x) % p.n_splits;  // the splits of one unit are adjacent
+  const int cta = static_cast<int>(blockIdx.x) / p.n_splits;
   const int per_group = p.bh_group * p.n_units;
-  const int grp = blockIdx.x / per_group;
-  const int within = blockIdx.x - grp * per_group;
+  const int grp = cta / per_group;
+  const int within = cta - grp * per_group;
   const int gs = min(p.bh_group, BH - grp * p.bh_group);
   int u = within / gs;
   const int bh = grp * p.bh_group + (within - u * gs);
@@ -185,9 +195,12 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
   const int hkv = h / (p.H_q / p.H_kv);
   const int q0 = u * L::UNIT;
   const int diag = p.S_k - p.S_q;  // bottom-right causal: key j visible to row i iff j <= i + diag
+  // key blocks j0 + j, j < nblk[t], of this CTA's split that tile t sees
+  const int j0 = split * p.split_blocks;
   int nblk[2];
-  nblk[0] = tile_blocks(q0, p.S_q, p.S_k, CAUSAL, L::BN);
-  nblk[1] = tile_blocks(q0 + L::BM, p.S_q, p.S_k, CAUSAL, L::BN);
+#pragma unroll
+  for (int t = 0; t < 2; ++t)
+    nblk[t] = min(max(tile_blocks(q0 + t * L::BM, p.S_q, p.S_k, CAUSAL, L::BN) - j0, 0), p.split_blocks);
   const int n_blocks = max(nblk[0], nblk[1]);
 
   // ---- setup
@@ -237,7 +250,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
 #pragma unroll
         for (int x = 0; x < L::NBOX; ++x)
           tma_load_4d(sbase + L::K_OFF + s * L::TILE_BYTES + x * L::BOX_BYTES, &tm_k, bar(L::B_K_FULL + s),
-                      x * 64, hkv, j * L::BN, b);
+                      x * 64, hkv, (j0 + j) * L::BN, b);
         issued = j + 1;
       }
       // Drain: every load this thread issued has landed before the CTA may exit.
@@ -257,7 +270,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
 #pragma unroll
         for (int x = 0; x < L::NBOX; ++x)
           tma_load_4d(sbase + L::V_OFF + s * L::TILE_BYTES + x * L::BOX_BYTES, &tm_v, bar(L::B_V_FULL + s),
-                      x * 64, hkv, j * L::BN, b);
+                      x * 64, hkv, (j0 + j) * L::BN, b);
         issued = j + 1;
       }
       for (int s = 0; s < L::VST && s < issued; ++s)
@@ -374,7 +387,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       for (int ch = 0; ch < 4; ++ch) tmem_ld_wait(sr + ch * 32);
 
       float* s = reinterpret_cast<float*>(sr);
-      const int kbase = j * L::BN;
+      const int kbase = (j0 + j) * L::BN;
       const bool need_mask = (kbase + L::BN - 1 > lim_tile) || (kbase + L::BN > p.S_k);
       if (need_mask) {
         const int lim_c = lim - kbase;
@@ -427,7 +440,36 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       ok = mbar_wait(bar(L::B_O_FINAL + t), 0, ctl);
       ok = __all_sync(0xffffffffu, ok);
     }
-    if (ok) {
+    if (ok && p.n_splits > 1) {
+      // partial result of this split: fp32 O_s, lse_s
+      tc_fence_after();
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      const bool valid = qi < p.S_q;
+      const size_t part = static_cast<size_t>(split) * p.B + b;
+      float* prow = p.o_part + ((part * p.S_q + qi) * p.H_q + h) * D;
+      const uint32_t o_addr = tmem + lane_addr + L::o_col(t);
+#pragma unroll 1
+      for (int ch = 0; ch < D / 32; ++ch) {
+        uint32_t orr[32];
+        if (nb > 0) {
+          tmem_ld32(o_addr + ch * 32, orr);
+          tmem_ld_wait(orr);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) orr[i] = 0u;
+        }
+        if (valid) {
+          float4* dst = reinterpret_cast<float4*>(prow + ch * 32);
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            dst[i] = make_float4(__uint_as_float(orr[4 * i]) * inv_l, __uint_as_float(orr[4 * i + 1]) * inv_l,
+                                 __uint_as_float(orr[4 * i + 2]) * inv_l, __uint_as_float(orr[4 * i + 3]) * inv_l);
+        }
+      }
+      if (valid)
+        p.lse_part[(part * p.H_q + h) * p.S_q + qi] =
+            l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    } else if (ok) {
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       const bool valid = qi < p.S_q;
@@ -466,6 +508,52 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
   if (warp == L::WARP_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, L::TMEM_COLS);
+  }
+}
+
+// Split-KV combine, one warp per (b, q, h) row.  Split s saw a disjoint key range
+// and produced O_s (normalized over its keys) and lse_s = log sum over its keys
+// of exp(scale * s_ij); then, exactly,
+//   lse = log sum_s exp(lse_s),   O = sum_s exp(lse_s - lse) O_s,
+// evaluated with the largest lse_s factored out.  Rows that saw no key in any
+// split (every lse_s = -inf) give O = 0 and lse = -inf, as the unsplit kernel.
+template <int D>
+__global__ void __launch_bounds__(256) attn_fwd_combine_kernel(const FwdParams p) {
+  constexpr int PER = D / 32;  // values per lane
+  static_assert(PER == 2 || PER == 4, "head dim 64 or 128");
+  const long long rows = static_cast<long long>(p.B) * p.S_q * p.H_q;
+  const int lane = threadIdx.x & 31;
+  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  for (long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; w < rows; w += n_warps) {
+    // w = (b * S_q + q) * H_q + h, the row of O; the split-s row of o_part is s * rows + w
+    const int h = static_cast<int>(w % p.H_q);
+    const long long bq = w / p.H_q;
+    const int q = static_cast<int>(bq % p.S_q);
+    const int b = static_cast<int>(bq / p.S_q);
+    const size_t lse_stride = static_cast<size_t>(p.B) * p.H_q * p.S_q;
+    const size_t lse_row = (static_cast<size_t>(b) * p.H_q + h) * p.S_q + q;
+    float m = -INFINITY;
+    for (int s = 0; s < p.n_splits; ++s) m = fmaxf(m, p.lse_part[s * lse_stride + lse_row]);
+    float acc[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+    float sum = 0.f;
+    if (m > -INFINITY) {
+      for (int s = 0; s < p.n_splits; ++s) {
+        const float ls = p.lse_part[s * lse_stride + lse_row];
+        if (ls == -INFINITY) continue;
+        const float wgt = exp2_mufu((ls - m) * 1.4426950408889634f);
+        sum += wgt;
+        const float* src = p.o_part + (static_cast<size_t>(s) * rows + w) * D + lane * PER;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) acc[i] += wgt * src[i];
+      }
+    }
+    const float inv = sum > 0.f ? 1.f / sum : 0.f;
+    uint32_t* dst = reinterpret_cast<uint32_t*>(p.o + w * D + lane * PER);
+#pragma unroll
+    for (int i = 0; i < PER / 2; ++i) dst[i] = pack_bf16x2(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+    if (lane == 0) p.lse[lse_row] = sum > 0.f ? m + logf(sum) : -INFINITY;
   }
 }
 

@@ -92,6 +92,40 @@ attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, 
                           const attn_fwd_options_t* opt, void* stream);
 
 /*
+ * Split-KV forward for shapes with few query rows and many keys (decoding
+ * shapes: S_q << S_k), where one CTA per 256 query rows of each (batch, head)
+ * would leave most of the 148 SMs idle.  The pages describe no such variant;
+ * it computes the same O and lse as attn_fwd.  The ceil(S_k / 128) key blocks
+ * are cut into ranges of ceil(blocks / n_splits) blocks (trailing empty ranges
+ * are dropped).  Each range is processed by its own CTAs with the attn_fwd
+ * kernel, which writes the range's O_s (normalized over its keys, fp32) and
+ * lse_s into `workspace`.  A second kernel merges them with the log-sum-exp
+ * identity lse = log sum_s exp(lse_s), O = sum_s exp(lse_s - lse) O_s.  Causal
+ * masking is bottom-right as in attn_fwd.  Default attn_fwd options.
+ *
+ *   n_splits  : 0 = attn_fwd_split_count(...); 1 = plain attn_fwd (workspace may
+ *               be NULL); 2..128 = at most that many ranges.
+ *   workspace : device, 16-byte aligned, attn_fwd_split_workspace_size(B, H_q,
+ *               S_q, D, n_splits) bytes for the n_splits passed (or chosen);
+ *               owned by the caller, unused when only one range results.
+ * Errors as attn_fwd; ATTN_ERR_INVALID_ARG also for n_splits outside [0, 128]
+ * or a NULL workspace when more than one range results.
+ */
+attn_status_t attn_fwd_split(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace,
+                             int B, int H_q, int H_kv, int S_q, int S_k, int D, int causal, float scale,
+                             int n_splits, void* stream);
+
+/* The n_splits attn_fwd_split uses for n_splits = 0: 1 when ceil(S_q / 256) * B * H_q
+ * CTAs already fill the 148 SMs; otherwise the count (at most 128) that minimises
+ * waves of CTAs x (key blocks per range + 2), the 2 standing for a CTA's fixed cost. */
+int attn_fwd_split_count(int B, int H_q, int S_q, int S_k, int causal);
+
+/* Bytes of workspace attn_fwd_split needs for n_splits ranges: fp32 O_s
+ * [n_splits, B, S_q, H_q, D] and lse_s [n_splits, B, H_q, S_q]; 0 for n_splits = 1
+ * or invalid sizes. */
+size_t attn_fwd_split_workspace_size(int B, int H_q, int S_q, int D, int n_splits);
+
+/*
  * Bytes of device workspace attn_bwd needs: an fp32 dQ accumulator
  * [B, S_q, H_q, D] and two fp32 row-term arrays [B, H_q, S_pad] (S_pad =
  * S_q rounded up to 64): -lse_i * log2(e) and delta_i = sum_d dO_id O_id.

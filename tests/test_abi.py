@@ -86,3 +86,39 @@ def test_bwd_rejects_bad_arguments(lib):
 def test_exp2_eval_rejects_bad_arguments(lib):
     assert lib.attn_exp2_poly_eval(None, None, -1, None) == 1
     assert lib.attn_exp2_poly_eval(None, None, 0, None) == 0
+
+
+def test_fwd_split_count(lib):
+    # enough CTAs already: no split
+    assert lib.attn_fwd_split_count(2, 16, 8192, 8192, 1) == 1
+    # one query row per head, long context: split, never more ranges than key blocks or 128
+    n = lib.attn_fwd_split_count(1, 32, 1, 32768, 1)
+    assert 1 < n <= 128
+    assert lib.attn_fwd_split_count(1, 1, 1, 128, 0) == 1  # a single key block cannot be split
+    assert lib.attn_fwd_split_count(1, 1, 1, 1 << 20, 0) == 128
+    for S_k in (129, 1000, 4096, 70000):
+        n = lib.attn_fwd_split_count(1, 4, 3, S_k, 0)
+        assert 1 <= n <= (S_k + 127) // 128
+    assert lib.attn_fwd_split_count(0, 4, 3, 100, 0) == 1
+
+
+def test_fwd_split_workspace_size(lib):
+    B, H, S, D, n = 2, 8, 5, 128, 7
+    size = lib.attn_fwd_split_workspace_size(B, H, S, D, n)
+    assert size >= n * B * H * S * (D + 1) * 4
+    assert size % 256 == 0
+    assert lib.attn_fwd_split_workspace_size(B, H, S, D, 1) == 0
+    assert lib.attn_fwd_split_workspace_size(B, H, S, 96, n) == 0
+    assert lib.attn_fwd_split_workspace_size(B, H, S, D, 129) == 0
+
+
+def test_fwd_split_rejects_bad_arguments(lib):
+    p = [16] * 5
+    # n_splits out of range
+    assert lib.attn_fwd_split(*p, 16, 1, 2, 2, 8, 4096, 64, 0, 0.125, -1, None) == 1
+    assert lib.attn_fwd_split(*p, 16, 1, 2, 2, 8, 4096, 64, 0, 0.125, 129, None) == 1
+    # more than one key range needs a workspace
+    assert lib.attn_fwd_split(*p, None, 1, 2, 2, 8, 4096, 64, 0, 0.125, 4, None) == 1
+    # sizes are checked as for attn_fwd
+    assert lib.attn_fwd_split(*p, 16, 1, 3, 2, 8, 4096, 64, 0, 0.125, 4, None) == 1
+    assert lib.attn_fwd_split(*p, 16, 1, 2, 2, 8, 4096, 80, 0, 0.125, 4, None) == 2
