@@ -126,11 +126,12 @@ def bwd_workspace_size(B, H_q, S_q, D) -> int:
 
 
 def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, dq=None, dk=None, dv=None,
-        workspace=None, stream=None, main_pass_events=None):
+        workspace=None, stream=None, main_pass_events=None, deterministic: bool = False):
     """Backward attention.  Returns (dq, dk, dv) bf16 with the shapes of q, k, v.
 
     ``main_pass_events``: optional (start, stop) torch.cuda.Event pair recorded
-    around the main-pass kernel (diagnostic timing)."""
+    around the main-pass kernel (diagnostic timing).  ``deterministic``: add the
+    dQ parts of each query block in key-tile order (bitwise reproducible dQ)."""
     on_host = not q.is_cuda
     if on_host:
         dev = torch.device("cuda", torch.cuda.current_device())
@@ -154,12 +155,15 @@ def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, d
     if workspace.numel() * workspace.element_size() < need or not workspace.is_cuda:
         raise ValueError(f"workspace must be a CUDA buffer of at least {need} bytes")
     opt = None
-    if main_pass_events is not None:
-        s = torch.cuda.current_stream() if stream is None else stream
-        for e in main_pass_events:
-            if e.cuda_event == 0:  # torch creates the CUDA event lazily, on its first record
-                e.record(s)
-        opt = ctypes.byref(_abi.BwdOptions(main_pass_events[0].cuda_event, main_pass_events[1].cuda_event))
+    if main_pass_events is not None or deterministic:
+        ev = (None, None)
+        if main_pass_events is not None:
+            s = torch.cuda.current_stream() if stream is None else stream
+            for e in main_pass_events:
+                if e.cuda_event == 0:  # torch creates the CUDA event lazily, on its first record
+                    e.record(s)
+            ev = (main_pass_events[0].cuda_event, main_pass_events[1].cuda_event)
+        opt = ctypes.byref(_abi.BwdOptions(ev[0], ev[1], int(bool(deterministic))))
     code = load().attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
                               dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
                               B, H_q, H_kv, S_q, S_k, D, int(bool(causal)), scale, opt, _stream_ptr(stream))

@@ -55,7 +55,8 @@ class FwdOptions(ctypes.Structure):
 class BwdOptions(ctypes.Structure):
     """attn_bwd_options_t"""
 
-    _fields_ = [("main_pass_start", ctypes.c_void_p), ("main_pass_stop", ctypes.c_void_p)]
+    _fields_ = [("main_pass_start", ctypes.c_void_p), ("main_pass_stop", ctypes.c_void_p),
+                ("deterministic", ctypes.c_int)]
 
 
 _vp = ctypes.c_void_p

@@ -352,7 +352,8 @@ size_t attn_bwd_workspace_size(int B, int H_q, int S_q, int D) {
   const size_t s_pad = (static_cast<size_t>(S_q) + 63) / 64 * 64;
   const size_t dq_acc = static_cast<size_t>(B) * S_q * H_q * D * sizeof(float);
   const size_t rows = static_cast<size_t>(B) * H_q * s_pad * sizeof(float);
-  return (dq_acc + 255) / 256 * 256 + 2 * ((rows + 255) / 256 * 256);
+  const size_t sems = static_cast<size_t>(B) * H_q * (s_pad / 64) * sizeof(int);
+  return (dq_acc + 255) / 256 * 256 + 2 * ((rows + 255) / 256 * 256) + (sems + 255) / 256 * 256;
 }
 
 attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -379,6 +380,8 @@ attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const voi
   p.dq_acc = reinterpret_cast<float*>(ws);
   p.nlse2 = reinterpret_cast<float*>(ws + dq_bytes);
   p.delta = reinterpret_cast<float*>(ws + dq_bytes + row_bytes);
+  p.dq_sem = reinterpret_cast<int*>(ws + dq_bytes + 2 * row_bytes);
+  p.deterministic = (opt && opt->deterministic) ? 1 : 0;
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);

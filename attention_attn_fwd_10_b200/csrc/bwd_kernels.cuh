@@ -47,6 +47,8 @@ struct BwdParams {
   float* dq_acc;            // [B, S_q, H_q, D] fp32 (workspace)
   float* nlse2;             // [B, H_q, S_pad] = -lse * log2(e); -inf for padding / empty rows (workspace)
   float* delta;             // [B, H_q, S_pad] (workspace)
+  int* dq_sem;              // [B, H_q, S_pad / 64] dQ turn counters (workspace; deterministic mode)
+  int deterministic;        // 1: dQ contributions are added in key-tile order
   __nv_bfloat16* dq;        // [B, S_q, H_q, D]
   __nv_bfloat16* dk;        // [B, S_k, H_kv, D]
   __nv_bfloat16* dv;        // [B, S_k, H_kv, D]
@@ -97,6 +99,8 @@ __global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(const BwdParam
     }
 #pragma unroll
     for (int off = LANES / 2; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off, LANES);
+    if (in_range && sub == 0 && (q & 63) == 0)
+      p.dq_sem[(static_cast<size_t>(b) * p.H_q + h) * (p.S_pad / 64) + q / 64] = 0;
     if (in_range && sub == 0) {
       const size_t r = (static_cast<size_t>(b) * p.H_q + h) * p.S_pad + q;
       float nl = -INFINITY;  // padding rows and rows that saw no key give P = 0
@@ -501,9 +505,27 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
       if (!wg_sync()) break;
       if (wl == 0) {
         const int h = hkv * G + i / per_head;
-        const int q0 = (qb0 + i % per_head) * L::BQ;
-        tma_reduce_add_4d(&tm_dqacc, sbase + L::DQ_STAGE_OFF, 0, h, q0, b);
-        bulk_commit_group();
+        const int qb = qb0 + i % per_head;
+        // Deterministic mode: the key tiles that see query block qb are 0..J (lower
+        // keys are visible to more queries), so tile j adds its part after exactly
+        // j others, always in the order 0, 1, ..., J.  Tile j - 1 has the lower
+        // block index and was dispatched first, so the wait always ends.
+        int* sem = p.dq_sem + (static_cast<size_t>(b) * p.H_q + h) * (p.S_pad / 64) + qb;
+        bool turn = true;
+        if (p.deterministic) {
+          turn = sem_wait_eq(sem, j, ctl);
+          fence_proxy_async_global();
+        }
+        if (turn) {
+          tma_reduce_add_4d(&tm_dqacc, sbase + L::DQ_STAGE_OFF, 0, h, qb * L::BQ, b);
+          bulk_commit_group();
+          if (p.deterministic) {
+            bulk_wait_all();  // the additions are performed
+            fence_proxy_async_global();
+            __threadfence();
+            sem_release_add(sem);
+          }
+        }
       }
     }
     if (wl == 0) bulk_wait_all();

@@ -105,6 +105,35 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   }
 }
 
+// Waits until the global int at `sem` equals `want` (acquire at GPU scope), with
+// the same bound and abort protocol as mbar_wait.
+__device__ __forceinline__ bool sem_wait_eq(const int* sem, int want, const WaitCtl& ctl) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(sem) : "memory");
+    if (v == want) return true;
+    if ((it & 15u) == 0) {
+      if (*ctl.abort_flag) return false;
+      if (globaltimer_ns() - t0 > ctl.limit_ns) {
+        *ctl.abort_flag = 1;
+        atomicExch(ctl.status, kDevWaitTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// Adds 1 to the global int at `sem` with release semantics at GPU scope.
+__device__ __forceinline__ void sem_release_add(int* sem) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(sem) : "memory");
+}
+
+// Orders global-memory accesses of the async proxy (TMA) against the generic proxy.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Same, but with a fixed limit and no abort check: used only while draining
 // in-flight asynchronous work before a CTA exits.
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {

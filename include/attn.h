@@ -127,8 +127,9 @@ size_t attn_fwd_split_workspace_size(int B, int H_q, int S_q, int D, int n_split
 
 /*
  * Bytes of device workspace attn_bwd needs: an fp32 dQ accumulator
- * [B, S_q, H_q, D] and two fp32 row-term arrays [B, H_q, S_pad] (S_pad =
- * S_q rounded up to 64): -lse_i * log2(e) and delta_i = sum_d dO_id O_id.
+ * [B, S_q, H_q, D], two fp32 row-term arrays [B, H_q, S_pad] (S_pad =
+ * S_q rounded up to 64): -lse_i * log2(e) and delta_i = sum_d dO_id O_id, and
+ * one int per (b, h, 64-query block) for the deterministic mode's turn counters.
  * Returns 0 for invalid sizes.
  */
 size_t attn_bwd_workspace_size(int B, int H_q, int S_q, int D);
@@ -145,17 +146,26 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
                        int H_kv, int S_q, int S_k, int D, int causal, float scale, void* stream);
 
 /*
- * Diagnostics of the backward.  main_pass_start / main_pass_stop: optional
- * cudaEvent_t handles (created by the caller) that the library records on
- * `stream` immediately before and after the main-pass kernel, so the caller
- * can time that kernel alone.  NULL = not recorded.
+ * Options of the backward.
+ *   main_pass_start / main_pass_stop : optional cudaEvent_t handles (created by
+ *       the caller) that the library records on `stream` immediately before and
+ *       after the main-pass kernel, so the caller can time that kernel alone.
+ *       NULL = not recorded.
+ *   deterministic : 0 (default) = each key tile adds its dQ part for a query
+ *       block as soon as it has it, so the fp32 sums (and the bf16 dQ) may
+ *       differ in the last bits between runs.  1 = the parts for each (b, h,
+ *       64-query block) are added in increasing key-tile order, one tile waiting
+ *       (bounded) for the previous one's addition to complete.  dQ is then
+ *       bitwise identical from run to run (the pages' atomic reductions, section
+ *       7 item 3, leave the order open); dK, dV are deterministic in both modes.
  */
 typedef struct {
   void* main_pass_start;
   void* main_pass_stop;
+  int deterministic;
 } attn_bwd_options_t;
 
-/* attn_bwd with explicit options (`opt` NULL = none). */
+/* attn_bwd with explicit options (`opt` NULL = all fields 0). */
 attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse,
                           const void* dO, void* dq, void* dk, void* dv, void* workspace, int B, int H_q,
                           int H_kv, int S_q, int S_k, int D, int causal, float scale,

@@ -94,3 +94,43 @@ def test_unsupported_head_dim_is_rejected():
     q = torch.zeros(1, 8, 1, 96, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(RuntimeError, match="UNSUPPORTED"):
         attn.bwd(q, q, q, q, torch.zeros(1, 1, 8, device="cuda"), q)
+
+
+def _bwd_twice(w, deterministic):
+    attn = _attn()
+    x = workloads.make_inputs(w)
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = attn.fwd(q, k, v, causal=w.causal, scale=w.scale)
+    runs = [attn.bwd(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, deterministic=deterministic)
+            for _ in range(2)]
+    torch.cuda.synchronize()
+    assert attn.device_status() == 0
+    return x, runs
+
+
+@pytest.mark.parametrize("S_q,S_k,causal,H_q,H_kv", [(1536, 1536, True, 4, 2), (1536, 1536, False, 2, 2),
+                                                    (100, 900, True, 4, 1), (900, 100, True, 2, 2),
+                                                    (333, 333, False, 6, 3)])
+def test_deterministic_mode(S_q, S_k, causal, H_q, H_kv):
+    w = workloads.small(B=2, H_q=H_q, H_kv=H_kv, S_q=S_q, S_k=S_k, D=128, causal=causal, seed=S_q + S_k,
+                        backward=True)
+    x, (g1, g2) = _bwd_twice(w, True)
+    for a, b_ in zip(g1, g2):
+        assert torch.equal(a, b_), "deterministic backward differs between runs"
+    _check(w, x, g1)
+
+
+def test_deterministic_mode_head_dim_64():
+    w = workloads.small(B=1, H_q=4, H_kv=2, S_q=700, S_k=700, D=64, causal=True, seed=3, backward=True)
+    x, (g1, g2) = _bwd_twice(w, True)
+    for a, b_ in zip(g1, g2):
+        assert torch.equal(a, b_)
+    _check(w, x, g1)
+
+
+def test_deterministic_mode_backward_config():
+    w = workloads.BWD_CAUSAL
+    x, (g1, g2) = _bwd_twice(w, True)
+    for a, b_ in zip(g1, g2):
+        assert torch.equal(a, b_)
+    _check(w, x, g1, groups=[0], batches=[0])
