@@ -167,11 +167,11 @@ cudaError_t launch_fwd_poly(int poly, const CUtensorMap& mq, const CUtensorMap& 
 
 // Evaluates the kernels' packed-pair cubic on x[2i], x[2i+1] (the last element of
 // an odd-length array is paired with itself).
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool DET>
 cudaError_t launch_bwd(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mq, const CUtensorMap& mdo,
                        const CUtensorMap& mdq, const BwdParams& p, unsigned grid, cudaStream_t st) {
-  using L = BwdLayout<D>;
-  auto kern = attn_bwd_kernel<D, CAUSAL>;
+  using L = BwdLayout<D, DET>;
+  auto kern = attn_bwd_kernel<D, CAUSAL, DET>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
@@ -381,7 +381,7 @@ attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const voi
   p.nlse2 = reinterpret_cast<float*>(ws + dq_bytes);
   p.delta = reinterpret_cast<float*>(ws + dq_bytes + row_bytes);
   p.dq_sem = reinterpret_cast<int*>(ws + dq_bytes + 2 * row_bytes);
-  p.deterministic = (opt && opt->deterministic) ? 1 : 0;
+  const bool det = opt && opt->deterministic;
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
@@ -423,11 +423,15 @@ attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const voi
     const unsigned grid = static_cast<unsigned>(p.n_kv_tiles) * B * H_kv;
     cudaError_t err;
     if (D == 128)
-      err = causal ? launch_bwd<128, true>(mk, mv, mq, mdo, mdq, p, grid, s)
-                   : launch_bwd<128, false>(mk, mv, mq, mdo, mdq, p, grid, s);
+      err = det ? (causal ? launch_bwd<128, true, true>(mk, mv, mq, mdo, mdq, p, grid, s)
+                          : launch_bwd<128, false, true>(mk, mv, mq, mdo, mdq, p, grid, s))
+                : (causal ? launch_bwd<128, true, false>(mk, mv, mq, mdo, mdq, p, grid, s)
+                          : launch_bwd<128, false, false>(mk, mv, mq, mdo, mdq, p, grid, s));
     else
-      err = causal ? launch_bwd<64, true>(mk, mv, mq, mdo, mdq, p, grid, s)
-                   : launch_bwd<64, false>(mk, mv, mq, mdo, mdq, p, grid, s);
+      err = det ? (causal ? launch_bwd<64, true, true>(mk, mv, mq, mdo, mdq, p, grid, s)
+                          : launch_bwd<64, false, true>(mk, mv, mq, mdo, mdq, p, grid, s))
+                : (causal ? launch_bwd<64, true, false>(mk, mv, mq, mdo, mdq, p, grid, s)
+                          : launch_bwd<64, false, false>(mk, mv, mq, mdo, mdq, p, grid, s));
     if (err != cudaSuccess) return ATTN_ERR_CUDA;
   }
   if (opt && opt->main_pass_stop && cudaEventRecord(static_cast<cudaEvent_t>(opt->main_pass_stop), s) != cudaSuccess)

@@ -48,7 +48,6 @@ struct BwdParams {
   float* nlse2;             // [B, H_q, S_pad] = -lse * log2(e); -inf for padding / empty rows (workspace)
   float* delta;             // [B, H_q, S_pad] (workspace)
   int* dq_sem;              // [B, H_q, S_pad / 64] dQ turn counters (workspace; deterministic mode)
-  int deterministic;        // 1: dQ contributions are added in key-tile order
   __nv_bfloat16* dq;        // [B, S_q, H_q, D]
   __nv_bfloat16* dk;        // [B, S_k, H_kv, D]
   __nv_bfloat16* dv;        // [B, S_k, H_kv, D]
@@ -132,8 +131,10 @@ __global__ void __launch_bounds__(256) attn_bwd_convert_kernel(const BwdParams p
 }
 
 // ---------------------------------------------------------------------------
-// 2. main pass
-template <int D>
+// 2. main pass.  DET = deterministic dQ order; it trades the third Q/dO stage
+// for a second dQ staging tile, so a tile can wait for its turn while the next
+// block is staged.
+template <int D, bool DET>
 struct BwdLayout {
   static constexpr int BN = 128;                  // keys per CTA
   static constexpr int BQ = 64;                   // queries per block
@@ -144,16 +145,17 @@ struct BwdLayout {
   static constexpr int Q_TILE = 64 * D * 2;
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = K_OFF + KV_TILE;
-  static constexpr int NST = 3;                   // Q/dO ring depth
+  static constexpr int NST = DET ? 2 : 3;         // Q/dO ring depth
+  static constexpr int NDQ = DET ? 2 : 1;         // dQ staging tiles
   static constexpr int STAGE_OFF = V_OFF + KV_TILE;
   // one stage: Q_i, dO_i (1024-aligned); their -lse2_i and delta_i (64 fp32 each) sit in LD_OFF
   static constexpr int ST_Q = 0, ST_DO = Q_TILE;
   static constexpr int STAGE_BYTES = 2 * Q_TILE;
   static constexpr int DS_OFF = STAGE_OFF + NST * STAGE_BYTES;  // two dS^T buffers, 128 x 64 bf16
   static constexpr int DS_BYTES = 128 * 64 * 2;
-  static constexpr int DQ_STAGE_OFF = DS_OFF + 2 * DS_BYTES;  // dQ_i staging, fp32 [64 q][D]
+  static constexpr int DQ_STAGE_OFF = DS_OFF + 2 * DS_BYTES;  // NDQ dQ_i staging tiles, fp32 [64 q][D]
   static constexpr int DQ_STAGE_BYTES = 64 * D * 4;
-  static constexpr int LD_OFF = DQ_STAGE_OFF + DQ_STAGE_BYTES;  // per stage: -lse2 (256 B), delta (256 B)
+  static constexpr int LD_OFF = DQ_STAGE_OFF + NDQ * DQ_STAGE_BYTES;  // per stage: -lse2 (256 B), delta (256 B)
   static constexpr int BAR_OFF = LD_OFF + NST * 512;
   static constexpr int B_KV_FULL = 0;
   static constexpr int B_QDO_FULL = 1;            // [NST]
@@ -165,8 +167,9 @@ struct BwdLayout {
   static constexpr int B_DQ_FREE = B_S_FULL + 4;  // 4 warp arrivals: dQ^T_i read out
   static constexpr int B_D_FINAL = B_S_FULL + 5;
   static constexpr int B_DRAIN = B_S_FULL + 6;
-  static constexpr int B_DQ_WG = B_S_FULL + 7;    // 4 warp arrivals: barrier among the dQ warpgroup
-  static constexpr int N_BARS = B_S_FULL + 8;
+  static constexpr int B_STAGED = B_S_FULL + 7;   // [NDQ] 4 warp arrivals: dQ_i staged in tile i % NDQ
+  static constexpr int B_STAGE_FREE = B_S_FULL + 7 + NDQ;  // [NDQ] the reduce of that tile has read it
+  static constexpr int N_BARS = B_S_FULL + 7 + 2 * NDQ;
   static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * N_BARS;
   static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 4;
   static constexpr int SMEM_USED = ABORT_OFF + 4;
@@ -182,17 +185,18 @@ struct BwdLayout {
   static constexpr uint32_t DQ_COL = 192 + 2 * D;   // 64 columns
   static constexpr uint32_t TMEM_COLS = 512;
   // warps 0-7 softmax / dS (two warps per key row, 32 queries each), 8-11 dQ
-  // reduction, 12 TMA, 13 TMEM + MMA, 14-15 idle; 128 registers per thread.
+  // staging, 12 TMA, 13 TMEM + MMA, 14 dQ reduce issue, 15 idle; 128 registers
+  // per thread.
   static constexpr int THREADS = 512;
-  static constexpr int WARP_TMA = 12, WARP_MMA = 13;
+  static constexpr int WARP_TMA = 12, WARP_MMA = 13, WARP_RED = 14;
 };
 
-template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
+template <int D, bool CAUSAL, bool DET>
+__global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams p) {
-  using L = BwdLayout<D>;
+  using L = BwdLayout<D, DET>;
   static_assert(D == 64 || D == 128, "head dim 64 or 128");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -230,7 +234,8 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::N_BARS; ++i)
-      mbar_init(bar(i), i == L::B_DS_READY ? 8u : ((i == L::B_DQ_FREE || i == L::B_DQ_WG) ? 4u : 1u));
+      mbar_init(bar(i), i == L::B_DS_READY ? 8u
+                        : (i == L::B_DQ_FREE || (i >= L::B_STAGED && i < L::B_STAGED + L::NDQ)) ? 4u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -467,24 +472,14 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
     }
   } else if (warp < 12) {
     // ===================== dQ reduction warpgroup: thread = head-dim index =====================
-    // dQ_i^T (TMEM) -> fp32 [64 q][D] tile in shared memory -> one TMA reduce-add
-    // into the dQ accumulator (rows past S_q are clipped by the tensor map).
+    // dQ_i^T (TMEM) -> fp32 [64 q][D] tile in shared memory (NDQ tiles, used in
+    // turn); warp WARP_RED adds each tile into the dQ accumulator.
     // dQ^T has M = D rows.  For D = 128 row d is TMEM lane d.  For D = 64 (an M = 64
     // accumulator) rows 16g..16g+15 sit in lanes 32g..32g+15: only the low 16 lanes
     // of each warp hold a row.
     const int wl = (warp & 3) * 32 + lane;  // this thread's TMEM lane
     const int d = D == 128 ? wl : ((lane < 16) ? (warp & 3) * 16 + lane : -1);
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    float* stage = reinterpret_cast<float*>(sptr + L::DQ_STAGE_OFF);
-    // Barrier among the 128 threads of this warpgroup built on an mbarrier, so
-    // that every wait is bounded (a warp that gave up cannot strand the others).
-    uint32_t wg_phase = 0;
-    auto wg_sync = [&]() -> bool {
-      mbar_arrive_warp(bar(L::B_DQ_WG));
-      const bool r = mbar_wait(bar(L::B_DQ_WG), wg_phase & 1, ctl);
-      ++wg_phase;
-      return __all_sync(0xffffffffu, r);
-    };
     for (int i = 0; i < m; ++i) {
       bool ok = mbar_wait(bar(L::B_DQ_FULL), i & 1, ctl);
       if (!__all_sync(0xffffffffu, ok)) break;
@@ -496,14 +491,24 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
       tmem_ld_wait(v + 32);
       tc_fence_before();
       mbar_arrive_warp(bar(L::B_DQ_FREE));
-      if (wl == 0) bulk_wait_read_all();  // the previous reduce has read the staging tile
-      if (!wg_sync()) break;
+      const int buf = i % L::NDQ;
+      if (i >= L::NDQ) {  // the reduce of block i - NDQ has read this tile
+        ok = mbar_wait(bar(L::B_STAGE_FREE + buf), ((i / L::NDQ) - 1) & 1, ctl);
+        if (!__all_sync(0xffffffffu, ok)) break;
+      }
+      float* stage = reinterpret_cast<float*>(sptr + L::DQ_STAGE_OFF + buf * L::DQ_STAGE_BYTES);
 #pragma unroll
       for (int c = 0; c < L::BQ; ++c)
         if (d >= 0) stage[c * D + d] = __uint_as_float(v[c]);
       fence_proxy_async_smem();
-      if (!wg_sync()) break;
-      if (wl == 0) {
+      mbar_arrive_warp(bar(L::B_STAGED + buf));
+    }
+  } else if (warp == L::WARP_RED) {
+    // ===================== dQ reduce issue: one TMA reduce-add per staged tile =====================
+    if (lane == 0) {
+      for (int i = 0; i < m; ++i) {
+        const int buf = i % L::NDQ;
+        if (!mbar_wait(bar(L::B_STAGED + buf), (i / L::NDQ) & 1, ctl)) break;
         const int h = hkv * G + i / per_head;
         const int qb = qb0 + i % per_head;
         // Deterministic mode: the key tiles that see query block qb are 0..J (lower
@@ -511,24 +516,24 @@ __global__ void __launch_bounds__(BwdLayout<D>::THREADS, 1)
         // j others, always in the order 0, 1, ..., J.  Tile j - 1 has the lower
         // block index and was dispatched first, so the wait always ends.
         int* sem = p.dq_sem + (static_cast<size_t>(b) * p.H_q + h) * (p.S_pad / 64) + qb;
-        bool turn = true;
-        if (p.deterministic) {
-          turn = sem_wait_eq(sem, j, ctl);
+        if (DET) {
+          if (!sem_wait_eq(sem, j, ctl)) break;
           fence_proxy_async_global();
         }
-        if (turn) {
-          tma_reduce_add_4d(&tm_dqacc, sbase + L::DQ_STAGE_OFF, 0, h, qb * L::BQ, b);
-          bulk_commit_group();
-          if (p.deterministic) {
-            bulk_wait_all();  // the additions are performed
-            fence_proxy_async_global();
-            __threadfence();
-            sem_release_add(sem);
-          }
+        tma_reduce_add_4d(&tm_dqacc, sbase + L::DQ_STAGE_OFF + buf * L::DQ_STAGE_BYTES, 0, h, qb * L::BQ, b);
+        bulk_commit_group();
+        if (DET) {
+          bulk_wait_all();  // the additions are performed
+          fence_proxy_async_global();
+          __threadfence();
+          sem_release_add(sem);
+        } else {
+          bulk_wait_read_all();  // the tile has been read
         }
+        mbar_arrive(bar(L::B_STAGE_FREE + buf));
       }
+      bulk_wait_all();
     }
-    if (wl == 0) bulk_wait_all();
   }
 
   tc_fence_before();
