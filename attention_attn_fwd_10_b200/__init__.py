@@ -24,7 +24,7 @@ import torch
 from . import _abi
 from ._abi import FwdOptions, load, status_string  # noqa: F401
 
-__all__ = ["fwd", "fwd_split", "fwd_split_count", "bwd", "fwd_bwd", "device_status", "set_wait_limit_ns", "exp2_poly_eval", "bwd_workspace_size",
+__all__ = ["fwd", "fwd_split", "fwd_split_count", "bwd", "fwd_bwd", "FwdBwdPipeline", "device_status", "set_wait_limit_ns", "exp2_poly_eval", "bwd_workspace_size",
            "load", "status_string"]
 
 
@@ -193,6 +193,80 @@ def fwd_bwd(q, k, v, do, causal: bool = False, scale: float | None = None, host_
             host_out[name] = t.to("cpu")
     torch.cuda.current_stream().synchronize()
     return host_out
+
+
+class FwdBwdPipeline:
+    """Attention training steps (forward + backward) from pinned host buffers,
+    with the copies of one step overlapping the kernels of its neighbours.
+
+    Three streams: the inputs of a step (q, k, v, dO) go up on one copy stream,
+    its kernels run on a compute stream, and its results (o, lse, dq, dk, dv)
+    come down on a second copy stream.  ``depth`` sets of device buffers rotate
+    between steps, so step k+1 uploads while step k computes and step k-1
+    downloads.  Every step still moves all its inputs up and all its results
+    down; only the order of the work changes.
+
+        pipe = FwdBwdPipeline(B, S_q, S_k, H_q, H_kv, D, causal=True)
+        for hq, hk, hv, hdo, out in steps:      # pinned CPU tensors; out: dict of pinned tensors
+            pipe.submit(hq, hk, hv, hdo, out)
+        pipe.synchronize()                        # every submitted step's results are in `out`
+    """
+
+    def __init__(self, B, S_q, S_k, H_q, H_kv, D, causal: bool = False, scale: float | None = None,
+                 depth: int = 2, device=None):
+        self.dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.causal = bool(causal)
+        self.scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+        self.up, self.compute, self.down = (torch.cuda.Stream(self.dev) for _ in range(3))
+        bf, dev = torch.bfloat16, self.dev
+        ws = bwd_workspace_size(B, H_q, S_q, D)
+        self.sets = []
+        for _ in range(max(1, int(depth))):
+            self.sets.append({
+                "q": torch.empty((B, S_q, H_q, D), dtype=bf, device=dev),
+                "k": torch.empty((B, S_k, H_kv, D), dtype=bf, device=dev),
+                "v": torch.empty((B, S_k, H_kv, D), dtype=bf, device=dev),
+                "do": torch.empty((B, S_q, H_q, D), dtype=bf, device=dev),
+                "o": torch.empty((B, S_q, H_q, D), dtype=bf, device=dev),
+                "lse": torch.empty((B, H_q, S_q), dtype=torch.float32, device=dev),
+                "dq": torch.empty((B, S_q, H_q, D), dtype=bf, device=dev),
+                "dk": torch.empty((B, S_k, H_kv, D), dtype=bf, device=dev),
+                "dv": torch.empty((B, S_k, H_kv, D), dtype=bf, device=dev),
+                "ws": torch.empty(ws, dtype=torch.uint8, device=dev),
+                "uploaded": torch.cuda.Event(), "computed": torch.cuda.Event(), "downloaded": None,
+            })
+        self.n = 0
+
+    def submit(self, q, k, v, do, host_out: dict) -> None:
+        """Enqueue one step.  q, k, v, do: pinned CPU tensors; host_out: dict with
+        pinned CPU tensors "o", "lse", "dq", "dk", "dv" that receive the results
+        (valid after synchronize(), or once a later step's submit returned and
+        the caller synchronised).  Neither may be modified until then."""
+        s = self.sets[self.n % len(self.sets)]
+        self.n += 1
+        if s["downloaded"] is not None:  # this set's previous results must be down first
+            self.up.wait_event(s["downloaded"])
+        with torch.cuda.stream(self.up):
+            for name, t in (("q", q), ("k", k), ("v", v), ("do", do)):
+                s[name].copy_(t, non_blocking=True)
+            s["uploaded"].record(self.up)
+        self.compute.wait_event(s["uploaded"])
+        fwd(s["q"], s["k"], s["v"], causal=self.causal, scale=self.scale, out=s["o"], lse=s["lse"],
+            stream=self.compute)
+        bwd(s["q"], s["k"], s["v"], s["o"], s["lse"], s["do"], causal=self.causal, scale=self.scale,
+            dq=s["dq"], dk=s["dk"], dv=s["dv"], workspace=s["ws"], stream=self.compute)
+        s["computed"].record(self.compute)
+        self.down.wait_event(s["computed"])
+        with torch.cuda.stream(self.down):
+            for name in ("o", "lse", "dq", "dk", "dv"):
+                host_out[name].copy_(s[name], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(self.down)
+            s["downloaded"] = ev
+
+    def synchronize(self) -> None:
+        for st in (self.up, self.compute, self.down):
+            st.synchronize()
 
 
 def device_status(stream=None) -> int:
