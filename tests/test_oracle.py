@@ -376,6 +376,38 @@ def _pins_pass(fwd) -> bool:
         return False
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_range_merge_by_logsumexp(causal):
+    """The split-KV forward's combine step: attention over disjoint key ranges,
+    each normalised over its own keys (O_s, lse_s), merges into the full result
+    by lse = log sum_s exp(lse_s), O = sum_s exp(lse_s - lse) O_s.  Checked with
+    per-range softmaxes computed here from explicit fp64 scores (global causal
+    mask, so ranges that see no key of a row contribute lse_s = -inf)."""
+    B, S_q, S_k, H, D, scale = 1, 5, 40, 2, 8, 0.3
+    q, k, v = _rand((B, S_q, H, D), 1), _rand((B, S_k, H, D), 2), _rand((B, S_k, H, D), 3)
+    o_ref, lse_ref = ref.forward(q, k, v, causal, scale)
+    mask = ref.visible(S_q, S_k, causal)
+    for bounds in ([0, 40], [0, 13, 40], [0, 1, 2, 30, 39, 40], [0, 8, 16, 24, 32, 40]):
+        o_parts, l_parts = [], []
+        for a, b_ in zip(bounds[:-1], bounds[1:]):
+            s = np.einsum("bqhd,bkhd->bhqk", q, k[:, a:b_]) * scale
+            s = np.where(mask[None, None, :, a:b_], s, -np.inf)
+            m = s.max(axis=-1, keepdims=True)
+            e = np.where(np.isfinite(m), np.exp(s - np.where(np.isfinite(m), m, 0.0)), 0.0)
+            l = e.sum(axis=-1, keepdims=True)
+            with np.errstate(divide="ignore", invalid="ignore"):
+                o_parts.append(np.where(l > 0, np.einsum("bhqk,bkhd->bhqd", e, v[:, a:b_]) / l, 0.0))
+                l_parts.append(np.where(l[..., 0] > 0, m[..., 0] + np.log(l[..., 0]), -np.inf))
+        ls = np.stack(l_parts)                      # [splits, B, H, S_q]
+        mx = ls.max(axis=0)
+        w = np.where(np.isfinite(ls), np.exp(ls - np.where(np.isfinite(mx), mx, 0.0)), 0.0)
+        tot = w.sum(axis=0)
+        lse = np.where(tot > 0, mx + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+        o = np.einsum("sbhq,sbhqd->bhqd", w, np.stack(o_parts)) / np.where(tot > 0, tot, 1.0)[..., None]
+        np.testing.assert_allclose(lse, lse_ref, atol=1e-12)
+        np.testing.assert_allclose(o.transpose(0, 2, 1, 3), o_ref, atol=1e-12)
+
+
 def test_pins_catch_planted_mistakes():
     assert _pins_pass(lambda *a, **kw: ref.forward(*a, **kw))
     for m in _mutants():
