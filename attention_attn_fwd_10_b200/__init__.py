@@ -86,9 +86,9 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse
     return out, lse
 
 
-def fwd_split_count(B, H_q, S_q, S_k, causal: bool = False) -> int:
+def fwd_split_count(B, H_q, H_kv, S_q, S_k, causal: bool = False) -> int:
     """Number of key ranges fwd_split uses by default (attn_fwd_split_count)."""
-    return int(load().attn_fwd_split_count(B, H_q, S_q, S_k, int(bool(causal))))
+    return int(load().attn_fwd_split_count(B, H_q, H_kv, S_q, S_k, int(bool(causal))))
 
 
 def fwd_split(q, k, v, causal: bool = False, scale: float | None = None, num_splits: int = 0, out=None, lse=None,
@@ -108,7 +108,7 @@ def fwd_split(q, k, v, causal: bool = False, scale: float | None = None, num_spl
     _check_tensor("out", out, (B, S_q, H_q, D))
     _check_tensor("lse", lse, (B, H_q, S_q), torch.float32)
     lib = load()
-    n = int(num_splits) if num_splits else fwd_split_count(B, H_q, S_q, S_k, causal)
+    n = int(num_splits) if num_splits else fwd_split_count(B, H_q, H_kv, S_q, S_k, causal)
     need = int(lib.attn_fwd_split_workspace_size(B, H_q, S_q, D, n)) if n > 1 else 0
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)

@@ -63,14 +63,15 @@ EncodeTiledFn encode_fn() {
 }
 
 // bf16 BSHD tensor viewed as (D, H, S, B); boxes of 64 x 1 x box_rows x 1, 128-byte swizzle.
-bool make_bshd_map(CUtensorMap* map, const void* ptr, int B, int S, int H, int D, int box_rows = 128) {
+bool make_bshd_map(CUtensorMap* map, const void* ptr, int B, int S, int H, int D, int box_rows = 128,
+                   int box_heads = 1) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(B)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
                                  static_cast<cuuint64_t>(S) * H * D * 2};
-  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_heads), static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estride[4] = {1, 1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estride,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -195,6 +196,15 @@ __global__ void exp2_poly_eval_kernel(const float* x, float* y, long long n) {
   }
 }
 
+// Query heads packed into one forward tile: the whole kv group when S_q is short
+// (a tile of one head would be mostly empty) and the group size is a power of two
+// that leaves at least one query position per tile; else 1.
+int fwd_head_pack(int H_q, int H_kv, int S_q) {
+  const int G = H_q / H_kv;
+  if (S_q > 128 || G < 2 || G > 64 || (G & (G - 1)) != 0) return 1;
+  return G;
+}
+
 // Forward (unsplit when n_splits == 1); with n_splits > 1 the kernel writes
 // per-split partial results into `workspace` and a combine kernel merges them.
 attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace, int B,
@@ -215,8 +225,11 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   if (opt.poly_exp_every != 0 && opt.poly_exp_every != 4 && opt.poly_exp_every != 8) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_MISALIGNED;
 
+  const int gp = fwd_head_pack(H_q, H_kv, S_q);
+  int gp_log2 = 0;
+  while ((1 << gp_log2) < gp) ++gp_log2;
   CUtensorMap mq, mk, mv;
-  if (!make_bshd_map(&mq, q, B, S_q, H_q, D) || !make_bshd_map(&mk, k, B, S_k, H_kv, D) ||
+  if (!make_bshd_map(&mq, q, B, S_q, H_q, D, 128 / gp, gp) || !make_bshd_map(&mk, k, B, S_k, H_kv, D) ||
       !make_bshd_map(&mv, v, B, S_k, H_kv, D))
     return ATTN_ERR_CUDA;
   int* status = status_ptr();
@@ -230,8 +243,10 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   p.H_kv = H_kv;
   p.S_q = S_q;
   p.S_k = S_k;
-  p.n_units = (S_q + 255) / 256;
-  p.bh_group = kFwdBhGroup < B * H_q ? kFwdBhGroup : B * H_q;
+  p.gp = gp;
+  p.gp_log2 = gp_log2;
+  p.n_units = (S_q + 256 / gp - 1) / (256 / gp);
+  p.bh_group = kFwdBhGroup < B * (H_q / gp) ? kFwdBhGroup : B * (H_q / gp);
   p.n_splits = n_splits;
   p.split_blocks = split_blocks;
   if (n_splits > 1) {
@@ -244,7 +259,7 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   p.status = status;
   p.rescale_count = opt.rescale_count;
   p.wait_limit_ns = g_wait_limit_ns.load();
-  const unsigned grid = static_cast<unsigned>(p.n_units) * B * H_q * n_splits;
+  const unsigned grid = static_cast<unsigned>(p.n_units) * B * (H_q / gp) * n_splits;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t err;
   if (D == 128)
@@ -308,10 +323,11 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   return attn_fwd_ex(q, k, v, o, lse, B, H_q, H_kv, S_q, S_k, D, causal, scale, nullptr, stream);
 }
 
-int attn_fwd_split_count(int B, int H_q, int S_q, int S_k, int causal) {
+int attn_fwd_split_count(int B, int H_q, int H_kv, int S_q, int S_k, int causal) {
   (void)causal;
-  if (B < 1 || H_q < 1 || S_q < 1 || S_k < 1) return 1;
-  const long long ctas = static_cast<long long>((S_q + 255) / 256) * B * H_q;
+  if (B < 1 || H_q < 1 || H_kv < 1 || H_q % H_kv != 0 || S_q < 1 || S_k < 1) return 1;
+  const int gp = fwd_head_pack(H_q, H_kv, S_q);
+  const long long ctas = static_cast<long long>((S_q + 256 / gp - 1) / (256 / gp)) * B * (H_q / gp);
   const int n_kv = (S_k + 127) / 128;
   if (ctas >= kNumSms) return 1;
   // time ~ waves of CTAs x (key blocks per range + ~2 blocks of per-CTA fixed cost)
@@ -341,7 +357,7 @@ attn_status_t attn_fwd_split(const void* q, const void* k, const void* v, void* 
                              int B, int H_q, int H_kv, int S_q, int S_k, int D, int causal, float scale,
                              int n_splits, void* stream) {
   if (n_splits < 0 || n_splits > kMaxSplits) return ATTN_ERR_INVALID_ARG;
-  if (n_splits == 0) n_splits = attn_fwd_split_count(B, H_q, S_q, S_k, causal);
+  if (n_splits == 0) n_splits = attn_fwd_split_count(B, H_q, H_kv, S_q, S_k, causal);
   return run_fwd(q, k, v, o, lse, workspace, B, H_q, H_kv, S_q, S_k, D, causal, scale, nullptr, n_splits, stream);
 }
 

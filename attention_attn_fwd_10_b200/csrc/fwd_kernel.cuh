@@ -2,7 +2,9 @@
 //
 // One CTA owns a work unit of 256 query rows of one (batch, query head) -- two
 // 128-row Q tiles, A and B -- and streams the key/value blocks they can see;
-// each K_j / V_j block is loaded once and used by both tiles.  Warp roles:
+// each K_j / V_j block is loaded once and used by both tiles.  For short S_q the
+// query heads of one kv group share the tiles instead (row r = position r / gp
+// of head r % gp), so K / V are streamed once for the whole group.  Warp roles:
 //   warps 0-3   softmax warpgroup of tile A (thread t owns row t: TMEM lane t)
 //   warps 4-7   softmax warpgroup of tile B
 //   warp  8     TMA producer: Q_A, Q_B once, then K_j into a 3-stage ring
@@ -45,8 +47,13 @@ struct FwdParams {
   __nv_bfloat16* o;  // [B, S_q, H_q, D]
   float* lse;        // [B, H_q, S_q]
   int B, H_q, H_kv, S_q, S_k;
-  int n_units;       // ceil(S_q / 256) work units per (batch, head)
-  int bh_group;      // grid order: (batch, head) pairs per group
+  int n_units;       // work units per (batch, head pack): ceil(S_q / (256 / gp))
+  int bh_group;      // grid order: (batch, head pack) pairs per group
+  // Head packing: gp query heads of one kv group share a tile, tile row r holding
+  // query position r / gp of head r % gp (gp = 1: one head per tile).  Used for
+  // short S_q, where a tile of one head would be mostly empty; K / V are then
+  // streamed once per pack instead of once per head.
+  int gp, gp_log2;
   // Split-KV: each (unit, batch, head) is processed by n_splits CTAs, split s
   // taking key blocks [s * split_blocks, (s + 1) * split_blocks).  With
   // n_splits > 1 the kernel writes O_s (normalized within the split, fp32,
@@ -151,13 +158,13 @@ __device__ __forceinline__ float row_max128(const uint32_t* sr) {
   return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
-// Number of key blocks the rows [row0, row0 + 128) of a tile can see (0 if the
-// tile has no valid row, or none of its rows sees a key).
-__device__ __forceinline__ int tile_blocks(int row0, int S_q, int S_k, bool causal, int BN) {
+// Number of key blocks the query positions [row0, row0 + rows) of a tile can see
+// (0 if the tile has no valid row, or none of its rows sees a key).
+__device__ __forceinline__ int tile_blocks(int row0, int rows, int S_q, int S_k, bool causal, int BN) {
   if (row0 >= S_q) return 0;
   const int n_kv = (S_k + BN - 1) / BN;
   if (!causal) return n_kv;
-  const int last_key = min(row0 + 127, S_q - 1) + (S_k - S_q);
+  const int last_key = min(row0 + rows - 1, S_q - 1) + (S_k - S_q);
   return last_key < 0 ? 0 : min(n_kv, last_key / BN + 1);
 }
 
@@ -180,7 +187,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
   // ---- work decode: groups of bh_group (batch, head) pairs run together, so the
   // K / V rows they read stay in L2 (heads of one kv group are adjacent); inside a
   // group, longest units first for causal (blocks are dispatched in index order)
-  const int BH = p.B * p.H_q;
+  const int BH = p.B * (p.H_q >> p.gp_log2);  // (batch, head pack) pairs
   const int split = static_cast<int>(blockIdx.x) % p.n_splits;  // the splits of one unit are adjacent
   const int cta = static_cast<int>(blockIdx.x) / p.n_splits;
   const int per_group = p.bh_group * p.n_units;
@@ -190,17 +197,19 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
   int u = within / gs;
   const int bh = grp * p.bh_group + (within - u * gs);
   if (CAUSAL) u = p.n_units - 1 - u;
-  const int b = bh / p.H_q;
-  const int h = bh - b * p.H_q;
-  const int hkv = h / (p.H_q / p.H_kv);
-  const int q0 = u * L::UNIT;
+  const int b = bh / (p.H_q >> p.gp_log2);
+  const int h0 = (bh - b * (p.H_q >> p.gp_log2)) << p.gp_log2;  // first query head of the pack
+  const int hkv = h0 / (p.H_q / p.H_kv);
+  const int tile_pos = L::BM >> p.gp_log2;  // query positions per tile
+  const int q0 = u * 2 * tile_pos;          // first query position of the unit
   const int diag = p.S_k - p.S_q;  // bottom-right causal: key j visible to row i iff j <= i + diag
   // key blocks j0 + j, j < nblk[t], of this CTA's split that tile t sees
   const int j0 = split * p.split_blocks;
   int nblk[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t)
-    nblk[t] = min(max(tile_blocks(q0 + t * L::BM, p.S_q, p.S_k, CAUSAL, L::BN) - j0, 0), p.split_blocks);
+    nblk[t] = min(max(tile_blocks(q0 + t * tile_pos, tile_pos, p.S_q, p.S_k, CAUSAL, L::BN) - j0, 0),
+                  p.split_blocks);
   const int n_blocks = max(nblk[0], nblk[1]);
 
   // ---- setup
@@ -240,7 +249,7 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
 #pragma unroll
         for (int x = 0; x < L::NBOX; ++x)
           tma_load_4d(sbase + L::Q_OFF + t * L::TILE_BYTES + x * L::BOX_BYTES, &tm_q, bar(L::B_Q_FULL + t),
-                      x * 64, h, q0 + t * L::BM, b);
+                      x * 64, h0, q0 + t * tile_pos, b);
       }
       int issued = 0;
       for (int j = 0; j < n_blocks; ++j) {
@@ -364,8 +373,9 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
     setmaxnreg_inc<L::REG_SOFTMAX>();
     const int t = warp >> 2;
     const int row = threadIdx.x & 127;  // == TMEM lane
-    const int row0 = q0 + t * L::BM;
-    const int qi = row0 + row;
+    const int row0 = q0 + t * tile_pos;          // first query position of the tile
+    const int qi = row0 + (row >> p.gp_log2);     // this row's query position
+    const int h = h0 + (row & (p.gp - 1));        // and query head
     const int nb = nblk[t];
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float c = p.scale_log2;

@@ -115,10 +115,12 @@ attn_status_t attn_fwd_split(const void* q, const void* k, const void* v, void* 
                              int B, int H_q, int H_kv, int S_q, int S_k, int D, int causal, float scale,
                              int n_splits, void* stream);
 
-/* The n_splits attn_fwd_split uses for n_splits = 0: 1 when ceil(S_q / 256) * B * H_q
- * CTAs already fill the 148 SMs; otherwise the count (at most 128) that minimises
- * waves of CTAs x (key blocks per range + 2), the 2 standing for a CTA's fixed cost. */
-int attn_fwd_split_count(int B, int H_q, int S_q, int S_k, int causal);
+/* The n_splits attn_fwd_split uses for n_splits = 0: 1 when the forward's CTAs
+ * (one per 256 query rows of a (batch, head), or of a pack of the query heads of one
+ * kv group when S_q <= 128) already fill the 148 SMs; otherwise the count (at most
+ * 128) that minimises waves of CTAs x (key blocks per range + 2), the 2 standing
+ * for a CTA's fixed cost. */
+int attn_fwd_split_count(int B, int H_q, int H_kv, int S_q, int S_k, int causal);
 
 /* Bytes of workspace attn_fwd_split needs for n_splits ranges: fp32 O_s
  * [n_splits, B, S_q, H_q, D] and lse_s [n_splits, B, H_q, S_q]; 0 for n_splits = 1

@@ -90,16 +90,19 @@ def test_exp2_eval_rejects_bad_arguments(lib):
 
 def test_fwd_split_count(lib):
     # enough CTAs already: no split
-    assert lib.attn_fwd_split_count(2, 16, 8192, 8192, 1) == 1
+    assert lib.attn_fwd_split_count(2, 16, 16, 8192, 8192, 1) == 1
     # one query row per head, long context: split, never more ranges than key blocks or 128
-    n = lib.attn_fwd_split_count(1, 32, 1, 32768, 1)
+    n = lib.attn_fwd_split_count(1, 32, 8, 1, 32768, 1)
     assert 1 < n <= 128
-    assert lib.attn_fwd_split_count(1, 1, 1, 128, 0) == 1  # a single key block cannot be split
-    assert lib.attn_fwd_split_count(1, 1, 1, 1 << 20, 0) == 128
+    # packing the 4 heads of a kv group into one CTA leaves fewer CTAs: at least as many ranges
+    assert lib.attn_fwd_split_count(1, 32, 8, 1, 32768, 1) >= lib.attn_fwd_split_count(1, 32, 32, 1, 32768, 1)
+    assert lib.attn_fwd_split_count(1, 1, 1, 1, 128, 0) == 1  # a single key block cannot be split
+    assert lib.attn_fwd_split_count(1, 1, 1, 1, 1 << 20, 0) == 128
     for S_k in (129, 1000, 4096, 70000):
-        n = lib.attn_fwd_split_count(1, 4, 3, S_k, 0)
+        n = lib.attn_fwd_split_count(1, 4, 2, 3, S_k, 0)
         assert 1 <= n <= (S_k + 127) // 128
-    assert lib.attn_fwd_split_count(0, 4, 3, 100, 0) == 1
+    assert lib.attn_fwd_split_count(0, 4, 4, 3, 100, 0) == 1
+    assert lib.attn_fwd_split_count(1, 4, 3, 3, 100, 0) == 1  # H_q not a multiple of H_kv
 
 
 def test_fwd_split_workspace_size(lib):

@@ -127,3 +127,23 @@ def test_host_buffers_round_trip():
     o_ref, lse_ref = ref.forward(x["q"], x["k"], x["v"], False, w.scale)
     parity.check_o(o, o_ref)
     parity.check_lse(lse, lse_ref)
+
+
+@pytest.mark.parametrize("S_q,S_k", [(1, 300), (17, 17), (64, 500), (100, 100), (128, 1000)])
+@pytest.mark.parametrize("H_q,H_kv", [(4, 2), (8, 2), (16, 2), (64, 1)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_packed_query_heads(S_q, S_k, H_q, H_kv, causal):
+    # S_q <= 128 with a power-of-two group: the group's query heads share a tile
+    w = workloads.small(B=2, H_q=H_q, H_kv=H_kv, S_q=S_q, S_k=S_k, D=128, causal=causal, seed=S_q + H_q)
+    x, o, lse = _run(w)
+    o_ref, lse_ref = ref.forward(x["q"], x["k"], x["v"], causal, w.scale)
+    parity.check_o(o, o_ref, w.name)
+    parity.check_lse(lse, lse_ref, w.name)
+
+
+def test_packed_query_heads_d64():
+    w = workloads.small(B=1, H_q=8, H_kv=1, S_q=33, S_k=700, D=64, causal=True, seed=4)
+    x, o, lse = _run(w)
+    o_ref, lse_ref = ref.forward(x["q"], x["k"], x["v"], True, w.scale)
+    parity.check_o(o, o_ref, w.name)
+    parity.check_lse(lse, lse_ref, w.name)

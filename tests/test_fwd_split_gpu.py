@@ -73,7 +73,7 @@ def test_long_decode_sampled_heads():
     # one query row per head against 32768 keys (a decoding step with a long context, GQA 4:1)
     w = workloads.small(B=1, H_q=32, H_kv=8, S_q=1, S_k=32768, D=128, causal=True, seed=17)
     x, o, lse = _run(w, 0)
-    assert _attn().fwd_split_count(1, 32, 1, 32768, True) > 1
+    assert _attn().fwd_split_count(1, 32, 8, 1, 32768, True) > 1
     o_ref, lse_ref = ref.forward(x["q"], x["k"], x["v"], True, w.scale)
     parity.check_o(o, o_ref, w.name)
     parity.check_lse(lse, lse_ref, w.name)
