@@ -216,8 +216,9 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
   const int grp = blockIdx.x / per_group;
   const int within = blockIdx.x - grp * per_group;
   const int gs = min(p.bh_group, BH - grp * p.bh_group);
-  const int j = within / gs;
-  const int bh = grp * p.bh_group + (within - j * gs);
+  // deterministic instance: highest key tile first (see the dQ reduce below)
+  const int j = DET ? p.n_kv_tiles - 1 - within / gs : within / gs;
+  const int bh = grp * p.bh_group + (within % gs);
   const int b = bh / p.H_kv;
   const int hkv = bh - b * p.H_kv;
   const int G = p.H_q / p.H_kv;
@@ -512,12 +513,16 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
         const int h = hkv * G + i / per_head;
         const int qb = qb0 + i % per_head;
         // Deterministic mode: the key tiles that see query block qb are 0..J (lower
-        // keys are visible to more queries), so tile j adds its part after exactly
-        // j others, always in the order 0, 1, ..., J.  Tile j - 1 has the lower
-        // block index and was dispatched first, so the wait always ends.
+        // keys are visible to more queries).  They add their parts in the order J,
+        // J - 1, ..., 0 -- the order in which they reach the block, since tile j
+        // starts its sweep two blocks before tile j - 1 -- so tile j waits for
+        // J - j others.  The grid dispatches high tiles first, so tile j + 1 has
+        // the lower block index and is running or done: the wait always ends.
         int* sem = p.dq_sem + (static_cast<size_t>(b) * p.H_q + h) * (p.S_pad / 64) + qb;
         if (DET) {
-          if (!sem_wait_eq(sem, j, ctl)) break;
+          // J: the last tile whose first visited block, max(0, (128 J - diag) / 64), is <= qb
+          const int J = CAUSAL ? min(p.n_kv_tiles - 1, (64 * qb + 63 + (p.S_k - p.S_q)) / 128) : p.n_kv_tiles - 1;
+          if (!sem_wait_eq(sem, J - j, ctl)) break;
           fence_proxy_async_global();
         }
         tma_reduce_add_4d(&tm_dqacc, sbase + L::DQ_STAGE_OFF + buf * L::DQ_STAGE_BYTES, 0, h, qb * L::BQ, b);
