@@ -350,16 +350,6 @@ constexpr float kExp2C1 = 6.958335638e-01f;  // 0x3f322226
 constexpr float kExp2C2 = 2.260671407e-01f;  // 0x3e677e25
 constexpr float kExp2C3 = 7.802452892e-02f;  // 0x3d9fcb53
 
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = __fadd_rd(x, 12582912.0f);  // 1.5 * 2^23 + floor(x), exact
-  const float n = t - 12582912.0f;            // floor(x), exact
-  const float f = x - n;                      // [0, 1), exact
-  float p = fmaf(kExp2C3, f, kExp2C2);
-  p = fmaf(p, f, kExp2C1);
-  p = fmaf(p, f, kExp2C0);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
 
 // ----------------------------------------------------------------------------
 // Packed fp32 pairs (sm_100 f32x2 instructions: one issue slot per two lanes of work)
@@ -397,7 +387,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// The same cubic on a packed pair (two lanes of work per f32x2 instruction):
+// The cubic above on a packed pair (two lanes of work per f32x2 instruction):
 // clamp (two scalar max), floor via add.rm against 1.5*2^23, exact reduction,
 // Horner in fma.f32x2, then the exponent-field add per lane.
 __device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float& e0, float& e1) {
