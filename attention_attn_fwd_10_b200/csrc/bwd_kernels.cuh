@@ -18,22 +18,26 @@
 //          dS^T also goes to shared memory for the dQ product
 //   dV_j += P^T dO_i     (A from TMEM X)         dK_j += dS^T Q_i    (A from TMEM Y)
 //   dQ_i^T = K_j^T dS^T  (128 x 64: both operands MN-major in shared memory)
-// dV_j, dK_j accumulate in TMEM over all query blocks; dQ_i^T goes to one of
-// two TMEM buffers and a second warpgroup stages it in shared memory and adds
-// it into the fp32 dQ accumulator with one TMA reduce-add per block (the
-// "atomic reductions" of section 7, item 3).  Every MMA has M = 128.
+// dV_j, dK_j accumulate in TMEM over all query blocks.  dQ_i^T goes to a TMEM
+// buffer, a warpgroup copies it into a shared-memory staging tile, and a
+// separate warp adds the tile into the fp32 dQ accumulator with one TMA
+// reduce-add (the "atomic reductions" of section 7, item 3).  Every MMA has
+// M = 128 except dQ^T at D = 64 (M = 64).
 // Tensor-pipe order per block i: S^T_{i+1}, dP^T_{i+1}, dV_i, dK_i, dQ^T_i, so
 // the softmax of block i+1 overlaps dV_i, dK_i and dQ^T_i.  Barriers: the
 // softmax writes P^T_{i+1}, dS^T_{i+1} only after dV_i, dK_i completed
 // (PD_FREE); dQ^T_{i+1} waits for the dQ warpgroup to have read dQ^T_i.
+// Deterministic instance (DET): the additions into each (b, h, 64-query block)
+// of the accumulator happen in a fixed order of key tiles, through bounded turn
+// counters in global memory.
 //
 // Warp roles (512 threads): warps 0-7 softmax / dS and the dK, dV epilogue
 // (thread = key row = TMEM lane, two warps per row, 32 queries each: P^T and dS^T
-// need no row reduction, so the row splits freely); warps 8-11 dQ reduction
+// need no row reduction, so the row splits freely); warps 8-11 dQ staging
 // (thread = head-dim row of dQ^T; at D = 64 dQ^T is an M = 64 accumulator whose
 // rows 16w..16w+15 sit in lanes 32w..32w+15, so half of each warp is idle);
-// warp 12 TMA producer; warp 13 TMEM allocator and MMA issuer; warps 14-15 idle.
-// Head dims 64 and 128.
+// warp 12 TMA producer; warp 13 TMEM allocator and MMA issuer; warp 14 issues
+// the dQ reduce-adds; warp 15 idle.  Head dims 64 and 128.
 #pragma once
 
 #include "sm100_common.cuh"

@@ -140,8 +140,10 @@ size_t attn_bwd_workspace_size(int B, int H_q, int S_q, int D);
  * Backward pass.  q, k, v, o, lse as produced/consumed by attn_fwd with the
  * same arguments; dO is the gradient of the loss w.r.t. o.  Writes dq, dk, dv
  * (bf16).  `workspace` must hold attn_bwd_workspace_size(...) bytes, 16-byte
- * aligned; its contents on entry are ignored.  The dQ accumulation uses atomic
- * fp32 additions, so results may differ in the last bits from run to run.
+ * aligned; its contents on entry are ignored.  The dQ parts of the key tiles are
+ * added into an fp32 accumulator in the order the tiles finish, so dQ may differ
+ * in the last bits from run to run (attn_bwd_ex with deterministic = 1 fixes the
+ * order).  D = 64 or 128.
  */
 attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                        const void* dO, void* dq, void* dk, void* dv, void* workspace, int B, int H_q,
