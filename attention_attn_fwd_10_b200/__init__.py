@@ -24,7 +24,7 @@ import torch
 from . import _abi
 from ._abi import FwdOptions, load, status_string  # noqa: F401
 
-__all__ = ["fwd", "fwd_split", "fwd_split_count", "bwd", "fwd_bwd", "FwdBwdPipeline", "device_status", "set_wait_limit_ns", "exp2_poly_eval", "bwd_workspace_size",
+__all__ = ["fwd", "fwd_qk8", "fwd_split", "fwd_split_count", "bwd", "fwd_bwd", "FwdBwdPipeline", "device_status", "set_wait_limit_ns", "exp2_poly_eval", "bwd_workspace_size",
            "load", "status_string"]
 
 
@@ -83,6 +83,30 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse
     _abi.check(code, "attn_fwd")
     if on_host:
         return out.cpu(), lse.cpu()
+    return out, lse
+
+
+def fwd_qk8(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
+            rescale_threshold: float = 8.0, poly_exp_every: int = 8, stream=None):
+    """Forward with 8-bit Q and K (attn_fwd_qk8): q, k torch.float8_e4m3fn, v bf16,
+    head dim 128.  Returns (o bf16, lse fp32) of attention over the e4m3 values of
+    q and k.  Device tensors only."""
+    B, S_q, H_q, S_k, H_kv, D = _shapes(q, k)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    _check_tensor("q", q, (B, S_q, H_q, D), torch.float8_e4m3fn)
+    _check_tensor("k", k, (B, S_k, H_kv, D), torch.float8_e4m3fn)
+    _check_tensor("v", v, (B, S_k, H_kv, D))
+    if out is None:
+        out = torch.empty((B, S_q, H_q, D), dtype=torch.bfloat16, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H_q, S_q), dtype=torch.float32, device=q.device)
+    _check_tensor("out", out, (B, S_q, H_q, D))
+    _check_tensor("lse", lse, (B, H_q, S_q), torch.float32)
+    opt = FwdOptions(float(rescale_threshold), int(poly_exp_every), None)
+    code = load().attn_fwd_qk8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                               B, H_q, H_kv, S_q, S_k, D, int(bool(causal)), scale, ctypes.byref(opt),
+                               _stream_ptr(stream))
+    _abi.check(code, "attn_fwd_qk8")
     return out, lse
 
 

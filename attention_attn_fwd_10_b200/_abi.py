@@ -29,6 +29,7 @@ EXPORTED = (
     "attn_fwd",
     "attn_fwd_default_options",
     "attn_fwd_ex",
+    "attn_fwd_qk8",
     "attn_fwd_split",
     "attn_fwd_split_count",
     "attn_fwd_split_workspace_size",
@@ -70,6 +71,8 @@ _SIGNATURES = {
     "attn_fwd_default_options": (None, [ctypes.POINTER(FwdOptions)]),
     "attn_fwd_ex": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
                          ctypes.POINTER(FwdOptions), _vp]),
+    "attn_fwd_qk8": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
+                          ctypes.POINTER(FwdOptions), _vp]),
     "attn_fwd_split": (_i, [_vp] * 6 + [_i, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
     "attn_fwd_split_count": (_i, [_i, _i, _i, _i, _i, _i]),
     "attn_fwd_split_workspace_size": (ctypes.c_size_t, [_i, _i, _i, _i, _i]),

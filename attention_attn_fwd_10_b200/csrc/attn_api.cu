@@ -64,16 +64,20 @@ EncodeTiledFn encode_fn() {
 
 // bf16 BSHD tensor viewed as (D, H, S, B); boxes of 64 x 1 x box_rows x 1, 128-byte swizzle.
 bool make_bshd_map(CUtensorMap* map, const void* ptr, int B, int S, int H, int D, int box_rows = 128,
-                   int box_heads = 1) {
+                   int box_heads = 1, int elem_bytes = 2) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(B)};
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
-                                 static_cast<cuuint64_t>(S) * H * D * 2};
-  const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_heads), static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint64_t eb = static_cast<cuuint64_t>(elem_bytes);
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * eb, static_cast<cuuint64_t>(H) * D * eb,
+                                 static_cast<cuuint64_t>(S) * H * D * eb};
+  // 128-byte rows: 64 bf16 or 128 one-byte elements
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(box_heads),
+                             static_cast<cuuint32_t>(box_rows), 1};
   const cuuint32_t estride[4] = {1, 1, 1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estride,
+  const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return enc(map, dt, 4, const_cast<void*>(ptr), dims, strides, box, estride,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -141,11 +145,11 @@ attn_status_t check_common(int B, int H_q, int H_kv, int S_q, int S_k, int D, in
   return ATTN_OK;
 }
 
-template <int D, bool CAUSAL, int POLY>
+template <int D, bool CAUSAL, int POLY, bool QK8>
 cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
                        unsigned grid, cudaStream_t st) {
-  using L = FwdLayout<D>;
-  auto kern = attn_fwd_kernel<D, CAUSAL, POLY>;
+  using L = FwdLayout<D, QK8>;
+  auto kern = attn_fwd_kernel<D, CAUSAL, POLY, QK8>;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [&] {
@@ -156,18 +160,16 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   return cudaGetLastError();
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool QK8 = false>
 cudaError_t launch_fwd_poly(int poly, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                             const FwdParams& p, unsigned grid, cudaStream_t st) {
   switch (poly) {
-    case 0: return launch_fwd<D, CAUSAL, 0>(mq, mk, mv, p, grid, st);
-    case 4: return launch_fwd<D, CAUSAL, 4>(mq, mk, mv, p, grid, st);
-    default: return launch_fwd<D, CAUSAL, 8>(mq, mk, mv, p, grid, st);
+    case 0: return launch_fwd<D, CAUSAL, 0, QK8>(mq, mk, mv, p, grid, st);
+    case 4: return launch_fwd<D, CAUSAL, 4, QK8>(mq, mk, mv, p, grid, st);
+    default: return launch_fwd<D, CAUSAL, 8, QK8>(mq, mk, mv, p, grid, st);
   }
 }
 
-// Evaluates the kernels' packed-pair cubic on x[2i], x[2i+1] (the last element of
-// an odd-length array is paired with itself).
 template <int D, bool CAUSAL, bool DET>
 cudaError_t launch_bwd(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mq, const CUtensorMap& mdo,
                        const CUtensorMap& mdq, const BwdParams& p, unsigned grid, cudaStream_t st) {
@@ -183,6 +185,8 @@ cudaError_t launch_bwd(const CUtensorMap& mk, const CUtensorMap& mv, const CUten
   return cudaGetLastError();
 }
 
+// Evaluates the kernels' packed-pair cubic on x[2i], x[2i+1] (the last element of
+// an odd-length array is paired with itself).
 __global__ void exp2_poly_eval_kernel(const float* x, float* y, long long n) {
   const long long pairs = (n + 1) / 2;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < pairs;
@@ -209,13 +213,14 @@ int fwd_head_pack(int H_q, int H_kv, int S_q) {
 // per-split partial results into `workspace` and a combine kernel merges them.
 attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace, int B,
                       int H_q, int H_kv, int S_q, int S_k, int D, int causal, float scale,
-                      const attn_fwd_options_t* opt_in, int n_splits, void* stream) {
+                      const attn_fwd_options_t* opt_in, int n_splits, void* stream, bool qk8 = false) {
   attn_fwd_options_t opt;
   attn_fwd_default_options(&opt);
   if (opt_in) opt = *opt_in;
   attn_status_t st = check_common(B, H_q, H_kv, S_q, S_k, D, causal, scale);
   if (st != ATTN_OK) return st;
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (qk8 && D != 128) return ATTN_ERR_UNSUPPORTED;
   // split ranges: split_blocks key blocks each; trailing splits that would be empty are dropped
   const int n_kv = (S_k + 127) / 128;
   const int split_blocks = (n_kv + n_splits - 1) / n_splits;
@@ -229,8 +234,9 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   int gp_log2 = 0;
   while ((1 << gp_log2) < gp) ++gp_log2;
   CUtensorMap mq, mk, mv;
-  if (!make_bshd_map(&mq, q, B, S_q, H_q, D, 128 / gp, gp) || !make_bshd_map(&mk, k, B, S_k, H_kv, D) ||
-      !make_bshd_map(&mv, v, B, S_k, H_kv, D))
+  const int qk_bytes = qk8 ? 1 : 2;
+  if (!make_bshd_map(&mq, q, B, S_q, H_q, D, 128 / gp, gp, qk_bytes) ||
+      !make_bshd_map(&mk, k, B, S_k, H_kv, D, 128, 1, qk_bytes) || !make_bshd_map(&mv, v, B, S_k, H_kv, D))
     return ATTN_ERR_CUDA;
   int* status = status_ptr();
   if (!status) return ATTN_ERR_CUDA;
@@ -262,7 +268,10 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   const unsigned grid = static_cast<unsigned>(p.n_units) * B * (H_q / gp) * n_splits;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t err;
-  if (D == 128)
+  if (qk8)
+    err = causal ? launch_fwd_poly<128, true, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s)
+                 : launch_fwd_poly<128, false, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s);
+  else if (D == 128)
     err = causal ? launch_fwd_poly<128, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s)
                  : launch_fwd_poly<128, false>(opt.poly_exp_every, mq, mk, mv, p, grid, s);
   else
@@ -344,6 +353,12 @@ int attn_fwd_split_count(int B, int H_q, int H_kv, int S_q, int S_k, int causal)
     }
   }
   return best;
+}
+
+attn_status_t attn_fwd_qk8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H_q,
+                           int H_kv, int S_q, int S_k, int D, int causal, float scale,
+                           const attn_fwd_options_t* opt, void* stream) {
+  return run_fwd(q, k, v, o, lse, nullptr, B, H_q, H_kv, S_q, S_k, D, causal, scale, opt, 1, stream, true);
 }
 
 size_t attn_fwd_split_workspace_size(int B, int H_q, int S_q, int D, int n_splits) {

@@ -69,7 +69,9 @@ struct FwdParams {
   uint64_t wait_limit_ns;
 };
 
-template <int D>
+// QK8: Q and K are e4m3 (1 byte per element; head dim 128 only), S = Q K^T runs
+// as kind::f8f6f4; V, P and O stay bf16.
+template <int D, bool QK8 = false>
 struct FwdLayout {
   static constexpr int BM = 128;                 // query rows per tile
   static constexpr int UNIT = 256;               // query rows per work unit (two tiles)
@@ -79,9 +81,12 @@ struct FwdLayout {
   static constexpr int NBOX = D / 64;            // 64-element (128 B) TMA boxes per row block
   static constexpr int BOX_BYTES = 128 * 128;    // one 128 x 64 bf16 box
   static constexpr int TILE_BYTES = 128 * D * 2; // one 128 x D bf16 tile
+  static_assert(!QK8 || D == 128, "8-bit Q/K: head dim 128 (one 128-byte row per key)");
+  static constexpr int QK_BYTES = QK8 ? 128 * D : TILE_BYTES;  // one Q or K tile
+  static constexpr int QK_NBOX = QK8 ? 1 : NBOX;                // 128-byte TMA boxes per Q / K row
   static constexpr int Q_OFF = 0;                // two Q tiles
-  static constexpr int K_OFF = Q_OFF + 2 * TILE_BYTES;
-  static constexpr int V_OFF = K_OFF + KST * TILE_BYTES;
+  static constexpr int K_OFF = Q_OFF + 2 * QK_BYTES;
+  static constexpr int V_OFF = K_OFF + KST * QK_BYTES;
   static constexpr int BAR_OFF = V_OFF + VST * TILE_BYTES;
   // barrier slots (8 bytes each); [t] = per Q tile, [s] = per ring stage
   static constexpr int B_Q_FULL = 0;                    // [t]
@@ -168,11 +173,11 @@ __device__ __forceinline__ int tile_blocks(int row0, int rows, int S_q, int S_k,
   return last_key < 0 ? 0 : min(n_kv, last_key / BN + 1);
 }
 
-template <int D, bool CAUSAL, int POLY_EVERY>
-__global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
+template <int D, bool CAUSAL, int POLY_EVERY, bool QK8 = false>
+__global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using L = FwdLayout<D>;
+  using L = FwdLayout<D, QK8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -245,20 +250,20 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         if (nblk[t] == 0) continue;
-        mbar_arrive_expect_tx(bar(L::B_Q_FULL + t), L::TILE_BYTES);
+        mbar_arrive_expect_tx(bar(L::B_Q_FULL + t), L::QK_BYTES);
 #pragma unroll
-        for (int x = 0; x < L::NBOX; ++x)
-          tma_load_4d(sbase + L::Q_OFF + t * L::TILE_BYTES + x * L::BOX_BYTES, &tm_q, bar(L::B_Q_FULL + t),
+        for (int x = 0; x < L::QK_NBOX; ++x)
+          tma_load_4d(sbase + L::Q_OFF + t * L::QK_BYTES + x * L::BOX_BYTES, &tm_q, bar(L::B_Q_FULL + t),
                       x * 64, h0, q0 + t * tile_pos, b);
       }
       int issued = 0;
       for (int j = 0; j < n_blocks; ++j) {
         const int s = j % L::KST;
         if (j >= L::KST && !mbar_wait(bar(L::B_K_EMPTY + s), ((j / L::KST) - 1) & 1, ctl)) break;
-        mbar_arrive_expect_tx(bar(L::B_K_FULL + s), L::TILE_BYTES);
+        mbar_arrive_expect_tx(bar(L::B_K_FULL + s), L::QK_BYTES);
 #pragma unroll
-        for (int x = 0; x < L::NBOX; ++x)
-          tma_load_4d(sbase + L::K_OFF + s * L::TILE_BYTES + x * L::BOX_BYTES, &tm_k, bar(L::B_K_FULL + s),
+        for (int x = 0; x < L::QK_NBOX; ++x)
+          tma_load_4d(sbase + L::K_OFF + s * L::QK_BYTES + x * L::BOX_BYTES, &tm_k, bar(L::B_K_FULL + s),
                       x * 64, hkv, (j0 + j) * L::BN, b);
         issued = j + 1;
       }
@@ -291,8 +296,17 @@ __global__ void __launch_bounds__(FwdLayout<D>::THREADS, 1)
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
       auto issue_s = [&](int t, int stage) {
-        const uint32_t q_base = sbase + L::Q_OFF + t * L::TILE_BYTES;
-        const uint32_t k_base = sbase + L::K_OFF + stage * L::TILE_BYTES;
+        const uint32_t q_base = sbase + L::Q_OFF + t * L::QK_BYTES;
+        const uint32_t k_base = sbase + L::K_OFF + stage * L::QK_BYTES;
+        if constexpr (QK8) {
+          // 32 head dims (32 bytes of the 128-byte row) per MMA
+#pragma unroll
+          for (int kk = 0; kk < D / 32; ++kk)
+            umma_ss_f8(tmem + L::s_col(t), sdesc_sw128(q_base + kk * 32, 16, 1024),
+                       sdesc_sw128(k_base + kk * 32, 16, 1024), idesc_e4m3_f32(128, 128), kk > 0 ? 1u : 0u);
+          umma_commit(bar(L::B_S_FULL + t));
+          return;
+        }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32;

@@ -92,6 +92,21 @@ attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, 
                           const attn_fwd_options_t* opt, void* stream);
 
 /*
+ * Forward with 8-bit Q and K: q and k hold float8 e4m3 values (one byte per
+ * element, the same BSHD layout); v and o are bf16.  S = scale * Q K^T runs on
+ * the tensor cores' 8-bit path (kind::f8f6f4, fp32 accumulation, twice the
+ * bf16 rate); the softmax, P (bf16) and O += P V are as in attn_fwd.  The
+ * result is the attention of the e4m3 values themselves: the caller's
+ * quantisation of q and k is the only precision change (the "reduce precision"
+ * lever of AI Infra series ch. 6, GPU performance engineering (II), section 5).
+ * Head dim 128 only (else ATTN_ERR_UNSUPPORTED); options and errors as
+ * attn_fwd_ex.
+ */
+attn_status_t attn_fwd_qk8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H_q,
+                           int H_kv, int S_q, int S_k, int D, int causal, float scale,
+                           const attn_fwd_options_t* opt, void* stream);
+
+/*
  * Split-KV forward for shapes with few query rows and many keys (decoding
  * shapes: S_q << S_k), where one CTA per 256 query rows of each (batch, head)
  * would leave most of the 148 SMs idle.  The pages describe no such variant;

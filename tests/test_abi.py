@@ -125,3 +125,10 @@ def test_fwd_split_rejects_bad_arguments(lib):
     # sizes are checked as for attn_fwd
     assert lib.attn_fwd_split(*p, 16, 1, 3, 2, 8, 4096, 64, 0, 0.125, 4, None) == 1
     assert lib.attn_fwd_split(*p, 16, 1, 2, 2, 8, 4096, 80, 0, 0.125, 4, None) == 2
+
+
+def test_fwd_qk8_rejects_bad_arguments(lib):
+    p = [16] * 5
+    assert lib.attn_fwd_qk8(*p, 1, 2, 2, 8, 8, 64, 0, 0.125, None, None) == 2   # head dim 64: unsupported
+    assert lib.attn_fwd_qk8(*p, 1, 3, 2, 8, 8, 128, 0, 0.125, None, None) == 1  # H_q % H_kv != 0
+    assert lib.attn_fwd_qk8(16, 32, 48, None, 80, 1, 2, 2, 8, 8, 128, 0, 0.125, None, None) == 1

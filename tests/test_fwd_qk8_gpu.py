@@ -1,0 +1,59 @@
+"""GPU forward with 8-bit (e4m3) Q and K vs the fp64 oracle on the same e4m3 values.
+
+The kernel computes S = Q K^T on the tensor cores' 8-bit path with fp32
+accumulation; the oracle takes the e4m3 values of q and k (converted exactly to
+fp64).  Everything after S is as in the bf16 forward, so are the tolerances."""
+import pytest
+import torch
+
+import workloads
+from oracle import reference as ref
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(w, **kw):
+    import attention_attn_fwd_10_b200 as attn
+
+    x = workloads.make_inputs(w)
+    q8 = x["q"].to(torch.float8_e4m3fn)
+    k8 = x["k"].to(torch.float8_e4m3fn)
+    o, lse = attn.fwd_qk8(q8.cuda(), k8.cuda(), x["v"].cuda(), causal=w.causal, scale=w.scale, **kw)
+    torch.cuda.synchronize()
+    assert attn.device_status() == 0
+    # the oracle sees exactly the e4m3 values (fp8 -> fp32 is exact)
+    return q8.float(), k8.float(), x, o, lse
+
+
+@pytest.mark.parametrize("S_q,S_k", [(1, 1), (17, 17), (128, 128), (129, 129), (300, 300), (64, 500), (500, 64)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_small_shapes(S_q, S_k, causal):
+    w = workloads.small(B=2, H_q=2, S_q=S_q, S_k=S_k, D=128, causal=causal, seed=S_q * 13 + S_k)
+    q, k, x, o, lse = _run(w)
+    o_ref, lse_ref = ref.forward(q, k, x["v"], causal, w.scale)
+    parity.check_o(o, o_ref, w.name)
+    parity.check_lse(lse, lse_ref, w.name)
+
+
+@pytest.mark.parametrize("H_q,H_kv,S", [(4, 1, 400), (8, 2, 40)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa(H_q, H_kv, S, causal):
+    w = workloads.small(B=1, H_q=H_q, H_kv=H_kv, S_q=S, S_k=S, D=128, causal=causal, seed=5)
+    q, k, x, o, lse = _run(w)
+    o_ref, lse_ref = ref.forward(q, k, x["v"], causal, w.scale)
+    parity.check_o(o, o_ref, w.name)
+    parity.check_lse(lse, lse_ref, w.name)
+
+
+@pytest.mark.parametrize("poly", [0, 8])
+def test_causal_config_sampled(poly):
+    w = workloads.FWD_CAUSAL
+    q, k, x, o, lse = _run(w, poly_exp_every=poly)
+    o_c, lse_c = o.cpu(), lse.cpu()
+    rows = [0, 1, 127, 128, 255, 4095, 8190, 8191]
+    for (b, h) in [(0, 0), (1, 15)]:
+        o_ref, lse_ref = ref.forward_rows(q, k, x["v"], True, w.scale, b, h, rows)
+        parity.check_o(o_c[b, rows, h, :], o_ref, f"{w.name} b={b} h={h}")
+        parity.check_lse(lse_c[b, h, rows], lse_ref, f"{w.name} b={b} h={h}")
+    assert torch.isfinite(o_c.float()).all() and torch.isfinite(lse_c).all()
