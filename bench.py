@@ -461,6 +461,71 @@ def run_profile(args):
         sys.exit(1)
 
 
+def run_variants(args):
+    """Side measurements (not the contract line): the forward on each forward
+    configuration in bf16 and with 8-bit Q/K, the decode shapes through the plain
+    and the split-KV forward, and the backward in its normal and deterministic
+    modes.  CUDA events around each call, L2 flushed before each, median of
+    K timed calls after W warm-up calls.  One human-readable line each."""
+    import torch
+
+    import attention_attn_fwd_10_b200 as attn
+
+    torch.cuda.set_device(0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        ts = []
+        for _ in range(args.steps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        if attn.device_status() != 0:
+            raise RuntimeError("device status not OK")
+        return statistics.median(ts)
+
+    for w in (workloads.FWD_CAUSAL, workloads.FWD_NONCAUSAL, workloads.FWD_CAUSAL_GQA):
+        x = workloads.make_inputs(w)
+        q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+        q8, k8 = q.to(torch.float8_e4m3fn), k.to(torch.float8_e4m3fn)
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H_q, w.S_q), dtype=torch.float32, device="cuda")
+        ms16 = timed(lambda: attn.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse))
+        ms8 = timed(lambda: attn.fwd_qk8(q8, k8, v, causal=w.causal, scale=w.scale, out=o, lse=lse))
+        print(f"forward {w.name}: bf16 {ms16:.3f} ms {w.fwd_flops() / ms16 / 1e9:.0f} TFLOPS | "
+              f"e4m3 Q/K {ms8:.3f} ms {w.fwd_flops() / ms8 / 1e9:.0f} TFLOPS", flush=True)
+        del q, k, v, q8, k8, o, lse, x
+    for (B, H_q, H_kv, S_q, S_k) in ((1, 32, 8, 1, 32768), (8, 32, 8, 1, 8192), (4, 32, 8, 16, 65536),
+                                     (1, 16, 16, 128, 16384)):
+        w = workloads.small(B=B, H_q=H_q, H_kv=H_kv, S_q=S_q, S_k=S_k, D=128, causal=True, seed=1)
+        x = workloads.make_inputs(w)
+        q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+        ms_plain = timed(lambda: attn.fwd(q, k, v, causal=True, scale=w.scale))
+        ms_split = timed(lambda: attn.fwd_split(q, k, v, causal=True, scale=w.scale))
+        kv_bytes = 2 * B * S_k * H_kv * 128 * 2
+        n = attn.fwd_split_count(B, H_q, H_kv, S_q, S_k, True)
+        print(f"decode B{B} H_q{H_q} H_kv{H_kv} S_q{S_q} S_k{S_k}: forward {ms_plain * 1e3:.1f} us | "
+              f"split-KV ({n} ranges) {ms_split * 1e3:.1f} us, K+V {kv_bytes / ms_split / 1e9:.2f} TB/s", flush=True)
+        del q, k, v, x
+    wb = workloads.BWD_CAUSAL
+    x = workloads.make_inputs(wb)
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = attn.fwd(q, k, v, causal=True, scale=wb.scale)
+    ws = torch.empty(attn.bwd_workspace_size(wb.B, wb.H_q, wb.S_q, wb.D), dtype=torch.uint8, device="cuda")
+    grads = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
+    for det in (False, True):
+        ms = timed(lambda: attn.bwd(q, k, v, o, lse, do, causal=True, scale=wb.scale, dq=grads[0], dk=grads[1],
+                                    dv=grads[2], workspace=ws, deterministic=det))
+        print(f"backward {wb.name} deterministic={det}: {ms:.3f} ms {wb.bwd_flops() / ms / 1e9:.0f} TFLOPS",
+              flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -472,9 +537,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile", choices=("fwd", "bwd"), default=None,
                     help="only launch one pass W+K times (driver for ncu captures); prints no JSON")
+    ap.add_argument("--variants", action="store_true",
+                    help="side measurements (bf16 / e4m3 Q-K forward, decode shapes, deterministic backward); "
+                         "prints lines, not the JSON contract")
     args = ap.parse_args()
     if args.profile:
         run_profile(args)
+        return
+    if args.variants:
+        run_variants(args)
         return
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be >= 3")
