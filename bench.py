@@ -16,9 +16,15 @@ rank runs the same workload independently (replicas: the path has no
 exchange step), steps are bracketed by barriers and the slowest rank's time
 is reported; value = all ranks' FLOPs / that time.
 
+The e2e figure times the same steps from pinned host buffers through
+attn.FwdBwdPipeline (every step's inputs go up and its results come down inside
+the timed region; copies overlap the neighbouring steps' kernels).
+
 --impl reference times the fp64 CPU oracle on the host cores on a bounded
 sample of the same workload (the one other use of oracle/ here, besides the
-cpu_baseline leg).
+cpu_baseline leg).  --profile fwd|bwd launches one pass repeatedly (the driver
+for ncu captures); --variants prints timed side measurements (e4m3 Q/K forward,
+decode shapes, deterministic backward) instead of the JSON line.
 """
 from __future__ import annotations
 
