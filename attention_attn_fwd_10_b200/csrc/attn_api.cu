@@ -298,7 +298,7 @@ using namespace attn;
 
 extern "C" {
 
-int attn_abi_version(void) { return 1; }
+int attn_abi_version(void) { return 2; }
 
 const char* attn_status_string(attn_status_t s) {
   switch (s) {

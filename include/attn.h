@@ -47,7 +47,8 @@ typedef enum {
   ATTN_ERR_SCRATCH_TOO_SMALL = 6 /* attn_bwd_noalloc: the problem needs more than its fixed scratch */
 } attn_status_t;
 
-/* Version of this ABI (bumped on any incompatible change). */
+/* Version of this ABI (bumped on any incompatible change; 2: attn_bwd_options_t gained
+ * `deterministic`, the split-KV and 8-bit Q/K forwards were added). */
 int attn_abi_version(void);
 
 /* Human-readable name of a status code (static storage). */

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(lib):
 def test_status_strings(lib):
     for code, name in _abi.STATUS_NAMES.items():
         assert _abi.status_string(code).startswith(name)
-    assert lib.attn_abi_version() == 1
+    assert lib.attn_abi_version() == 2
 
 
 def _fwd(lib, **kw):
