@@ -1,0 +1,44 @@
+"""The forward and backward launch only kernels on the caller's stream (no host
+synchronisation, no allocation), so a whole training step can be captured in a
+CUDA graph and replayed; the replay gives the results of eager calls."""
+import pytest
+import torch
+
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+def test_fwd_bwd_step_in_a_cuda_graph():
+    import attention_attn_fwd_10_b200 as attn
+
+    w = workloads.small(B=1, H_q=4, H_kv=2, S_q=700, S_k=700, D=128, causal=True, seed=8, backward=True)
+    x = workloads.make_inputs(w)
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H_q, w.S_q), dtype=torch.float32, device="cuda")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(attn.bwd_workspace_size(w.B, w.H_q, w.S_q, w.D), dtype=torch.uint8, device="cuda")
+
+    def step(stream=None):
+        attn.fwd(q, k, v, causal=True, scale=w.scale, out=o, lse=lse, stream=stream)
+        attn.bwd(q, k, v, o, lse, do, causal=True, scale=w.scale, dq=dq, dk=dk, dv=dv, workspace=ws,
+                 stream=stream)
+
+    step()  # eager: one-time setup (kernel attributes, status word) happens here
+    torch.cuda.synchronize()
+    ref = [t.clone() for t in (o, lse, dq, dk, dv)]
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step(stream=s)
+    for t in (o, lse, dq, dk, dv):
+        t.zero_()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert attn.device_status() == 0
+    assert torch.equal(o, ref[0]) and torch.equal(lse, ref[1])
+    assert torch.equal(dk, ref[3]) and torch.equal(dv, ref[4])
+    # dQ sums the key tiles' parts in completion order: equal up to fp32 reassociation
+    assert (dq.float() - ref[2].float()).abs().max() <= 1e-2 * ref[2].float().abs().max()
