@@ -519,17 +519,22 @@ def run_variants(args):
         print(f"decode B{B} H_q{H_q} H_kv{H_kv} S_q{S_q} S_k{S_k}: forward {ms_plain * 1e3:.1f} us | "
               f"split-KV ({n} ranges) {ms_split * 1e3:.1f} us, K+V {kv_bytes / ms_split / 1e9:.2f} TB/s", flush=True)
         del q, k, v, x
-    wb = workloads.BWD_CAUSAL
-    x = workloads.make_inputs(wb)
-    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
-    o, lse = attn.fwd(q, k, v, causal=True, scale=wb.scale)
-    ws = torch.empty(attn.bwd_workspace_size(wb.B, wb.H_q, wb.S_q, wb.D), dtype=torch.uint8, device="cuda")
-    grads = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
-    for det in (False, True):
-        ms = timed(lambda: attn.bwd(q, k, v, o, lse, do, causal=True, scale=wb.scale, dq=grads[0], dk=grads[1],
-                                    dv=grads[2], workspace=ws, deterministic=det))
-        print(f"backward {wb.name} deterministic={det}: {ms:.3f} ms {wb.bwd_flops() / ms / 1e9:.0f} TFLOPS",
-              flush=True)
+    for wb in (workloads.BWD_CAUSAL,
+               workloads.small(B=2, H_q=16, S_q=8192, S_k=8192, D=64, causal=True, seed=2, backward=True)):
+        x = workloads.make_inputs(wb)
+        q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+        o, lse = attn.fwd(q, k, v, causal=True, scale=wb.scale)
+        if wb.D == 64:
+            ms = timed(lambda: attn.fwd(q, k, v, causal=True, scale=wb.scale, out=o, lse=lse))
+            print(f"forward {wb.name}: bf16 {ms:.3f} ms {wb.fwd_flops() / ms / 1e9:.0f} TFLOPS", flush=True)
+        ws = torch.empty(attn.bwd_workspace_size(wb.B, wb.H_q, wb.S_q, wb.D), dtype=torch.uint8, device="cuda")
+        grads = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
+        for det in (False, True):
+            ms = timed(lambda: attn.bwd(q, k, v, o, lse, do, causal=True, scale=wb.scale, dq=grads[0],
+                                        dk=grads[1], dv=grads[2], workspace=ws, deterministic=det))
+            print(f"backward {wb.name} deterministic={det}: {ms:.3f} ms {wb.bwd_flops() / ms / 1e9:.0f} TFLOPS",
+                  flush=True)
+        del q, k, v, do, o, lse, ws, grads, x
 
 
 def main():
