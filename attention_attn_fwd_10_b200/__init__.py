@@ -119,14 +119,17 @@ def fwd_split(q, k, v, causal: bool = False, scale: float | None = None, num_spl
               workspace=None, stream=None):
     """Split-KV forward (attn_fwd_split): the same (o, lse) as fwd, with the key
     blocks divided among ``num_splits`` ranges (0 = library default) whose partial
-    results are merged by the log-sum-exp identity.  Device tensors only."""
+    results are merged by the log-sum-exp identity.  q and k may both be
+    torch.float8_e4m3fn (attn_fwd_split_qk8, head dim 128).  Device tensors only."""
     B, S_q, H_q, S_k, H_kv, D = _shapes(q, k)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
-    _check_tensor("q", q, (B, S_q, H_q, D))
-    _check_tensor("k", k, (B, S_k, H_kv, D))
+    qk8 = q.dtype == torch.float8_e4m3fn
+    qk_dtype = torch.float8_e4m3fn if qk8 else torch.bfloat16
+    _check_tensor("q", q, (B, S_q, H_q, D), qk_dtype)
+    _check_tensor("k", k, (B, S_k, H_kv, D), qk_dtype)
     _check_tensor("v", v, (B, S_k, H_kv, D))
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty((B, S_q, H_q, D), dtype=torch.bfloat16, device=q.device)
     if lse is None:
         lse = torch.empty((B, H_q, S_q), dtype=torch.float32, device=q.device)
     _check_tensor("out", out, (B, S_q, H_q, D))
@@ -138,10 +141,11 @@ def fwd_split(q, k, v, causal: bool = False, scale: float | None = None, num_spl
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     if workspace is not None and workspace.numel() * workspace.element_size() < need:
         raise ValueError(f"workspace holds {workspace.numel() * workspace.element_size()} bytes, needs {need}")
-    code = lib.attn_fwd_split(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                              workspace.data_ptr() if workspace is not None else None, B, H_q, H_kv, S_q, S_k, D,
-                              int(bool(causal)), scale, n, _stream_ptr(stream))
-    _abi.check(code, "attn_fwd_split")
+    fn = lib.attn_fwd_split_qk8 if qk8 else lib.attn_fwd_split
+    code = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+              workspace.data_ptr() if workspace is not None else None, B, H_q, H_kv, S_q, S_k, D,
+              int(bool(causal)), scale, n, _stream_ptr(stream))
+    _abi.check(code, "attn_fwd_split_qk8" if qk8 else "attn_fwd_split")
     return out, lse
 
 

@@ -31,6 +31,7 @@ EXPORTED = (
     "attn_fwd_ex",
     "attn_fwd_qk8",
     "attn_fwd_split",
+    "attn_fwd_split_qk8",
     "attn_fwd_split_count",
     "attn_fwd_split_workspace_size",
     "attn_bwd_workspace_size",
@@ -74,6 +75,7 @@ _SIGNATURES = {
     "attn_fwd_qk8": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
                           ctypes.POINTER(FwdOptions), _vp]),
     "attn_fwd_split": (_i, [_vp] * 6 + [_i, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
+    "attn_fwd_split_qk8": (_i, [_vp] * 6 + [_i, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
     "attn_fwd_split_count": (_i, [_i, _i, _i, _i, _i, _i]),
     "attn_fwd_split_workspace_size": (ctypes.c_size_t, [_i, _i, _i, _i, _i]),
     "attn_bwd_workspace_size": (ctypes.c_size_t, [_i, _i, _i, _i]),

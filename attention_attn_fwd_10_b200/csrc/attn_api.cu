@@ -361,6 +361,15 @@ attn_status_t attn_fwd_qk8(const void* q, const void* k, const void* v, void* o,
   return run_fwd(q, k, v, o, lse, nullptr, B, H_q, H_kv, S_q, S_k, D, causal, scale, opt, 1, stream, true);
 }
 
+attn_status_t attn_fwd_split_qk8(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 void* workspace, int B, int H_q, int H_kv, int S_q, int S_k, int D, int causal,
+                                 float scale, int n_splits, void* stream) {
+  if (n_splits < 0 || n_splits > kMaxSplits) return ATTN_ERR_INVALID_ARG;
+  if (n_splits == 0) n_splits = attn_fwd_split_count(B, H_q, H_kv, S_q, S_k, causal);
+  return run_fwd(q, k, v, o, lse, workspace, B, H_q, H_kv, S_q, S_k, D, causal, scale, nullptr, n_splits, stream,
+                 true);
+}
+
 size_t attn_fwd_split_workspace_size(int B, int H_q, int S_q, int D, int n_splits) {
   if (B < 1 || H_q < 1 || S_q < 1 || (D != 64 && D != 128) || n_splits < 1 || n_splits > kMaxSplits) return 0;
   if (n_splits == 1) return 0;

@@ -512,13 +512,16 @@ def run_variants(args):
         w = workloads.small(B=B, H_q=H_q, H_kv=H_kv, S_q=S_q, S_k=S_k, D=128, causal=True, seed=1)
         x = workloads.make_inputs(w)
         q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+        q8, k8 = q.to(torch.float8_e4m3fn), k.to(torch.float8_e4m3fn)
         ms_plain = timed(lambda: attn.fwd(q, k, v, causal=True, scale=w.scale))
         ms_split = timed(lambda: attn.fwd_split(q, k, v, causal=True, scale=w.scale))
+        ms_split8 = timed(lambda: attn.fwd_split(q8, k8, v, causal=True, scale=w.scale))
         kv_bytes = 2 * B * S_k * H_kv * 128 * 2
         n = attn.fwd_split_count(B, H_q, H_kv, S_q, S_k, True)
         print(f"decode B{B} H_q{H_q} H_kv{H_kv} S_q{S_q} S_k{S_k}: forward {ms_plain * 1e3:.1f} us | "
-              f"split-KV ({n} ranges) {ms_split * 1e3:.1f} us, K+V {kv_bytes / ms_split / 1e9:.2f} TB/s", flush=True)
-        del q, k, v, x
+              f"split-KV ({n} ranges) {ms_split * 1e3:.1f} us, K+V {kv_bytes / ms_split / 1e9:.2f} TB/s | "
+              f"split-KV with e4m3 Q/K {ms_split8 * 1e3:.1f} us", flush=True)
+        del q, k, v, q8, k8, x
     for wb in (workloads.BWD_CAUSAL,
                workloads.small(B=2, H_q=16, S_q=8192, S_k=8192, D=64, causal=True, seed=2, backward=True)):
         x = workloads.make_inputs(wb)

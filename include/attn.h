@@ -131,6 +131,14 @@ attn_status_t attn_fwd_split(const void* q, const void* k, const void* v, void* 
                              int B, int H_q, int H_kv, int S_q, int S_k, int D, int causal, float scale,
                              int n_splits, void* stream);
 
+/* attn_fwd_split with 8-bit Q and K as in attn_fwd_qk8 (q, k e4m3; v, o bf16; head
+ * dim 128): for decoding shapes, where the step is bound by streaming K and V,
+ * e4m3 K moves half the bytes of bf16 K.  Arguments, workspace and errors as
+ * attn_fwd_split. */
+attn_status_t attn_fwd_split_qk8(const void* q, const void* k, const void* v, void* o, float* lse,
+                                 void* workspace, int B, int H_q, int H_kv, int S_q, int S_k, int D, int causal,
+                                 float scale, int n_splits, void* stream);
+
 /* The n_splits attn_fwd_split uses for n_splits = 0: 1 when the forward's CTAs
  * (one per 256 query rows of a (batch, head), or of a pack of the query heads of one
  * kv group when S_q <= 128) already fill the 148 SMs; otherwise the count (at most

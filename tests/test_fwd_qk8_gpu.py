@@ -57,3 +57,19 @@ def test_causal_config_sampled(poly):
         parity.check_o(o_c[b, rows, h, :], o_ref, f"{w.name} b={b} h={h}")
         parity.check_lse(lse_c[b, h, rows], lse_ref, f"{w.name} b={b} h={h}")
     assert torch.isfinite(o_c.float()).all() and torch.isfinite(lse_c).all()
+
+
+@pytest.mark.parametrize("S_q,S_k,H_q,H_kv", [(1, 4096, 32, 8), (16, 3000, 8, 2), (100, 1000, 4, 4)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_split_kv_decode_shapes(S_q, S_k, H_q, H_kv, causal):
+    import attention_attn_fwd_10_b200 as attn
+
+    w = workloads.small(B=2, H_q=H_q, H_kv=H_kv, S_q=S_q, S_k=S_k, D=128, causal=causal, seed=S_q + S_k)
+    x = workloads.make_inputs(w)
+    q8, k8 = x["q"].to(torch.float8_e4m3fn), x["k"].to(torch.float8_e4m3fn)
+    o, lse = attn.fwd_split(q8.cuda(), k8.cuda(), x["v"].cuda(), causal=causal, scale=w.scale)
+    torch.cuda.synchronize()
+    assert attn.device_status() == 0
+    o_ref, lse_ref = ref.forward(q8.float(), k8.float(), x["v"], causal, w.scale)
+    parity.check_o(o, o_ref, w.name)
+    parity.check_lse(lse, lse_ref, w.name)
