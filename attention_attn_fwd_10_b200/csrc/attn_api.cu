@@ -265,7 +265,9 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   p.status = status;
   p.rescale_count = opt.rescale_count;
   p.wait_limit_ns = g_wait_limit_ns.load();
-  const unsigned grid = static_cast<unsigned>(p.n_units) * B * (H_q / gp) * n_splits;
+  const long long grid_ll = static_cast<long long>(p.n_units) * B * (H_q / gp) * n_splits;
+  if (grid_ll > 2147483647LL) return ATTN_ERR_UNSUPPORTED;  // one CTA per (unit, head pack, range)
+  const unsigned grid = static_cast<unsigned>(grid_ll);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t err;
   if (qk8)
