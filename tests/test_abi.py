@@ -132,3 +132,24 @@ def test_fwd_qk8_rejects_bad_arguments(lib):
     assert lib.attn_fwd_qk8(*p, 1, 2, 2, 8, 8, 64, 0, 0.125, None, None) == 2   # head dim 64: unsupported
     assert lib.attn_fwd_qk8(*p, 1, 3, 2, 8, 8, 128, 0, 0.125, None, None) == 1  # H_q % H_kv != 0
     assert lib.attn_fwd_qk8(16, 32, 48, None, 80, 1, 2, 2, 8, 8, 128, 0, 0.125, None, None) == 1
+
+
+def test_header_is_c99_and_links(lib, tmp_path):
+    """include/attn.h compiles as C99, every declared entry point resolves at link
+    time, and a C program can call the host-only entry points."""
+    import shutil
+    import subprocess
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    exe = tmp_path / "abi_consumer"
+    lib_dir = os.path.join(ROOT, "attention_attn_fwd_10_b200")
+    cmd = [gcc, "-std=c99", "-Wall", "-Werror", "-pedantic-errors", "-Wno-pedantic",
+           "-I", os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c", "abi_consumer.c"),
+           "-L", lib_dir, "-lattn", f"-Wl,-rpath,{lib_dir}", "-o", str(exe)]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert run.returncode == 0, (run.returncode, run.stdout, run.stderr)
+    assert "abi 2" in run.stdout
