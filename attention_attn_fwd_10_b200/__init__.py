@@ -28,9 +28,30 @@ __all__ = ["fwd", "fwd_qk8", "fwd_split", "fwd_split_count", "bwd", "fwd_bwd", "
            "load", "status_string"]
 
 
-def _stream_ptr(stream) -> int:
-    s = torch.cuda.current_stream() if stream is None else stream
-    return s.cuda_stream
+def _stream_ptr(stream, device=None) -> int:
+    """The raw cudaStream_t of ``stream`` (default: the current stream of
+    ``device``), which must belong to ``device``."""
+    if stream is None:
+        return torch.cuda.current_stream(device).cuda_stream
+    if device is not None and stream.device != torch.device(device):
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
+    return stream.cuda_stream
+
+
+def _device_of(*tensors) -> torch.device:
+    """The one CUDA device every given tensor lives on (the library's kernels run
+    on the current device and must only be handed its memory)."""
+    dev = None
+    for t in tensors:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("every tensor of a call must be a CUDA tensor")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"tensors on different devices ({dev} and {t.device}): all must be on one device")
+    return dev
 
 
 def _check_tensor(name, t, shape, dtype=torch.bfloat16):
@@ -75,11 +96,13 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse
         lse = torch.empty((B, H_q, S_q), dtype=torch.float32, device=q.device)
     _check_tensor("out", out, (B, S_q, H_q, D))
     _check_tensor("lse", lse, (B, H_q, S_q), torch.float32)
+    dev = _device_of(q, k, v, out, lse, rescale_count)
     opt = FwdOptions(float(rescale_threshold), int(poly_exp_every),
                      rescale_count.data_ptr() if rescale_count is not None else None)
-    code = load().attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                              B, H_q, H_kv, S_q, S_k, D, int(bool(causal)), scale, ctypes.byref(opt),
-                              _stream_ptr(stream))
+    with torch.cuda.device(dev):
+        code = load().attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                  B, H_q, H_kv, S_q, S_k, D, int(bool(causal)), scale, ctypes.byref(opt),
+                                  _stream_ptr(stream, dev))
     _abi.check(code, "attn_fwd")
     if on_host:
         return out.cpu(), lse.cpu()
@@ -102,10 +125,12 @@ def fwd_qk8(q, k, v, causal: bool = False, scale: float | None = None, out=None,
         lse = torch.empty((B, H_q, S_q), dtype=torch.float32, device=q.device)
     _check_tensor("out", out, (B, S_q, H_q, D))
     _check_tensor("lse", lse, (B, H_q, S_q), torch.float32)
+    dev = _device_of(q, k, v, out, lse)
     opt = FwdOptions(float(rescale_threshold), int(poly_exp_every), None)
-    code = load().attn_fwd_qk8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                               B, H_q, H_kv, S_q, S_k, D, int(bool(causal)), scale, ctypes.byref(opt),
-                               _stream_ptr(stream))
+    with torch.cuda.device(dev):
+        code = load().attn_fwd_qk8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                   B, H_q, H_kv, S_q, S_k, D, int(bool(causal)), scale, ctypes.byref(opt),
+                                   _stream_ptr(stream, dev))
     _abi.check(code, "attn_fwd_qk8")
     return out, lse
 
@@ -141,10 +166,12 @@ def fwd_split(q, k, v, causal: bool = False, scale: float | None = None, num_spl
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     if workspace is not None and workspace.numel() * workspace.element_size() < need:
         raise ValueError(f"workspace holds {workspace.numel() * workspace.element_size()} bytes, needs {need}")
+    dev = _device_of(q, k, v, out, lse, workspace)
     fn = lib.attn_fwd_split_qk8 if qk8 else lib.attn_fwd_split
-    code = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-              workspace.data_ptr() if workspace is not None else None, B, H_q, H_kv, S_q, S_k, D,
-              int(bool(causal)), scale, n, _stream_ptr(stream))
+    with torch.cuda.device(dev):
+        code = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                  workspace.data_ptr() if workspace is not None else None, B, H_q, H_kv, S_q, S_k, D,
+                  int(bool(causal)), scale, n, _stream_ptr(stream, dev))
     _abi.check(code, "attn_fwd_split_qk8" if qk8 else "attn_fwd_split")
     return out, lse
 
@@ -182,19 +209,22 @@ def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, d
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     if workspace.numel() * workspace.element_size() < need or not workspace.is_cuda:
         raise ValueError(f"workspace must be a CUDA buffer of at least {need} bytes")
+    dev = _device_of(q, k, v, o, lse, do, dq, dk, dv, workspace)
     opt = None
-    if main_pass_events is not None or deterministic:
-        ev = (None, None)
-        if main_pass_events is not None:
-            s = torch.cuda.current_stream() if stream is None else stream
-            for e in main_pass_events:
-                if e.cuda_event == 0:  # torch creates the CUDA event lazily, on its first record
-                    e.record(s)
-            ev = (main_pass_events[0].cuda_event, main_pass_events[1].cuda_event)
-        opt = ctypes.byref(_abi.BwdOptions(ev[0], ev[1], int(bool(deterministic))))
-    code = load().attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
-                              dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
-                              B, H_q, H_kv, S_q, S_k, D, int(bool(causal)), scale, opt, _stream_ptr(stream))
+    with torch.cuda.device(dev):
+        if main_pass_events is not None or deterministic:
+            ev = (None, None)
+            if main_pass_events is not None:
+                s = torch.cuda.current_stream(dev) if stream is None else stream
+                for e in main_pass_events:
+                    if e.cuda_event == 0:  # torch creates the CUDA event lazily, on its first record
+                        e.record(s)
+                ev = (main_pass_events[0].cuda_event, main_pass_events[1].cuda_event)
+            opt = ctypes.byref(_abi.BwdOptions(ev[0], ev[1], int(bool(deterministic))))
+        code = load().attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                  do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                                  B, H_q, H_kv, S_q, S_k, D, int(bool(causal)), scale, opt,
+                                  _stream_ptr(stream, dev))
     _abi.check(code, "attn_bwd")
     if on_host:
         return dq.cpu(), dk.cpu(), dv.cpu()
@@ -298,8 +328,11 @@ class FwdBwdPipeline:
 
 
 def device_status(stream=None) -> int:
-    """Synchronise the stream; return (and clear) the kernels' device status code."""
-    return int(load().attn_device_status(_stream_ptr(stream)))
+    """Read and clear the current device's status word after the stream's work;
+    returns the code (0 = OK).  The word is shared by every stream of the device."""
+    dev = stream.device if stream is not None else torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        return int(load().attn_device_status(_stream_ptr(stream, dev)))
 
 
 def set_wait_limit_ns(ns: int) -> None:
@@ -311,6 +344,7 @@ def exp2_poly_eval(x: torch.Tensor, stream=None) -> torch.Tensor:
     if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
         raise ValueError("x must be a contiguous CUDA float32 tensor")
     y = torch.empty_like(x)
-    _abi.check(load().attn_exp2_poly_eval(x.data_ptr(), y.data_ptr(), x.numel(), _stream_ptr(stream)),
-               "attn_exp2_poly_eval")
+    with torch.cuda.device(x.device):
+        _abi.check(load().attn_exp2_poly_eval(x.data_ptr(), y.data_ptr(), x.numel(), _stream_ptr(stream, x.device)),
+                   "attn_exp2_poly_eval")
     return y

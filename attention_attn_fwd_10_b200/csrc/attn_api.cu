@@ -18,6 +18,8 @@ namespace attn {
 
 // Device status word: kernels record kDevWaitTimeout here when they abandon a wait.
 __device__ int g_status = 0;
+// Where attn_device_status() puts the word it read (and cleared) in one atomic step.
+__device__ int g_status_taken = 0;
 
 // Fixed scratch for attn_bwd_noalloc: every device that loads this library
 // holds these bytes until the process exits.  Host code must not pass the
@@ -100,36 +102,93 @@ bool make_dqacc_map(CUtensorMap* map, void* ptr, int B, int S, int H, int D) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int* status_ptr() {
-  static int* ptr = nullptr;
-  static std::mutex mu;
-  std::lock_guard<std::mutex> lock(mu);
-  int dev = -1;
-  static int ptr_dev = -2;
-  cudaGetDevice(&dev);
-  if (ptr == nullptr || ptr_dev != dev) {
-    void* sym = nullptr;
-    if (cudaGetSymbolAddress(&sym, g_status) != cudaSuccess) return nullptr;
-    ptr = static_cast<int*>(sym);
-    ptr_dev = dev;
-  }
-  return ptr;
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+// The calling thread's current CUDA context (the runtime's primary context of
+// the current device once the runtime has initialised it), or nullptr.
+CUcontext current_ctx() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  CUcontext c = nullptr;
+  if (fn == nullptr || fn(&c) != CUDA_SUCCESS) return nullptr;
+  return c;
 }
 
-// Device address of g_bwd_scratch on the current device (looked up once per device).
-void* noalloc_scratch_ptr() {
-  constexpr int kMaxDevices = 64;
-  static void* ptrs[kMaxDevices] = {};
-  static std::mutex mu;
+constexpr int kMaxDevices = 64;
+
+// Per-device state of the library: device addresses of its __device__ symbols,
+// valid in the context they were looked up in.  A device reset (or anything else
+// that replaces the device's context) invalidates them; they are looked up again
+// when the current context is not the recorded one.
+struct DevState {
+  CUcontext ctx = nullptr;
+  int* status = nullptr;  // g_status
+  int* taken = nullptr;   // g_status_taken
+  void* scratch = nullptr;  // g_bwd_scratch (looked up on first use)
+};
+std::mutex g_dev_mu;
+DevState g_dev[kMaxDevices];
+
+// Current device's state, refreshed if the context changed.  `with_scratch` also
+// resolves the no-allocation backward's scratch buffer.
+bool device_state(DevState* out, bool with_scratch = false) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (ptrs[dev] == nullptr) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) != cudaSuccess) return nullptr;
-    ptrs[dev] = ptr;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DevState& s = g_dev[dev];
+  CUcontext ctx = current_ctx();
+  if (ctx == nullptr || ctx != s.ctx) {
+    void* st = nullptr;
+    void* tk = nullptr;
+    if (cudaGetSymbolAddress(&st, g_status) != cudaSuccess) return false;
+    if (cudaGetSymbolAddress(&tk, g_status_taken) != cudaSuccess) return false;
+    s = DevState{};
+    s.status = static_cast<int*>(st);
+    s.taken = static_cast<int*>(tk);
+    s.ctx = current_ctx();  // the lookup above initialised the context if it was not yet
   }
-  return ptrs[dev];
+  if (with_scratch && s.scratch == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_bwd_scratch) != cudaSuccess) return false;
+    s.scratch = ptr;
+  }
+  *out = s;
+  return true;
+}
+
+int* status_ptr() {
+  DevState s;
+  return device_state(&s) ? s.status : nullptr;
+}
+
+// Device address of g_bwd_scratch on the current device (looked up once per
+// device and context).
+void* noalloc_scratch_ptr() {
+  DevState s;
+  return device_state(&s, true) ? s.scratch : nullptr;
+}
+
+// The dynamic shared-memory opt-in of a kernel is an attribute of the current
+// device's context: set it once per (kernel, context).  `seen` is the kernel's
+// own record of the contexts it was set in, one slot per device.
+std::mutex g_attr_mu;
+template <typename Kern>
+cudaError_t smem_opt_in(Kern kern, int bytes, CUcontext* seen) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  const CUcontext ctx = current_ctx();
+  if (ctx != nullptr && seen[dev] == ctx) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) seen[dev] = current_ctx();
+  return e;
 }
 
 attn_status_t check_common(int B, int H_q, int H_kv, int S_q, int S_k, int D, int causal, float scale) {
@@ -150,11 +209,8 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
                        unsigned grid, cudaStream_t st) {
   using L = FwdLayout<D, QK8>;
   auto kern = attn_fwd_kernel<D, CAUSAL, POLY, QK8>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
-  });
+  static CUcontext seen[kMaxDevices] = {};
+  const cudaError_t attr_err = smem_opt_in(kern, L::SMEM_BYTES, seen);
   if (attr_err != cudaSuccess) return attr_err;
   kern<<<grid, L::THREADS, L::SMEM_BYTES, st>>>(mq, mk, mv, p);
   return cudaGetLastError();
@@ -175,15 +231,16 @@ cudaError_t launch_bwd(const CUtensorMap& mk, const CUtensorMap& mv, const CUten
                        const CUtensorMap& mdq, const BwdParams& p, unsigned grid, cudaStream_t st) {
   using L = BwdLayout<D, DET>;
   auto kern = attn_bwd_kernel<D, CAUSAL, DET>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [&] {
-    attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM_BYTES);
-  });
+  static CUcontext seen[kMaxDevices] = {};
+  const cudaError_t attr_err = smem_opt_in(kern, L::SMEM_BYTES, seen);
   if (attr_err != cudaSuccess) return attr_err;
   kern<<<grid, L::THREADS, L::SMEM_BYTES, st>>>(mk, mv, mq, mdo, mdq, p);
   return cudaGetLastError();
 }
+
+// Reads and clears the status word in one atomic step (a timeout recorded by a
+// kernel on another stream is never lost between a read and a clear).
+__global__ void take_status_kernel(int* status, int* taken) { *taken = atomicExch(status, 0); }
 
 // Evaluates the kernels' packed-pair cubic on x[2i], x[2i+1] (the last element of
 // an odd-length array is paired with itself).
@@ -395,7 +452,7 @@ size_t attn_bwd_workspace_size(int B, int H_q, int S_q, int D) {
   const size_t dq_acc = static_cast<size_t>(B) * S_q * H_q * D * sizeof(float);
   const size_t rows = static_cast<size_t>(B) * H_q * s_pad * sizeof(float);
   const size_t sems = static_cast<size_t>(B) * H_q * (s_pad / 64) * sizeof(int);
-  return (dq_acc + 255) / 256 * 256 + 2 * ((rows + 255) / 256 * 256) + (sems + 255) / 256 * 256;
+  return (dq_acc + 255) / 256 * 256 + 2 * ((rows + 255) / 256 * 256) + (sems + 255) / 256 * 256 + 256;
 }
 
 attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -423,6 +480,8 @@ attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const voi
   p.nlse2 = reinterpret_cast<float*>(ws + dq_bytes);
   p.delta = reinterpret_cast<float*>(ws + dq_bytes + row_bytes);
   p.dq_sem = reinterpret_cast<int*>(ws + dq_bytes + 2 * row_bytes);
+  const size_t sem_bytes = (static_cast<size_t>(B) * H_q * (s_pad / 64) * sizeof(int) + 255) / 256 * 256;
+  p.ticket = reinterpret_cast<int*>(ws + dq_bytes + 2 * row_bytes + sem_bytes);
   const bool det = opt && opt->deterministic;
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
@@ -509,15 +568,17 @@ attn_status_t attn_bwd_noalloc(const void* q, const void* k, const void* v, cons
 }
 
 attn_status_t attn_device_status(void* stream) {
+  // One caller at a time: the read-out slot g_status_taken is shared.
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
-  int* status = status_ptr();
-  if (!status) return ATTN_ERR_CUDA;
+  DevState ds;
+  if (!device_state(&ds)) return ATTN_ERR_CUDA;
+  take_status_kernel<<<1, 1, 0, s>>>(ds.status, ds.taken);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   int host = 0;
-  if (cudaMemcpy(&host, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
-  const int zero = 0;
-  if (host != 0 && cudaMemcpy(status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
-    return ATTN_ERR_CUDA;
+  if (cudaMemcpyAsync(&host, ds.taken, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return ATTN_ERR_CUDA;
   return host == 0 ? ATTN_OK : static_cast<attn_status_t>(host);
 }
 

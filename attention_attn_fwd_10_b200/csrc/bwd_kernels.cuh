@@ -42,6 +42,13 @@
 
 #include "sm100_common.cuh"
 
+#ifndef ATTN_BWD_INTERLEAVE
+#define ATTN_BWD_INTERLEAVE 0
+#endif
+#ifndef ATTN_BWD_DQ_DIRECT
+#define ATTN_BWD_DQ_DIRECT 0
+#endif
+
 namespace attn {
 
 struct BwdParams {
@@ -52,6 +59,7 @@ struct BwdParams {
   float* nlse2;             // [B, H_q, S_pad] = -lse * log2(e); -inf for padding / empty rows (workspace)
   float* delta;             // [B, H_q, S_pad] (workspace)
   int* dq_sem;              // [B, H_q, S_pad / 64] dQ turn counters (workspace; deterministic mode)
+  int* ticket;              // work-item counter of the deterministic main pass (workspace)
   __nv_bfloat16* dq;        // [B, S_q, H_q, D]
   __nv_bfloat16* dk;        // [B, S_k, H_kv, D]
   __nv_bfloat16* dv;        // [B, S_k, H_kv, D]
@@ -104,6 +112,7 @@ __global__ void __launch_bounds__(256) attn_bwd_preprocess_kernel(const BwdParam
     for (int off = LANES / 2; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off, LANES);
     if (in_range && sub == 0 && (q & 63) == 0)
       p.dq_sem[(static_cast<size_t>(b) * p.H_q + h) * (p.S_pad / 64) + q / 64] = 0;
+    if (r0 == 0 && lane == 0) *p.ticket = 0;
     if (in_range && sub == 0) {
       const size_t r = (static_cast<size_t>(b) * p.H_q + h) * p.S_pad + q;
       float nl = -INFINITY;  // padding rows and rows that saw no key give P = 0
@@ -176,7 +185,8 @@ struct BwdLayout {
   static constexpr int N_BARS = B_S_FULL + 7 + 2 * NDQ;
   static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * N_BARS;
   static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 4;
-  static constexpr int SMEM_USED = ABORT_OFF + 4;
+  static constexpr int TICKET_OFF = ABORT_OFF + 4;
+  static constexpr int SMEM_USED = TICKET_OFF + 4;
   static constexpr int SMEM_BYTES = (SMEM_USED + 1024) > 122880 ? (SMEM_USED + 1024) : 122880;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   // tensor memory columns (512): S^T 64 | dP^T 64 | P^T 32 | dS^T 32 | dV D | dK D | dQ^T 64
@@ -212,30 +222,13 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work decode: groups of bh_group (batch, kv head) pairs run together, so
-  // the dQ accumulator rows and Q / dO tiles they share stay in L2; inside a
-  // group, causal tiles with the most query blocks (low key index) come first
-  const int BH = p.B * p.H_kv;
-  const int per_group = p.bh_group * p.n_kv_tiles;
-  const int grp = blockIdx.x / per_group;
-  const int within = blockIdx.x - grp * per_group;
-  const int gs = min(p.bh_group, BH - grp * p.bh_group);
-  // deterministic instance: highest key tile first (see the dQ reduce below)
-  const int j = DET ? p.n_kv_tiles - 1 - within / gs : within / gs;
-  const int bh = grp * p.bh_group + (within % gs);
-  const int b = bh / p.H_kv;
-  const int hkv = bh - b * p.H_kv;
-  const int G = p.H_q / p.H_kv;
-  const int k0 = j * L::BN;
-  const int diag = p.S_k - p.S_q;  // key k visible to query q iff k <= q + diag
-  const int n_qb = p.S_pad / L::BQ;
-  int qb0 = 0;
-  if (CAUSAL) {
-    const int first_q = k0 - diag;  // first query that sees key k0
-    qb0 = first_q <= 0 ? 0 : min(n_qb, first_q / L::BQ);
-  }
-  const int per_head = n_qb - qb0;
-  const int m = G * per_head;  // query blocks this CTA visits
+  // Work item: the block index, or in the deterministic instance a ticket taken
+  // from a global counter when the CTA starts.  Items are ordered so that the
+  // dQ additions an item waits for belong to items with smaller numbers; with
+  // tickets those items were claimed by CTAs that had already started, so every
+  // wait ends whatever order the hardware dispatches the blocks in.
+  if (DET && threadIdx.x == 0)
+    *reinterpret_cast<volatile int*>(sptr + L::TICKET_OFF) = atomicAdd(p.ticket, 1);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::N_BARS; ++i)
@@ -258,6 +251,36 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sptr + L::TMEM_SLOT_OFF);
+
+  // ---- work decode: groups of bh_group (batch, kv head) pairs run together, so
+  // the dQ accumulator rows and Q / dO tiles they share stay in L2; inside a
+  // group, causal tiles with the most query blocks (low key index) come first
+  const int item = DET ? *reinterpret_cast<volatile int*>(sptr + L::TICKET_OFF) : static_cast<int>(blockIdx.x);
+  // A ticket beyond the grid would mean the counter was not reset before the
+  // launch: such a CTA touches nothing and records an error.
+  const bool live = item < static_cast<int>(gridDim.x);
+  if (!live && threadIdx.x == 0) atomicExch(p.status, kDevWaitTimeout);
+  const int BH = p.B * p.H_kv;
+  const int per_group = p.bh_group * p.n_kv_tiles;
+  const int grp = item / per_group;
+  const int within = item - grp * per_group;
+  const int gs = min(p.bh_group, BH - grp * p.bh_group);
+  // deterministic instance: highest key tile first (see the dQ reduce below)
+  const int j = DET ? p.n_kv_tiles - 1 - within / gs : within / gs;
+  const int bh = grp * p.bh_group + (within % gs);
+  const int b = bh / p.H_kv;
+  const int hkv = bh - b * p.H_kv;
+  const int G = p.H_q / p.H_kv;
+  const int k0 = j * L::BN;
+  const int diag = p.S_k - p.S_q;  // key k visible to query q iff k <= q + diag
+  const int n_qb = p.S_pad / L::BQ;
+  int qb0 = 0;
+  if (CAUSAL) {
+    const int first_q = k0 - diag;  // first query that sees key k0
+    qb0 = first_q <= 0 ? 0 : min(n_qb, first_q / L::BQ);
+  }
+  const int per_head = n_qb - qb0;
+  const int m = live ? G * per_head : 0;  // query blocks this CTA visits
 
 
   if (warp == L::WARP_TMA) {
@@ -303,6 +326,18 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
       const uint32_t k_base = sbase + L::K_OFF, v_base = sbase + L::V_OFF;
       auto issue_s_dp = [&](int st) {
         const uint32_t sb = sbase + L::STAGE_OFF + st * L::STAGE_BYTES;
+#if ATTN_BWD_INTERLEAVE
+        // S^T and dP^T instructions alternate (two independent accumulators)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ao = (kk >> 2) * L::KBOX_BYTES + (kk & 3) * 32;
+          const uint32_t bo = (kk >> 2) * L::QBOX_BYTES + (kk & 3) * 32;
+          umma_ss(tmem + L::X_COL, sdesc_sw128(k_base + ao, 16, 1024), sdesc_sw128(sb + L::ST_Q + bo, 16, 1024),
+                  IDESC_S, kk > 0 ? 1u : 0u);
+          umma_ss(tmem + L::Y_COL, sdesc_sw128(v_base + ao, 16, 1024), sdesc_sw128(sb + L::ST_DO + bo, 16, 1024),
+                  IDESC_S, kk > 0 ? 1u : 0u);
+        }
+#else
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ao = (kk >> 2) * L::KBOX_BYTES + (kk & 3) * 32;
@@ -317,6 +352,7 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
           umma_ss(tmem + L::Y_COL, sdesc_sw128(v_base + ao, 16, 1024), sdesc_sw128(sb + L::ST_DO + bo, 16, 1024),
                   IDESC_S, kk > 0 ? 1u : 0u);
         }
+#endif
         umma_commit(bar(L::B_S_FULL));
       };
       bool ok = mbar_wait(bar(L::B_KV_FULL), 0, ctl);
@@ -373,7 +409,7 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
     const int r = threadIdx.x & 127;   // key row == TMEM lane
     const int hc = threadIdx.x >> 7;   // query half: columns [32 hc, 32 hc + 32)
     const int key = k0 + r;
-    const bool valid_key = key < p.S_k;
+    const bool valid_key = live && key < p.S_k;
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
     bool ok = true;
@@ -496,6 +532,22 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
       tmem_ld_wait(v + 32);
       tc_fence_before();
       mbar_arrive_warp(bar(L::B_DQ_FREE));
+#if ATTN_BWD_DQ_DIRECT
+      if (!DET) {
+        // add dQ_i^T straight from registers: one coalesced fp32 reduction per query
+        const int h = hkv * G + i / per_head;
+        const int q0 = (qb0 + i % per_head) * L::BQ;
+        if (d >= 0) {
+          float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.S_q + q0) * p.H_q + h) * D + d;
+          const size_t qstride = static_cast<size_t>(p.H_q) * D;
+          const int nq = min(L::BQ, p.S_q - q0);
+#pragma unroll
+          for (int c = 0; c < L::BQ; ++c)
+            if (c < nq) red_add_f32(dst + c * qstride, __uint_as_float(v[c]));
+        }
+        continue;
+      }
+#endif
       const int buf = i % L::NDQ;
       if (i >= L::NDQ) {  // the reduce of block i - NDQ has read this tile
         ok = mbar_wait(bar(L::B_STAGE_FREE + buf), ((i / L::NDQ) - 1) & 1, ctl);
@@ -510,7 +562,7 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
     }
   } else if (warp == L::WARP_RED) {
     // ===================== dQ reduce issue: one TMA reduce-add per staged tile =====================
-    if (lane == 0) {
+    if (lane == 0 && (DET || !ATTN_BWD_DQ_DIRECT)) {
       for (int i = 0; i < m; ++i) {
         const int buf = i % L::NDQ;
         if (!mbar_wait(bar(L::B_STAGED + buf), (i / L::NDQ) & 1, ctl)) break;
@@ -520,8 +572,9 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
         // keys are visible to more queries).  They add their parts in the order J,
         // J - 1, ..., 0 -- the order in which they reach the block, since tile j
         // starts its sweep two blocks before tile j - 1 -- so tile j waits for
-        // J - j others.  The grid dispatches high tiles first, so tile j + 1 has
-        // the lower block index and is running or done: the wait always ends.
+        // J - j others.  High tiles have the smaller work-item numbers, so tile
+        // j + 1's item was claimed by a CTA that started before this one: it is
+        // running or done, and the wait always ends.
         int* sem = p.dq_sem + (static_cast<size_t>(b) * p.H_q + h) * (p.S_pad / 64) + qb;
         if (DET) {
           // J: the last tile whose first visited block, max(0, (128 J - diag) / 64), is <= qb

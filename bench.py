@@ -92,8 +92,9 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, interval_ms: int = 20):
         self.gpu = gpu_index
+        self.interval_ms = interval_ms
         self.proc = None
         self.file = None
 
@@ -102,7 +103,8 @@ class ClockSampler:
             self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+                 "-lms", str(self.interval_ms)], stdout=self.file, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)  # nvidia-smi starts sampling only after it has initialised
         except Exception:
             self.proc = None
         return self
@@ -291,6 +293,10 @@ def run_ours(args):
     e2e = run_e2e(args, attn, x, wf, wb, have_bwd, dev, world)
 
     peaks, peaks_src = measured_peaks()
+    configs = None
+    if world == 1 and not args.no_configs:
+        del q, k, v, do, o, lse, dq, dk, dv, ws
+        configs = run_configs(attn, dev, flush, peaks)
     fwd_tf = wf.fwd_flops() / (fwd_ms * 1e-3) / 1e12
     bwd_tf = wb.bwd_flops() / (bwd_ms * 1e-3) / 1e12 if have_bwd else None
     # dominant kernel: the one with the larger share of the step
@@ -333,6 +339,7 @@ def run_ours(args):
                      "traffic": captured_traffic("attn_bwd_kernel" if dom.startswith("attn_bwd") else "attn_fwd_kernel"),
                      "traffic_unit": "bytes per launch (ncu dram read + write)"},
         "e2e": e2e,
+        "configs": configs,
         "gpu_launches": args.steps * (1 + (3 if have_bwd else 0)),
         "clocks": clocks,
     }
@@ -405,9 +412,142 @@ def run_e2e(args, attn, x, wf, wb, have_bwd, dev, world):
         mode = "sequential"
     step_ms = max_over_ranks(world, step_ms)
     flops = wf.fwd_flops() + (wb.bwd_flops() if have_bwd else 0.0)
-    return {"value": round(world * flops / (step_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
-            "ms_per_step": round(step_ms, 3), "steps": n_steps, "mode": mode,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    res = {"value": round(world * flops / (step_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
+           "ms_per_step": round(step_ms, 3), "steps": n_steps, "mode": mode,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    if have_bwd:
+        # the latency one call sees: attn.fwd_bwd uploads the step's inputs, runs the
+        # forward and the backward, downloads every result and synchronises, nothing overlapped
+        for _ in range(2):
+            attn.fwd_bwd(hq, hk, hv, hdo, causal=wf.causal, scale=wf.scale, host_out=host_out)
+        ms = []
+        for _ in range(n_steps):
+            barrier(world)
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            attn.fwd_bwd(hq, hk, hv, hdo, causal=wf.causal, scale=wf.scale, host_out=host_out)
+            e1.record()
+            torch.cuda.synchronize()
+            ms.append(e0.elapsed_time(e1))
+        seq_ms = max_over_ranks(world, sum(ms) / len(ms))
+        res["sequential"] = {"value": round(world * flops / (seq_ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
+                             "ms_per_step": round(seq_ms, 3), "steps": n_steps,
+                             "mode": "one attn.fwd_bwd call per step: upload, kernels, download, in sequence"}
+    return res
+
+
+def timed_calls(fn, flush, stream, min_ms: float = 250.0, min_reps: int = 10, warmup: int = 3):
+    """Median device time (ms) of fn() over enough calls to span about min_ms of
+    kernel time, each call bracketed by CUDA events on `stream` with L2 flushed
+    before it (outside the events).  Returns (median_ms, reps)."""
+    import torch
+
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    est = max(e0.elapsed_time(e1), 1e-3)
+    reps = max(min_reps, int(math.ceil(min_ms / est)))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in evs:
+        flush.fill_(1)
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in evs), reps
+
+
+def run_configs(attn, dev, flush, peaks):
+    """Every forward configuration of the workload set, the split-KV decode shape
+    and the deterministic backward, each timed on its own (L2 flushed before each
+    call) with the SM clock sampled during its timed calls.  Returns a dict for
+    the JSON line's "configs" key."""
+    import torch
+
+    stream = torch.cuda.current_stream()
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    out = {}
+
+    def fwd_entry(w, extra=None):
+        x = workloads.make_inputs(w)
+        q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H_q, w.S_q), dtype=torch.float32, device=dev)
+        with ClockSampler(dev.index) as clk:
+            ms, reps = timed_calls(lambda: attn.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse),
+                                   flush, stream)
+        c = clk.summary()
+        tf = w.fwd_flops() / (ms * 1e-3) / 1e12
+        e = {"ms": round(ms, 4), "tflops": round(tf, 1), "frac_of_measured": round(tf / peak, 4),
+             "frac_of_spec_2250": round(tf / SPEC_PEAK_TFLOPS, 4), "reps": reps,
+             "sm_mhz": c["sm_mhz"], "clock_samples": c.get("samples"), "clock_reasons": c["reasons"]}
+        # O rescales counted at the default threshold (tau = 8) and with a rescale on
+        # every increase of the running max (tau = 0)
+        counts = {}
+        for tau in (8.0, 0.0):
+            cnt = torch.zeros(1, dtype=torch.int64, device=dev)
+            attn.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, rescale_threshold=tau,
+                     rescale_count=cnt)
+            counts[tau] = int(cnt.item())
+        e["rescale_count"] = {"tau8": counts[8.0], "tau0": counts[0.0],
+                              "tau0_over_tau8": round(counts[0.0] / counts[8.0], 1) if counts[8.0] else None}
+        if extra:
+            e.update(extra)
+        out[w.name] = e
+        del q, k, v, o, lse, x
+
+    for w in (workloads.FWD_NONCAUSAL, workloads.FWD_CAUSAL, workloads.FWD_CAUSAL_SPIKY, workloads.FWD_CAUSAL_GQA):
+        fwd_entry(w)
+
+    # decode: one query row per head against 32768 keys, split-KV forward (bytes-bound: K and V stream once)
+    w = workloads.small(B=1, H_q=32, H_kv=8, S_q=1, S_k=32768, D=128, causal=True, seed=1)
+    x = workloads.make_inputs(w)
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    n = attn.fwd_split_count(w.B, w.H_q, w.H_kv, w.S_q, w.S_k, True)
+    ws = torch.empty(attn.load().attn_fwd_split_workspace_size(w.B, w.H_q, w.S_q, w.D, n), dtype=torch.uint8,
+                     device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H_q, w.S_q), dtype=torch.float32, device=dev)
+    with ClockSampler(dev.index) as clk:
+        ms, reps = timed_calls(lambda: attn.fwd_split(q, k, v, causal=True, scale=w.scale, num_splits=n, out=o,
+                                                      lse=lse, workspace=ws), flush, stream)
+    c = clk.summary()
+    bytes_alg = sum(t.numel() * t.element_size() for t in (q, k, v, o, lse))
+    gbs = bytes_alg / (ms * 1e-3) / 1e9
+    out["decode_split_B1_Hq32_Hkv8_Sq1_Sk32768_D128"] = {
+        "us": round(ms * 1e3, 2), "gbs": round(gbs, 1), "frac_of_hbm": round(gbs / hbm, 4), "n_splits": n,
+        "algorithmic_bytes": bytes_alg, "reps": reps, "sm_mhz": c["sm_mhz"], "clock_samples": c.get("samples")}
+    del q, k, v, o, lse, ws, x
+
+    # the backward workload in its deterministic mode (fixed dQ order)
+    wb = workloads.BWD_CAUSAL
+    x = workloads.make_inputs(wb)
+    q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
+    o, lse = attn.fwd(q, k, v, causal=True, scale=wb.scale)
+    ws = torch.empty(attn.bwd_workspace_size(wb.B, wb.H_q, wb.S_q, wb.D), dtype=torch.uint8, device=dev)
+    g = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
+    for det in (False, True):
+        with ClockSampler(dev.index) as clk:
+            ms, reps = timed_calls(lambda: attn.bwd(q, k, v, o, lse, do, causal=True, scale=wb.scale, dq=g[0],
+                                                    dk=g[1], dv=g[2], workspace=ws, deterministic=det),
+                                   flush, stream)
+        c = clk.summary()
+        tf = wb.bwd_flops() / (ms * 1e-3) / 1e12
+        out[wb.name + ("_deterministic" if det else "")] = {
+            "ms": round(ms, 4), "tflops": round(tf, 1), "frac_of_measured": round(tf / peak, 4), "reps": reps,
+            "sm_mhz": c["sm_mhz"], "clock_samples": c.get("samples")}
+    del q, k, v, do, o, lse, ws, g, x
+    torch.cuda.synchronize()
+    if attn.device_status() != 0:
+        raise RuntimeError("device status not OK after the per-configuration measurements")
+    return out
 
 
 # --------------------------------------------------------------------------- reference arm (the oracle)
@@ -549,6 +689,7 @@ def main():
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="causal8k")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU time to sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration measurements")
     ap.add_argument("--profile", choices=("fwd", "bwd"), default=None,
                     help="only launch one pass W+K times (driver for ncu captures); prints no JSON")
     ap.add_argument("--variants", action="store_true",

@@ -18,7 +18,11 @@
  *   k, v, dk, dv : bf16 [B, S_k, H_kv, D]  contiguous
  *   lse          : fp32 [B, H_q, S_q]
  * Every pointer must be 16-byte aligned.  D is 64 or 128; H_q % H_kv == 0;
- * S_q, S_k >= 1; scale finite and > 0; causal is 0 or 1.
+ * S_q, S_k >= 1; scale finite and > 0; causal is 0 or 1.  Every device pointer
+ * of a call must point into the memory of the calling thread's current device
+ * (cudaSetDevice), and `stream` must belong to that device: the kernels run there
+ * and read their operands with TMA, which must never be handed another GPU's
+ * memory.
  *
  * Execution: calls enqueue work on `stream` (a cudaStream_t; NULL = legacy
  * default stream) and return without synchronising.  The return value reports
@@ -27,6 +31,12 @@
  * status word that attn_device_status() reads.  The library allocates no
  * device memory on any call: scratch space (the backward's workspace) is
  * passed in by the caller.  All entry points are thread-safe.
+ *
+ * Per-device state: the library caches, per device, the device addresses of
+ * its own __device__ variables and each kernel's shared-memory opt-in.  Both
+ * belong to the device's CUDA context; when the current context is no longer
+ * the one they were set up in (e.g. after cudaDeviceReset) the next call sets
+ * them up again.
  */
 #ifndef ATTN_B200_ATTN_H_
 #define ATTN_B200_ATTN_H_
@@ -154,8 +164,9 @@ size_t attn_fwd_split_workspace_size(int B, int H_q, int S_q, int D, int n_split
 /*
  * Bytes of device workspace attn_bwd needs: an fp32 dQ accumulator
  * [B, S_q, H_q, D], two fp32 row-term arrays [B, H_q, S_pad] (S_pad =
- * S_q rounded up to 64): -lse_i * log2(e) and delta_i = sum_d dO_id O_id, and
- * one int per (b, h, 64-query block) for the deterministic mode's turn counters.
+ * S_q rounded up to 64): -lse_i * log2(e) and delta_i = sum_d dO_id O_id,
+ * one int per (b, h, 64-query block) for the deterministic mode's turn counters,
+ * and one int for its work-item counter (each part 256-byte aligned).
  * Returns 0 for invalid sizes.
  */
 size_t attn_bwd_workspace_size(int B, int H_q, int S_q, int D);
@@ -182,8 +193,11 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
  *   deterministic : 0 (default) = each key tile adds its dQ part for a query
  *       block as soon as it has it, so the fp32 sums (and the bf16 dQ) may
  *       differ in the last bits between runs.  1 = the parts for each (b, h,
- *       64-query block) are added in increasing key-tile order, one tile waiting
- *       (bounded) for the previous one's addition to complete.  dQ is then
+ *       64-query block) are added in a fixed key-tile order, one tile waiting
+ *       (bounded) for the previous one's addition to complete.  The CTAs take
+ *       their work items from a counter as they start, so that a tile only ever
+ *       waits for tiles whose CTAs started before it: progress does not depend
+ *       on the order in which the hardware dispatches the blocks.  dQ is then
  *       bitwise identical from run to run (the pages' atomic reductions, section
  *       7 item 3, leave the order open); dK, dV are deterministic in both modes.
  */
@@ -209,11 +223,14 @@ attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const voi
  * reach cudaMalloc.)
  *
  * The buffer is a file-scope device array of 32 MiB (33554432 bytes) that
- * every GPU which loads the library holds until the process exits.  Problems whose attn_bwd_workspace_size() exceeds it return
- * ATTN_ERR_SCRATCH_TOO_SMALL before anything is launched.  The first call on a
- * device looks up the buffer's device address (cudaGetSymbolAddress); make that
- * first call before any stream capture.  No call allocates or frees device
- * memory.  All calls share the one buffer and it keeps the last call's
+ * every GPU which loads the library holds until the process exits.  Problems
+ * whose attn_bwd_workspace_size() exceeds it return ATTN_ERR_SCRATCH_TOO_SMALL
+ * before anything is launched.  The first call on a device looks up the
+ * buffer's device address (cudaGetSymbolAddress); make that first call before
+ * any stream capture.  The address is kept per device and context: after the
+ * device's context is replaced (cudaDeviceReset) the next call looks it up
+ * again, so that call too should come before any capture.  No call allocates
+ * or frees device memory.  All calls share the one buffer and it keeps the last call's
  * contents (each call clears what must start at zero): calls that may overlap
  * on the GPU -- on different streams, or from different host threads -- race
  * on it and must be serialised by the caller.  Arguments and results as attn_bwd.
@@ -223,9 +240,14 @@ attn_status_t attn_bwd_noalloc(const void* q, const void* k, const void* v, cons
                                int S_q, int S_k, int D, int causal, float scale, void* stream);
 
 /*
- * Synchronises `stream`, then returns and clears the device status word:
- * ATTN_OK, or ATTN_ERR_DEVICE_TIMEOUT if a kernel gave up on a wait since the
- * last call, or ATTN_ERR_CUDA if the synchronisation itself failed.
+ * Reads and clears the current device's status word in one atomic step, on
+ * `stream` (so after every kernel enqueued on it before), then synchronises
+ * `stream` and returns the value read: ATTN_OK, or ATTN_ERR_DEVICE_TIMEOUT if a
+ * kernel gave up on a wait since the last read, or ATTN_ERR_CUDA if a CUDA call
+ * failed.  There is one status word per device, shared by every stream: a
+ * timeout recorded by a kernel on another stream is reported by whichever read
+ * comes first after it, and a kernel still running on another stream may record
+ * one after this call returns.
  */
 attn_status_t attn_device_status(void* stream);
 

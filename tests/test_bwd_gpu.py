@@ -64,14 +64,36 @@ def test_medium_causal():
     _check(w, x, _gpu_fwd_bwd(x, True, w.scale))
 
 
-def test_backward_config_sampled_heads_and_invariants():
+# (batch, kv head) groups of the backward workload checked whole against the oracle:
+# the first and the last, and two in between (in the other batch entry)
+BWD_GROUPS = [(0, 0), (0, 9), (1, 6), (1, 15)]
+
+
+def _check_groups(w, x, grads, ref_by_group, what):
+    for (b, g), ref_g in zip(BWD_GROUPS, ref_by_group):
+        for name, gg, gr in zip(("dq", "dk", "dv"), grads, ref_g):
+            gg = parity.to_np(gg[b:b + 1, :, g:g + 1])
+            parity.check_grad(gg, gr, f"{w.name} {what} b={b} h_kv={g} {name}")
+
+
+def test_backward_config_groups_both_modes_and_invariants():
     w = workloads.BWD_CAUSAL
+    assert w.H_q == w.H_kv  # one query head per group: dq rows of group g are head g
     x = workloads.make_inputs(w)
-    dq, dk, dv = _gpu_fwd_bwd(x, w.causal, w.scale)
-    # whole (b, kv head) groups checked against the oracle: first and last
-    _check(w, x, (dq, dk, dv), groups=[0], batches=[0])
-    _check(w, x, (dq, dk, dv), groups=[w.H_kv - 1], batches=[w.B - 1])
+    attn = _attn()
+    q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
+    o, lse = attn.fwd(q, k, v, causal=True, scale=w.scale)
+    runs = {det: attn.bwd(q, k, v, o, lse, do, causal=True, scale=w.scale, deterministic=det)
+            for det in (False, True)}
+    torch.cuda.synchronize()
+    assert attn.device_status() == 0
+    ref_by_group = [[a[b:b + 1, :, g:g + 1].copy()
+                     for a in ref.backward(x["q"], x["k"], x["v"], x["do"], True, w.scale, groups=[g], batches=[b])]
+                    for (b, g) in BWD_GROUPS]
+    for det, grads in runs.items():
+        _check_groups(w, x, grads, ref_by_group, "deterministic" if det else "default")
     # properties at full size: sum over keys of dK is 0; sum over keys of dV = sum over queries of dO
+    dq, dk, dv = runs[False]
     dk64 = dk.double()
     assert torch.isfinite(dq.float()).all() and torch.isfinite(dk.float()).all() and torch.isfinite(dv.float()).all()
     assert dk64.sum(dim=1).abs().max() <= 3e-2 * dk64.abs().max() * w.S_k ** 0.5
@@ -128,9 +150,8 @@ def test_deterministic_mode_head_dim_64():
     _check(w, x, g1)
 
 
-def test_deterministic_mode_backward_config():
+def test_deterministic_mode_backward_config_repeats_bitwise():
     w = workloads.BWD_CAUSAL
     x, (g1, g2) = _bwd_twice(w, True)
     for a, b_ in zip(g1, g2):
         assert torch.equal(a, b_)
-    _check(w, x, g1, groups=[0], batches=[0])

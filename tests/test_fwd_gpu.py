@@ -74,36 +74,50 @@ def test_noncausal_config_full():
     parity.check_lse(lse, lse_ref, w.name)
 
 
-def _sampled(w, o, lse, x, heads, rows):
+def _sampled(w, o, lse, x, heads, rows_of):
+    """Check the rows rows_of(b, h) of every listed (b, h) against the oracle, row by row
+    (each output row depends only on its own query row and the keys)."""
     o_c, lse_c = o.cpu(), lse.cpu()
     vmax = float(x["v"].float().abs().max()) if w.spiky_keys else None
     for (b, h) in heads:
+        rows = rows_of(b, h)
         o_ref, lse_ref = ref.forward_rows(x["q"], x["k"], x["v"], w.causal, w.scale, b, h, rows)
         parity.check_o(o_c[b, rows, h, :], o_ref, f"{w.name} b={b} h={h}", v_absmax=vmax)
         parity.check_lse(lse_c[b, h, rows], lse_ref, f"{w.name} b={b} h={h}")
     assert torch.isfinite(o_c.float()).all() and torch.isfinite(lse_c).all()
 
 
-def _rows(S, n=48, seed=0):
-    g = np.random.default_rng(seed)
-    fixed = [0, 1, 127, 128, 129, S // 2, S - 129, S - 128, S - 1]
-    return sorted(set(fixed) | set(g.choice(S, n, replace=False).tolist()))
+def _unit_rows(S, n_random=64, seed=0):
+    """Rows of one head to check: its whole first and last 256-row work unit (the
+    longest and shortest causal units, and the diagonal blocks of both), plus
+    n_random rows drawn uniformly from the rest."""
+    def rows_of(b, h):
+        g = np.random.default_rng(seed + 1000 * b + h)
+        ends = set(range(0, min(256, S))) | set(range(max(0, S - 256), S))
+        rest = np.setdiff1d(np.arange(S), np.fromiter(ends, dtype=np.int64))
+        pick = g.choice(rest, min(n_random, len(rest)), replace=False).tolist() if len(rest) else []
+        return sorted(ends | set(pick))
+    return rows_of
+
+
+def _all_heads(w):
+    return [(b, h) for b in range(w.B) for h in range(w.H_q)]
 
 
 @pytest.mark.parametrize("w", [workloads.FWD_CAUSAL, workloads.FWD_CAUSAL_SPIKY], ids=lambda w: w.name)
-def test_causal_config_sampled(w):
+def test_causal_config_every_head(w):
     cnt = torch.zeros(1, dtype=torch.int64, device="cuda")
     x, o, lse = _run(w, rescale_count=cnt)
-    _sampled(w, o, lse, x, [(0, 0), (1, 15), (1, 7)], _rows(w.S_q))
+    _sampled(w, o, lse, x, _all_heads(w), _unit_rows(w.S_q))
     if w.spiky_keys:
         assert int(cnt.item()) > 0  # the spiky keys exercise the rescale path
 
 
-def test_gqa_long_config_sampled():
+def test_gqa_long_config_every_head():
     w = workloads.FWD_CAUSAL_GQA
     x, o, lse = _run(w)
-    # one full GQA group (query heads 4..7 share key/value head 1) plus the last head
-    _sampled(w, o, lse, x, [(0, 4), (0, 5), (0, 6), (0, 7), (0, 31)], _rows(w.S_q, n=24))
+    # every query head: the four of each kv group share one key/value head
+    _sampled(w, o, lse, x, _all_heads(w), _unit_rows(w.S_q))
 
 
 def test_deterministic_and_overwrites_poison():

@@ -16,6 +16,7 @@ import pytest
 import torch
 
 import workloads
+from oracle import reference as oracle_ref
 from tests import parity
 
 pytestmark = pytest.mark.gpu
@@ -36,6 +37,7 @@ def test_noalloc_backward_matches_workspace_backward_on_two_calls():
     ref = attn.bwd(q, k, v, o, lse, do, causal=True, scale=w.scale)  # caller-provided workspace
     torch.cuda.synchronize()
     ref = [parity.to_np(g) for g in ref]
+    exact = oracle_ref.backward(x["q"], x["k"], x["v"], x["do"], True, w.scale)  # fp64 oracle
     stream = torch.cuda.current_stream().cuda_stream
     for _ in range(2):
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -44,8 +46,9 @@ def test_noalloc_backward_matches_workspace_backward_on_two_calls():
                                   w.B, w.H_q, w.H_kv, w.S_q, w.S_k, w.D, 1, ctypes.c_float(w.scale), stream)
         assert rc == 0, _abi.status_string(rc)
         assert lib.attn_device_status(stream) == 0
-        for name, g, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
-            parity.check_grad(g, r, f"noalloc {name}")
+        for name, g, r, e in zip(("dq", "dk", "dv"), (dq, dk, dv), ref, exact):
+            parity.check_grad(g, r, f"noalloc {name} vs attn_bwd")
+            parity.check_grad(g, e, f"noalloc {name} vs the oracle")
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
