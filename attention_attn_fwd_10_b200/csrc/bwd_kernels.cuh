@@ -42,13 +42,6 @@
 
 #include "sm100_common.cuh"
 
-#ifndef ATTN_BWD_INTERLEAVE
-#define ATTN_BWD_INTERLEAVE 0
-#endif
-#ifndef ATTN_BWD_DQ_DIRECT
-#define ATTN_BWD_DQ_DIRECT 0
-#endif
-
 namespace attn {
 
 struct BwdParams {
@@ -326,18 +319,6 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
       const uint32_t k_base = sbase + L::K_OFF, v_base = sbase + L::V_OFF;
       auto issue_s_dp = [&](int st) {
         const uint32_t sb = sbase + L::STAGE_OFF + st * L::STAGE_BYTES;
-#if ATTN_BWD_INTERLEAVE
-        // S^T and dP^T instructions alternate (two independent accumulators)
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ao = (kk >> 2) * L::KBOX_BYTES + (kk & 3) * 32;
-          const uint32_t bo = (kk >> 2) * L::QBOX_BYTES + (kk & 3) * 32;
-          umma_ss(tmem + L::X_COL, sdesc_sw128(k_base + ao, 16, 1024), sdesc_sw128(sb + L::ST_Q + bo, 16, 1024),
-                  IDESC_S, kk > 0 ? 1u : 0u);
-          umma_ss(tmem + L::Y_COL, sdesc_sw128(v_base + ao, 16, 1024), sdesc_sw128(sb + L::ST_DO + bo, 16, 1024),
-                  IDESC_S, kk > 0 ? 1u : 0u);
-        }
-#else
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ao = (kk >> 2) * L::KBOX_BYTES + (kk & 3) * 32;
@@ -352,7 +333,6 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
           umma_ss(tmem + L::Y_COL, sdesc_sw128(v_base + ao, 16, 1024), sdesc_sw128(sb + L::ST_DO + bo, 16, 1024),
                   IDESC_S, kk > 0 ? 1u : 0u);
         }
-#endif
         umma_commit(bar(L::B_S_FULL));
       };
       bool ok = mbar_wait(bar(L::B_KV_FULL), 0, ctl);
@@ -532,22 +512,6 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
       tmem_ld_wait(v + 32);
       tc_fence_before();
       mbar_arrive_warp(bar(L::B_DQ_FREE));
-#if ATTN_BWD_DQ_DIRECT
-      if (!DET) {
-        // add dQ_i^T straight from registers: one coalesced fp32 reduction per query
-        const int h = hkv * G + i / per_head;
-        const int q0 = (qb0 + i % per_head) * L::BQ;
-        if (d >= 0) {
-          float* dst = p.dq_acc + ((static_cast<size_t>(b) * p.S_q + q0) * p.H_q + h) * D + d;
-          const size_t qstride = static_cast<size_t>(p.H_q) * D;
-          const int nq = min(L::BQ, p.S_q - q0);
-#pragma unroll
-          for (int c = 0; c < L::BQ; ++c)
-            if (c < nq) red_add_f32(dst + c * qstride, __uint_as_float(v[c]));
-        }
-        continue;
-      }
-#endif
       const int buf = i % L::NDQ;
       if (i >= L::NDQ) {  // the reduce of block i - NDQ has read this tile
         ok = mbar_wait(bar(L::B_STAGE_FREE + buf), ((i / L::NDQ) - 1) & 1, ctl);
@@ -562,7 +526,7 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
     }
   } else if (warp == L::WARP_RED) {
     // ===================== dQ reduce issue: one TMA reduce-add per staged tile =====================
-    if (lane == 0 && (DET || !ATTN_BWD_DQ_DIRECT)) {
+    if (lane == 0) {
       for (int i = 0; i < m; ++i) {
         const int buf = i % L::NDQ;
         if (!mbar_wait(bar(L::B_STAGED + buf), (i / L::NDQ) & 1, ctl)) break;

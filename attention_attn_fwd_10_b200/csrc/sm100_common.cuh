@@ -129,11 +129,6 @@ __device__ __forceinline__ void sem_release_add(int* sem) {
   asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(sem) : "memory");
 }
 
-// Fire-and-forget fp32 add into global memory (relaxed, GPU scope).
-__device__ __forceinline__ void red_add_f32(float* addr, float v) {
-  asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
-}
-
 // Orders global-memory accesses of the async proxy (TMA) against the generic proxy.
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
