@@ -312,6 +312,8 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   p.bh_group = kFwdBhGroup < B * (H_q / gp) ? kFwdBhGroup : B * (H_q / gp);
   p.n_splits = n_splits;
   p.split_blocks = split_blocks;
+  // one tile holds every query row: tile B takes half of the key blocks instead of idling
+  p.dual = S_q <= 128 / gp ? 1 : 0;
   if (n_splits > 1) {
     const size_t rows = static_cast<size_t>(n_splits) * B * H_q * S_q;
     p.o_part = static_cast<float*>(workspace);

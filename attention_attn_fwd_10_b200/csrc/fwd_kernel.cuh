@@ -62,6 +62,11 @@ struct FwdParams {
   int n_splits, split_blocks;
   float* o_part;
   float* lse_part;
+  // Dual stream (used when one tile holds every query row of the unit): tile B
+  // takes the odd key blocks of the CTA's range for the same rows as tile A, so
+  // the two tiles' softmax/MMA chains overlap; tile A merges the two partial
+  // results by the log-sum-exp identity in the epilogue.
+  int dual;
   float scale_log2;  // scale * log2(e)
   float tau;         // rescale threshold (base-2 units); 0 = rescale on every increase
   int* status;       // device status word
@@ -78,6 +83,10 @@ struct FwdLayout {
   static constexpr int BN = 128;                 // keys per block
   static constexpr int KST = 3;                  // K ring depth (released after the last S MMA of a block)
   static constexpr int VST = 2;                  // V ring depth (released after the last PV MMA of a block)
+  // In the dual stream tile B reads tile A's Q, and (bf16 Q, where a Q tile is
+  // exactly a V tile) tile B's Q buffer becomes a third V slot: each step then
+  // uses two V blocks and a third can be loading.
+  static constexpr int VST_DUAL = QK8 ? 2 : 3;
   static constexpr int NBOX = D / 64;            // 64-element (128 B) TMA boxes per row block
   static constexpr int BOX_BYTES = 128 * 128;    // one 128 x 64 bf16 box
   static constexpr int TILE_BYTES = 128 * D * 2; // one 128 x D bf16 tile
@@ -92,15 +101,17 @@ struct FwdLayout {
   static constexpr int B_Q_FULL = 0;                    // [t]
   static constexpr int B_K_FULL = B_Q_FULL + 2;        // [ks]
   static constexpr int B_K_EMPTY = B_K_FULL + KST;     // [ks]
-  static constexpr int B_V_FULL = B_K_EMPTY + KST;     // [vs]
-  static constexpr int B_V_EMPTY = B_V_FULL + VST;     // [vs]
-  static constexpr int B_S_FULL = B_V_EMPTY + VST;     // [t]
+  static constexpr int B_V_FULL = B_K_EMPTY + KST;     // [vs], up to 3
+  static constexpr int B_V_EMPTY = B_V_FULL + 3;       // [vs], up to 3
+  static constexpr int B_S_FULL = B_V_EMPTY + 3;       // [t]
   static constexpr int B_P_FULL = B_S_FULL + 2;         // [t][half]  (one arrival per softmax warp)
   static constexpr int B_PV_DONE = B_P_FULL + 4;        // [t]
   static constexpr int B_O_FINAL = B_PV_DONE + 2;       // [t]
   static constexpr int B_DRAIN = B_O_FINAL + 2;
-  static constexpr int N_BARS = B_DRAIN + 1;
-  static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * N_BARS;
+  static constexpr int B_XCHG = B_DRAIN + 1;            // dual stream: tile B's row statistics written (4 warps)
+  static constexpr int N_BARS = B_XCHG + 1;
+  static constexpr int XCHG_OFF = BAR_OFF + 8 * N_BARS;  // dual stream: tile B's running max, sum per row (2 x 128 fp32)
+  static constexpr int TMEM_SLOT_OFF = XCHG_OFF + 1024;
   static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 4;
   static constexpr int SMEM_USED = ABORT_OFF + 4;
   // 1 KiB of slack to align the base to 1024 bytes (128-byte swizzle atoms);
@@ -110,13 +121,15 @@ struct FwdLayout {
   // tensor memory columns
   __device__ static constexpr uint32_t s_col(int t) { return static_cast<uint32_t>(t) * 128u; }
   __device__ static constexpr uint32_t o_col(int t) { return 256u + static_cast<uint32_t>(t) * D; }
+  // shared-memory offset of V slot s (slot 2 only in the dual stream: tile B's Q buffer)
+  __device__ static constexpr int v_off(int s) { return s < 2 ? V_OFF + s * TILE_BYTES : Q_OFF + QK_BYTES; }
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int THREADS = 384;
   static constexpr int WARP_TMA = 8, WARP_MMA = 9, WARP_TMA_V = 10;
   // Register split: launched at 168 per thread (384 x 168 = 64512); the two
-  // softmax warpgroups grow to 216 and the third shrinks to 72:
-  // 2 x 128 x 216 + 128 x 72 = 64512, exactly the launch's total.
-  static constexpr int REG_SOFTMAX = 216, REG_OTHER = 72;
+  // softmax warpgroups grow to 208 and the third (producers, MMA issuer) shrinks
+  // to 80: 2 x 128 x 208 + 128 x 80 = 63488, within the launch's total.
+  static constexpr int REG_SOFTMAX = 208, REG_OTHER = 80;
 };
 
 // p = 2^(s * c - m) for one 128-column score row, packed to bf16 pairs; returns
@@ -208,19 +221,33 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
   const int tile_pos = L::BM >> p.gp_log2;  // query positions per tile
   const int q0 = u * 2 * tile_pos;          // first query position of the unit
   const int diag = p.S_k - p.S_q;  // bottom-right causal: key j visible to row i iff j <= i + diag
-  // key blocks j0 + j, j < nblk[t], of this CTA's split that tile t sees
+  // Key block of tile t's step j: j0 + j (both tiles take the same blocks), or in the
+  // dual stream j0 + 2j + t.  nblk[t] steps per tile; the producers load n_loads
+  // blocks j0, j0 + 1, ... in order either way.
   const int j0 = split * p.split_blocks;
+  const bool dual = p.dual != 0;
   int nblk[2];
+  int n_loads;
+  if (dual) {
+    const int nb_all = min(max(tile_blocks(q0, tile_pos, p.S_q, p.S_k, CAUSAL, L::BN) - j0, 0), p.split_blocks);
+    nblk[0] = (nb_all + 1) / 2;
+    nblk[1] = nb_all / 2;
+    n_loads = nb_all;
+  } else {
 #pragma unroll
-  for (int t = 0; t < 2; ++t)
-    nblk[t] = min(max(tile_blocks(q0 + t * tile_pos, tile_pos, p.S_q, p.S_k, CAUSAL, L::BN) - j0, 0),
-                  p.split_blocks);
+    for (int t = 0; t < 2; ++t)
+      nblk[t] = min(max(tile_blocks(q0 + t * tile_pos, tile_pos, p.S_q, p.S_k, CAUSAL, L::BN) - j0, 0),
+                    p.split_blocks);
+    n_loads = max(nblk[0], nblk[1]);
+  }
   const int n_blocks = max(nblk[0], nblk[1]);
+  // Q tiles loaded: one per tile, or only tile A's in the dual stream (both tiles read it)
+  const bool q_loaded[2] = {nblk[0] > 0, nblk[1] > 0 && !dual};
 
   // ---- setup
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::N_BARS; ++i)
-      mbar_init(bar(i), (i >= L::B_P_FULL && i < L::B_P_FULL + 4) ? 4u : 1u);
+      mbar_init(bar(i), ((i >= L::B_P_FULL && i < L::B_P_FULL + 4) || i == L::B_XCHG) ? 4u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -249,7 +276,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
     if (lane == 0 && n_blocks > 0) {
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
-        if (nblk[t] == 0) continue;
+        if (!q_loaded[t]) continue;
         mbar_arrive_expect_tx(bar(L::B_Q_FULL + t), L::QK_BYTES);
 #pragma unroll
         for (int x = 0; x < L::QK_NBOX; ++x)
@@ -257,7 +284,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
                       x * 64, h0, q0 + t * tile_pos, b);
       }
       int issued = 0;
-      for (int j = 0; j < n_blocks; ++j) {
+      for (int j = 0; j < n_loads; ++j) {
         const int s = j % L::KST;
         if (j >= L::KST && !mbar_wait(bar(L::B_K_EMPTY + s), ((j / L::KST) - 1) & 1, ctl)) break;
         mbar_arrive_expect_tx(bar(L::B_K_FULL + s), L::QK_BYTES);
@@ -269,7 +296,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
       }
       // Drain: every load this thread issued has landed before the CTA may exit.
       for (int t = 0; t < 2; ++t)
-        if (nblk[t] > 0) mbar_wait_drain(bar(L::B_Q_FULL + t), 0, 1000000000ull);
+        if (q_loaded[t]) mbar_wait_drain(bar(L::B_Q_FULL + t), 0, 1000000000ull);
       for (int s = 0; s < L::KST && s < issued; ++s)
         mbar_wait_drain(bar(L::B_K_FULL + s), ((issued - 1 - s) / L::KST) & 1, 1000000000ull);
     }
@@ -277,18 +304,19 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
     // ===================== TMA producer: V =====================
     if (lane == 0 && n_blocks > 0) {
       int issued = 0;
-      for (int j = 0; j < n_blocks; ++j) {
-        const int s = j % L::VST;
-        if (j >= L::VST && !mbar_wait(bar(L::B_V_EMPTY + s), ((j / L::VST) - 1) & 1, ctl)) break;
+      const int nv = dual ? L::VST_DUAL : L::VST;  // V slots in use
+      for (int j = 0; j < n_loads; ++j) {
+        const int s = j % nv;
+        if (j >= nv && !mbar_wait(bar(L::B_V_EMPTY + s), ((j / nv) - 1) & 1, ctl)) break;
         mbar_arrive_expect_tx(bar(L::B_V_FULL + s), L::TILE_BYTES);
 #pragma unroll
         for (int x = 0; x < L::NBOX; ++x)
-          tma_load_4d(sbase + L::V_OFF + s * L::TILE_BYTES + x * L::BOX_BYTES, &tm_v, bar(L::B_V_FULL + s),
+          tma_load_4d(sbase + L::v_off(s) + x * L::BOX_BYTES, &tm_v, bar(L::B_V_FULL + s),
                       x * 64, hkv, (j0 + j) * L::BN, b);
         issued = j + 1;
       }
-      for (int s = 0; s < L::VST && s < issued; ++s)
-        mbar_wait_drain(bar(L::B_V_FULL + s), ((issued - 1 - s) / L::VST) & 1, 1000000000ull);
+      for (int s = 0; s < nv && s < issued; ++s)
+        mbar_wait_drain(bar(L::B_V_FULL + s), ((issued - 1 - s) / nv) & 1, 1000000000ull);
     }
   } else if (warp == L::WARP_MMA) {
     // ===================== MMA issuer =====================
@@ -296,7 +324,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
       auto issue_s = [&](int t, int stage) {
-        const uint32_t q_base = sbase + L::Q_OFF + t * L::QK_BYTES;
+        const uint32_t q_base = sbase + L::Q_OFF + (dual ? 0 : t) * L::QK_BYTES;
         const uint32_t k_base = sbase + L::K_OFF + stage * L::QK_BYTES;
         if constexpr (QK8) {
           // 32 head dims (32 bytes of the 128-byte row) per MMA
@@ -317,7 +345,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
       };
       // PV_t(j) in two halves of 64 keys, each issued once its half of P_t(j) is in TMEM
       auto issue_pv_half = [&](int t, int stage, bool acc, int hf) {
-        const uint32_t v_base = sbase + L::V_OFF + stage * L::TILE_BYTES;
+        const uint32_t v_base = sbase + L::v_off(stage);
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
           const int kk = 4 * hf + k4;
@@ -329,54 +357,99 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
         if (hf == 1) umma_commit(bar(L::B_PV_DONE + t));
 #endif
       };
-      bool ok = mbar_wait(bar(L::B_K_FULL), 0, ctl);
-      for (int t = 0; ok && t < 2; ++t) {
-        if (nblk[t] == 0) continue;
-        ok = mbar_wait(bar(L::B_Q_FULL + t), 0, ctl);
-        if (ok) {
-          tc_fence_after();
-          issue_s(t, 0);
+      if (dual) {
+        // Dual stream: tile t takes key blocks j0 + 2j + t.  Load n = 2j + t sits in K
+        // slot n % KST and V slot n % VST_DUAL; the S and the PV MMAs each consume
+        // their loads in order n = 0, 1, 2, ..., so a running (slot, phase) pair per
+        // ring tracks them.  Each load is used by one tile only.
+        bool ok = true;
+        int ks = 0, kph = 0;  // K slot and phase of the next S MMA
+        int vs = 0, vph = 0;  // V slot and phase of the next PV MMA (V loads are consumed in order too)
+        for (int t = 0; ok && t < 2; ++t) {
+          if (nblk[t] == 0) continue;
+          ok = mbar_wait(bar(L::B_K_FULL + ks), kph, ctl);
+          if (ok && t == 0) ok = mbar_wait(bar(L::B_Q_FULL), 0, ctl);
+          if (ok) {
+            tc_fence_after();
+            issue_s(t, ks);
+            umma_commit(bar(L::B_K_EMPTY + ks));
+          }
+          if (++ks == L::KST) { ks = 0; kph ^= 1; }
         }
-      }
-      if (ok) umma_commit(bar(L::B_K_EMPTY));  // K_0 released once both S(0) complete
-      // Per key block j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1).  S_t(j+1) overwrites
-      // P_t(j), which PV_t(j) reads: the MMAs of this one issuing thread execute
-      // in issue order, so PV_t(j) has read P_t(j) before S_t(j+1) writes there
-      // (ATTN_FWD_PV_WAIT=1 makes the issuer wait for PV_t(j) to complete instead).
-      for (int j = 0; ok && j < n_blocks; ++j) {
-        const int vs = j % L::VST;
-        const int ks1 = (j + 1) % L::KST;
-        if (!mbar_wait(bar(L::B_V_FULL + vs), (j / L::VST) & 1, ctl)) break;
-        bool k_next_ready = false;
+        for (int j = 0; ok && j < n_blocks; ++j) {
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (!ok || j >= nblk[t]) continue;
-          ok = mbar_wait(bar(L::B_P_FULL + 2 * t), j & 1, ctl);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv_half(t, vs, j > 0, 0);
-          ok = mbar_wait(bar(L::B_P_FULL + 2 * t + 1), j & 1, ctl);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv_half(t, vs, j > 0, 1);
-          if (j == nblk[t] - 1) umma_commit(bar(L::B_O_FINAL + t));
-          if (j + 1 < nblk[t]) {
-            if (!k_next_ready) {
-              ok = mbar_wait(bar(L::B_K_FULL + ks1), ((j + 1) / L::KST) & 1, ctl);
-              if (!ok) break;
-              k_next_ready = true;
-            }
-#if ATTN_FWD_PV_WAIT
-            ok = mbar_wait(bar(L::B_PV_DONE + t), j & 1, ctl);
+          for (int t = 0; t < 2; ++t) {
+            if (!ok || j >= nblk[t]) continue;
+            ok = mbar_wait(bar(L::B_V_FULL + vs), vph, ctl) && mbar_wait(bar(L::B_P_FULL + 2 * t), j & 1, ctl);
             if (!ok) break;
             tc_fence_after();
-#endif
-            issue_s(t, ks1);
+            issue_pv_half(t, vs, j > 0, 0);
+            ok = mbar_wait(bar(L::B_P_FULL + 2 * t + 1), j & 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv_half(t, vs, j > 0, 1);
+            if (j == nblk[t] - 1) umma_commit(bar(L::B_O_FINAL + t));
+            umma_commit(bar(L::B_V_EMPTY + vs));
+            if (++vs == L::VST_DUAL) { vs = 0; vph ^= 1; }
+            if (j + 1 < nblk[t]) {
+              ok = mbar_wait(bar(L::B_K_FULL + ks), kph, ctl);
+              if (!ok) break;
+              issue_s(t, ks);
+              umma_commit(bar(L::B_K_EMPTY + ks));
+              if (++ks == L::KST) { ks = 0; kph ^= 1; }
+            }
           }
         }
-        if (!ok) break;
-        umma_commit(bar(L::B_V_EMPTY + vs));
-        if (k_next_ready) umma_commit(bar(L::B_K_EMPTY + ks1));
+      } else {
+        bool ok = mbar_wait(bar(L::B_K_FULL), 0, ctl);
+        for (int t = 0; ok && t < 2; ++t) {
+          if (nblk[t] == 0) continue;
+          ok = mbar_wait(bar(L::B_Q_FULL + t), 0, ctl);
+          if (ok) {
+            tc_fence_after();
+            issue_s(t, 0);
+          }
+        }
+        if (ok) umma_commit(bar(L::B_K_EMPTY));  // K_0 released once both S(0) complete
+        // Per key block j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1).  S_t(j+1) overwrites
+        // P_t(j), which PV_t(j) reads: the MMAs of this one issuing thread execute
+        // in issue order, so PV_t(j) has read P_t(j) before S_t(j+1) writes there
+        // (ATTN_FWD_PV_WAIT=1 makes the issuer wait for PV_t(j) to complete instead).
+        for (int j = 0; ok && j < n_blocks; ++j) {
+          const int vs = j % L::VST;
+          const int ks1 = (j + 1) % L::KST;
+          if (!mbar_wait(bar(L::B_V_FULL + vs), (j / L::VST) & 1, ctl)) break;
+          bool k_next_ready = false;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (!ok || j >= nblk[t]) continue;
+            ok = mbar_wait(bar(L::B_P_FULL + 2 * t), j & 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv_half(t, vs, j > 0, 0);
+            ok = mbar_wait(bar(L::B_P_FULL + 2 * t + 1), j & 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv_half(t, vs, j > 0, 1);
+            if (j == nblk[t] - 1) umma_commit(bar(L::B_O_FINAL + t));
+            if (j + 1 < nblk[t]) {
+              if (!k_next_ready) {
+                ok = mbar_wait(bar(L::B_K_FULL + ks1), ((j + 1) / L::KST) & 1, ctl);
+                if (!ok) break;
+                k_next_ready = true;
+              }
+#if ATTN_FWD_PV_WAIT
+              ok = mbar_wait(bar(L::B_PV_DONE + t), j & 1, ctl);
+              if (!ok) break;
+              tc_fence_after();
+#endif
+              issue_s(t, ks1);
+            }
+          }
+          if (!ok) break;
+          umma_commit(bar(L::B_V_EMPTY + vs));
+          if (k_next_ready) umma_commit(bar(L::B_K_EMPTY + ks1));
+        }
       }
       // Drain: no MMA may still be writing TMEM when it is released.
       umma_commit(bar(L::B_DRAIN));
@@ -387,7 +460,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
     setmaxnreg_inc<L::REG_SOFTMAX>();
     const int t = warp >> 2;
     const int row = threadIdx.x & 127;  // == TMEM lane
-    const int row0 = q0 + t * tile_pos;          // first query position of the tile
+    const int row0 = q0 + (dual ? 0 : t * tile_pos);  // first query position of the tile
     const int qi = row0 + (row >> p.gp_log2);     // this row's query position
     const int h = h0 + (row & (p.gp - 1));        // and query head
     const int nb = nblk[t];
@@ -411,7 +484,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
       for (int ch = 0; ch < 4; ++ch) tmem_ld_wait(sr + ch * 32);
 
       float* s = reinterpret_cast<float*>(sr);
-      const int kbase = (j0 + j) * L::BN;
+      const int kbase = (j0 + (dual ? 2 * j + t : j)) * L::BN;
       const bool need_mask = (kbase + L::BN - 1 > lim_tile) || (kbase + L::BN > p.S_k);
       if (need_mask) {
         const int lim_c = lim - kbase;
@@ -459,69 +532,83 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
     }
     if (p.rescale_count != nullptr && rescales) atomicAdd(p.rescale_count, (unsigned long long)rescales);
 
-    // ---- epilogue: O / l -> bf16, lse
+    // ---- epilogue: O / l -> bf16 (or the split's fp32 O_s), lse
     if (ok && nb > 0) {
       ok = mbar_wait(bar(L::B_O_FINAL + t), 0, ctl);
       ok = __all_sync(0xffffffffu, ok);
     }
-    if (ok && p.n_splits > 1) {
-      // partial result of this split: fp32 O_s, lse_s
-      tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      const bool valid = qi < p.S_q;
-      const size_t part = static_cast<size_t>(split) * p.B + b;
-      float* prow = p.o_part + ((part * p.S_q + qi) * p.H_q + h) * D;
-      const uint32_t o_addr = tmem + lane_addr + L::o_col(t);
-#pragma unroll 1
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t orr[32];
-        if (nb > 0) {
-          tmem_ld32(o_addr + ch * 32, orr);
-          tmem_ld_wait(orr);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) orr[i] = 0u;
-        }
-        if (valid) {
-          float4* dst = reinterpret_cast<float4*>(prow + ch * 32);
-#pragma unroll
-          for (int i = 0; i < 8; ++i)
-            dst[i] = make_float4(__uint_as_float(orr[4 * i]) * inv_l, __uint_as_float(orr[4 * i + 1]) * inv_l,
-                                 __uint_as_float(orr[4 * i + 2]) * inv_l, __uint_as_float(orr[4 * i + 3]) * inv_l);
-        }
-      }
-      if (valid)
-        p.lse_part[(part * p.H_q + h) * p.S_q + qi] =
-            l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+    float* xch = reinterpret_cast<float*>(sptr + L::XCHG_OFF);
+    if (dual && t == 1) {
+      // tile B hands its row statistics to tile A, which merges both halves
+      xch[row] = m_used;
+      xch[128 + row] = l;
+      mbar_arrive_warp(bar(L::B_XCHG));
     } else if (ok) {
-      tc_fence_after();
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      const bool valid = qi < p.S_q;
-      __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.S_q + qi) * p.H_q + h) * D;
-      const uint32_t o_addr = tmem + lane_addr + L::o_col(t);
-#pragma unroll 1
-      for (int ch = 0; ch < D / 32; ++ch) {
-        uint32_t orr[32];
-        if (nb > 0) {
-          tmem_ld32(o_addr + ch * 32, orr);
-          tmem_ld_wait(orr);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) orr[i] = 0u;
-        }
-        uint32_t pkd[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pkd[i] = pack_bf16x2(__uint_as_float(orr[2 * i]) * inv_l, __uint_as_float(orr[2 * i + 1]) * inv_l);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2], pkd[4 * i + 3]);
-        }
+      // Row result = (w_A O_A + w_B O_B) / (w_A l_A + w_B l_B), w = 2^(m - max m): the
+      // log-sum-exp merge of the two key halves in the dual stream; only this tile's
+      // O (w = 1) otherwise.  A half that saw no key has l = 0 and weight 0, and its O
+      // columns are never read into the result (select, not multiply).
+      float m_b = -INFINITY, l_b = 0.f;
+      const bool have_b = dual && nblk[1] > 0;
+      if (dual) {
+        ok = mbar_wait(bar(L::B_XCHG), 0, ctl);
+        if (ok && have_b) ok = mbar_wait(bar(L::B_O_FINAL + 1), 0, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        m_b = xch[row];
+        l_b = xch[128 + row];
       }
-      if (valid) {
-        p.lse[(static_cast<size_t>(b) * p.H_q + h) * p.S_q + qi] =
-            l > 0.f ? (m_used + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      if (ok) {
+        tc_fence_after();
+        const float mx = fmaxf(m_used, m_b);
+        const float w_a = l > 0.f ? exp2_mufu(m_used - mx) : 0.f;
+        const float w_b = l_b > 0.f ? exp2_mufu(m_b - mx) : 0.f;
+        const float lsum = l * w_a + l_b * w_b;
+        const float inv_l = lsum > 0.f ? 1.f / lsum : 0.f;
+        const float c_a = w_a * inv_l, c_b = w_b * inv_l;
+        const float lse_v = lsum > 0.f ? (mx + __log2f(lsum)) * 0.69314718055994531f : -INFINITY;
+        const bool valid = qi < p.S_q;
+        const uint32_t oa_addr = tmem + lane_addr + L::o_col(t);
+        const uint32_t ob_addr = tmem + lane_addr + L::o_col(1);
+        const size_t part = static_cast<size_t>(split) * p.B + b;
+#pragma unroll 1
+        for (int ch = 0; ch < D / 16; ++ch) {  // 16 columns at a time
+          uint32_t orr[16], obr[16];
+          if (nb > 0) {
+            tmem_ld16(oa_addr + ch * 16, orr);
+            tmem_ld_wait16(orr);
+          }
+          if (have_b) {
+            tmem_ld16(ob_addr + ch * 16, obr);
+            tmem_ld_wait16(obr);
+          }
+          float* ov = reinterpret_cast<float*>(orr);  // the result, in place
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float v = (nb > 0 && w_a > 0.f) ? __uint_as_float(orr[i]) * c_a : 0.f;
+            if (have_b && w_b > 0.f) v += __uint_as_float(obr[i]) * c_b;
+            ov[i] = v;
+          }
+          if (!valid) continue;
+          if (p.n_splits > 1) {
+            // partial result of this split: fp32 O_s
+            float4* dst = reinterpret_cast<float4*>(p.o_part + ((part * p.S_q + qi) * p.H_q + h) * D + ch * 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
+          } else {
+            uint32_t pkd[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) pkd[i] = pack_bf16x2(ov[2 * i], ov[2 * i + 1]);
+            uint4* dst = reinterpret_cast<uint4*>(p.o + ((static_cast<size_t>(b) * p.S_q + qi) * p.H_q + h) * D + ch * 16);
+            dst[0] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
+            dst[1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
+          }
+        }
+        if (valid) {
+          if (p.n_splits > 1)
+            p.lse_part[(part * p.H_q + h) * p.S_q + qi] = lse_v;
+          else
+            p.lse[(static_cast<size_t>(b) * p.H_q + h) * p.S_q + qi] = lse_v;
+        }
       }
     }
   }
@@ -541,6 +628,9 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
 //   lse = log sum_s exp(lse_s),   O = sum_s exp(lse_s - lse) O_s,
 // evaluated with the largest lse_s factored out.  Rows that saw no key in any
 // split (every lse_s = -inf) give O = 0 and lse = -inf, as the unsplit kernel.
+// The row's lse_s values are loaded by the lanes at once (lane s holds split s, 32
+// at a time) and reduced across the warp; the O_s rows are then streamed with
+// independent loads, so the row costs a few memory round trips, not one per split.
 template <int D>
 __global__ void __launch_bounds__(256) attn_fwd_combine_kernel(const FwdParams p) {
   constexpr int PER = D / 32;  // values per lane
@@ -557,20 +647,41 @@ __global__ void __launch_bounds__(256) attn_fwd_combine_kernel(const FwdParams p
     const size_t lse_stride = static_cast<size_t>(p.B) * p.H_q * p.S_q;
     const size_t lse_row = (static_cast<size_t>(b) * p.H_q + h) * p.S_q + q;
     float m = -INFINITY;
-    for (int s = 0; s < p.n_splits; ++s) m = fmaxf(m, p.lse_part[s * lse_stride + lse_row]);
+    for (int s0 = 0; s0 < p.n_splits; s0 += 32) {
+      const float ls = s0 + lane < p.n_splits ? p.lse_part[(s0 + lane) * lse_stride + lse_row] : -INFINITY;
+      m = fmaxf(m, ls);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     float acc[PER];
 #pragma unroll
     for (int i = 0; i < PER; ++i) acc[i] = 0.f;
     float sum = 0.f;
     if (m > -INFINITY) {
-      for (int s = 0; s < p.n_splits; ++s) {
-        const float ls = p.lse_part[s * lse_stride + lse_row];
-        if (ls == -INFINITY) continue;
-        const float wgt = exp2_mufu((ls - m) * 1.4426950408889634f);
-        sum += wgt;
-        const float* src = p.o_part + (static_cast<size_t>(s) * rows + w) * D + lane * PER;
+      for (int s0 = 0; s0 < p.n_splits; s0 += 32) {
+        const int ns = min(32, p.n_splits - s0);
+        const float ls = lane < ns ? p.lse_part[(s0 + lane) * lse_stride + lse_row] : -INFINITY;
+        const float wl = ls == -INFINITY ? 0.f : exp2_mufu((ls - m) * 1.4426950408889634f);  // lane's split weight
+        float part = wl;
 #pragma unroll
-        for (int i = 0; i < PER; ++i) acc[i] += wgt * src[i];
+        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+        sum += part;
+#pragma unroll 4
+        for (int s = 0; s < ns; ++s) {
+          const float wgt = __shfl_sync(0xffffffffu, wl, s);
+          const float* src = p.o_part + (static_cast<size_t>(s0 + s) * rows + w) * D + lane * PER;
+          if constexpr (PER == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(src);
+            acc[0] += wgt * v.x;
+            acc[1] += wgt * v.y;
+            acc[2] += wgt * v.z;
+            acc[3] += wgt * v.w;
+          } else {
+            const float2 v = *reinterpret_cast<const float2*>(src);
+            acc[0] += wgt * v.x;
+            acc[1] += wgt * v.y;
+          }
+        }
       }
     }
     const float inv = sum > 0.f ? 1.f / sum : 0.f;

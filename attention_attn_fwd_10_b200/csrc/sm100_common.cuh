@@ -311,6 +311,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
       : "r"(taddr));
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : ATTN_R8(r, 0), ATTN_R8(r, 8)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait16(uint32_t* r) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : ATTN_P8(r, 0), ATTN_P8(r, 8) : : "memory");
+}
+
 // Wait for this thread's outstanding tcgen05.ld; the registers are threaded
 // through the asm so no use of them can be scheduled before the wait.
 __device__ __forceinline__ void tmem_ld_wait(uint32_t* r) {

@@ -591,6 +591,19 @@ def run_profile(args):
 
     wf, wb = WORKLOADS[args.workload]
     torch.cuda.set_device(0)
+    if args.profile == "decode":
+        # one query row per head against 32768 keys: the split-KV forward and its merge
+        w = workloads.small(B=1, H_q=32, H_kv=8, S_q=1, S_k=32768, D=128, causal=True, seed=1)
+        xd = workloads.make_inputs(w)
+        q, k, v = (xd[n].cuda() for n in ("q", "k", "v"))
+        for _ in range(args.warmup + args.steps):
+            attn.fwd_split(q, k, v, causal=True, scale=w.scale)
+        torch.cuda.synchronize()
+        st = attn.device_status()
+        print(f"profile decode: {args.warmup + args.steps} calls, device status {st}")
+        if st != 0:
+            sys.exit(1)
+        return
     x = workloads.make_inputs(wb)
     q, k, v, do = (x[n].cuda() for n in ("q", "k", "v", "do"))
     o, lse = attn.fwd(q, k, v, causal=wf.causal, scale=wf.scale)
@@ -690,7 +703,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU time to sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration measurements")
-    ap.add_argument("--profile", choices=("fwd", "bwd"), default=None,
+    ap.add_argument("--profile", choices=("fwd", "bwd", "decode"), default=None,
                     help="only launch one pass W+K times (driver for ncu captures); prints no JSON")
     ap.add_argument("--variants", action="store_true",
                     help="side measurements (bf16 / e4m3 Q-K forward, decode shapes, deterministic backward); "
