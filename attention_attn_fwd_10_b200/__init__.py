@@ -113,12 +113,14 @@ def fwd_qk8(q, k, v, causal: bool = False, scale: float | None = None, out=None,
             rescale_threshold: float = 8.0, poly_exp_every: int = 8, stream=None):
     """Forward with 8-bit Q and K (attn_fwd_qk8): q, k torch.float8_e4m3fn, v bf16,
     head dim 128.  Returns (o bf16, lse fp32) of attention over the e4m3 values of
-    q and k.  Device tensors only."""
+    q and k.  With v torch.float8_e4m3fn as well, both products run on the 8-bit
+    path and P is rounded to e4m3 (attn_fwd_qkv8).  Device tensors only."""
     B, S_q, H_q, S_k, H_kv, D = _shapes(q, k)
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     _check_tensor("q", q, (B, S_q, H_q, D), torch.float8_e4m3fn)
     _check_tensor("k", k, (B, S_k, H_kv, D), torch.float8_e4m3fn)
-    _check_tensor("v", v, (B, S_k, H_kv, D))
+    pv8 = v.dtype == torch.float8_e4m3fn
+    _check_tensor("v", v, (B, S_k, H_kv, D), torch.float8_e4m3fn if pv8 else torch.bfloat16)
     if out is None:
         out = torch.empty((B, S_q, H_q, D), dtype=torch.bfloat16, device=q.device)
     if lse is None:
@@ -128,10 +130,10 @@ def fwd_qk8(q, k, v, causal: bool = False, scale: float | None = None, out=None,
     dev = _device_of(q, k, v, out, lse)
     opt = FwdOptions(float(rescale_threshold), int(poly_exp_every), None)
     with torch.cuda.device(dev):
-        code = load().attn_fwd_qk8(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                                   B, H_q, H_kv, S_q, S_k, D, int(bool(causal)), scale, ctypes.byref(opt),
-                                   _stream_ptr(stream, dev))
-    _abi.check(code, "attn_fwd_qk8")
+        fn = load().attn_fwd_qkv8 if pv8 else load().attn_fwd_qk8
+        code = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                  B, H_q, H_kv, S_q, S_k, D, int(bool(causal)), scale, ctypes.byref(opt), _stream_ptr(stream, dev))
+    _abi.check(code, "attn_fwd_qkv8" if pv8 else "attn_fwd_qk8")
     return out, lse
 
 

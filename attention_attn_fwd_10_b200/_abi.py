@@ -30,6 +30,7 @@ EXPORTED = (
     "attn_fwd_default_options",
     "attn_fwd_ex",
     "attn_fwd_qk8",
+    "attn_fwd_qkv8",
     "attn_fwd_split",
     "attn_fwd_split_qk8",
     "attn_fwd_split_count",
@@ -74,6 +75,8 @@ _SIGNATURES = {
                          ctypes.POINTER(FwdOptions), _vp]),
     "attn_fwd_qk8": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
                           ctypes.POINTER(FwdOptions), _vp]),
+    "attn_fwd_qkv8": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _f,
+                           ctypes.POINTER(FwdOptions), _vp]),
     "attn_fwd_split": (_i, [_vp] * 6 + [_i, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
     "attn_fwd_split_qk8": (_i, [_vp] * 6 + [_i, _i, _i, _i, _i, _i, _i, _f, _i, _vp]),
     "attn_fwd_split_count": (_i, [_i, _i, _i, _i, _i, _i]),

@@ -204,11 +204,11 @@ attn_status_t check_common(int B, int H_q, int H_kv, int S_q, int S_k, int D, in
   return ATTN_OK;
 }
 
-template <int D, bool CAUSAL, int POLY, bool QK8>
+template <int D, bool CAUSAL, int POLY, bool QK8, bool PV8 = false>
 cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const FwdParams& p,
                        unsigned grid, cudaStream_t st) {
-  using L = FwdLayout<D, QK8>;
-  auto kern = attn_fwd_kernel<D, CAUSAL, POLY, QK8>;
+  using L = FwdLayout<D, QK8, PV8>;
+  auto kern = attn_fwd_kernel<D, CAUSAL, POLY, QK8, PV8>;
   static CUcontext seen[kMaxDevices] = {};
   const cudaError_t attr_err = smem_opt_in(kern, L::SMEM_BYTES, seen);
   if (attr_err != cudaSuccess) return attr_err;
@@ -216,13 +216,13 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   return cudaGetLastError();
 }
 
-template <int D, bool CAUSAL, bool QK8 = false>
+template <int D, bool CAUSAL, bool QK8 = false, bool PV8 = false>
 cudaError_t launch_fwd_poly(int poly, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                             const FwdParams& p, unsigned grid, cudaStream_t st) {
   switch (poly) {
-    case 0: return launch_fwd<D, CAUSAL, 0, QK8>(mq, mk, mv, p, grid, st);
-    case 4: return launch_fwd<D, CAUSAL, 4, QK8>(mq, mk, mv, p, grid, st);
-    default: return launch_fwd<D, CAUSAL, 8, QK8>(mq, mk, mv, p, grid, st);
+    case 0: return launch_fwd<D, CAUSAL, 0, QK8, PV8>(mq, mk, mv, p, grid, st);
+    case 4: return launch_fwd<D, CAUSAL, 4, QK8, PV8>(mq, mk, mv, p, grid, st);
+    default: return launch_fwd<D, CAUSAL, 8, QK8, PV8>(mq, mk, mv, p, grid, st);
   }
 }
 
@@ -270,20 +270,23 @@ int fwd_head_pack(int H_q, int H_kv, int S_q) {
 // per-split partial results into `workspace` and a combine kernel merges them.
 attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace, int B,
                       int H_q, int H_kv, int S_q, int S_k, int D, int causal, float scale,
-                      const attn_fwd_options_t* opt_in, int n_splits, void* stream, bool qk8 = false) {
+                      const attn_fwd_options_t* opt_in, int n_splits, void* stream, bool qk8 = false,
+                      bool pv8 = false) {
   attn_fwd_options_t opt;
   attn_fwd_default_options(&opt);
   if (opt_in) opt = *opt_in;
   attn_status_t st = check_common(B, H_q, H_kv, S_q, S_k, D, causal, scale);
   if (st != ATTN_OK) return st;
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
-  if (qk8 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((qk8 || pv8) && D != 128) return ATTN_ERR_UNSUPPORTED;
   // split ranges: split_blocks key blocks each; trailing splits that would be empty are dropped
   const int n_kv = (S_k + 127) / 128;
   const int split_blocks = (n_kv + n_splits - 1) / n_splits;
   n_splits = (n_kv + split_blocks - 1) / split_blocks;
   if (n_splits > 1 && (!workspace || !aligned16(workspace))) return workspace ? ATTN_ERR_MISALIGNED : ATTN_ERR_INVALID_ARG;
   if (!(opt.rescale_threshold >= 0.f && opt.rescale_threshold <= 16.f)) return ATTN_ERR_INVALID_ARG;
+  // e4m3 weights: p <= 2^tau must stay below e4m3's largest value, 448
+  if (pv8 && opt.rescale_threshold > 8.f) return ATTN_ERR_INVALID_ARG;
   if (opt.poly_exp_every != 0 && opt.poly_exp_every != 4 && opt.poly_exp_every != 8) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_MISALIGNED;
 
@@ -293,7 +296,8 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   CUtensorMap mq, mk, mv;
   const int qk_bytes = qk8 ? 1 : 2;
   if (!make_bshd_map(&mq, q, B, S_q, H_q, D, 128 / gp, gp, qk_bytes) ||
-      !make_bshd_map(&mk, k, B, S_k, H_kv, D, 128, 1, qk_bytes) || !make_bshd_map(&mv, v, B, S_k, H_kv, D))
+      !make_bshd_map(&mk, k, B, S_k, H_kv, D, 128, 1, qk_bytes) ||
+      !make_bshd_map(&mv, v, B, S_k, H_kv, D, 128, 1, pv8 ? 1 : 2))
     return ATTN_ERR_CUDA;
   int* status = status_ptr();
   if (!status) return ATTN_ERR_CUDA;
@@ -329,7 +333,10 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   const unsigned grid = static_cast<unsigned>(grid_ll);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t err;
-  if (qk8)
+  if (pv8)
+    err = causal ? launch_fwd_poly<128, true, true, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s)
+                 : launch_fwd_poly<128, false, true, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s);
+  else if (qk8)
     err = causal ? launch_fwd_poly<128, true, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s)
                  : launch_fwd_poly<128, false, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s);
   else if (D == 128)
@@ -359,7 +366,7 @@ using namespace attn;
 
 extern "C" {
 
-int attn_abi_version(void) { return 2; }
+int attn_abi_version(void) { return 3; }
 
 const char* attn_status_string(attn_status_t s) {
   switch (s) {
@@ -420,6 +427,12 @@ attn_status_t attn_fwd_qk8(const void* q, const void* k, const void* v, void* o,
                            int H_kv, int S_q, int S_k, int D, int causal, float scale,
                            const attn_fwd_options_t* opt, void* stream) {
   return run_fwd(q, k, v, o, lse, nullptr, B, H_q, H_kv, S_q, S_k, D, causal, scale, opt, 1, stream, true);
+}
+
+attn_status_t attn_fwd_qkv8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H_q,
+                            int H_kv, int S_q, int S_k, int D, int causal, float scale,
+                            const attn_fwd_options_t* opt, void* stream) {
+  return run_fwd(q, k, v, o, lse, nullptr, B, H_q, H_kv, S_q, S_k, D, causal, scale, opt, 1, stream, true, true);
 }
 
 attn_status_t attn_fwd_split_qk8(const void* q, const void* k, const void* v, void* o, float* lse,

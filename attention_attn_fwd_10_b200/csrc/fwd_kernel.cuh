@@ -75,8 +75,9 @@ struct FwdParams {
 };
 
 // QK8: Q and K are e4m3 (1 byte per element; head dim 128 only), S = Q K^T runs
-// as kind::f8f6f4; V, P and O stay bf16.
-template <int D, bool QK8 = false>
+// as kind::f8f6f4; V, P and O stay bf16.  PV8 (with QK8): V is e4m3 too and P is
+// rounded to e4m3 in tensor memory, so O += P V runs as kind::f8f6f4 as well.
+template <int D, bool QK8 = false, bool PV8 = false>
 struct FwdLayout {
   static constexpr int BM = 128;                 // query rows per tile
   static constexpr int UNIT = 256;               // query rows per work unit (two tiles)
@@ -86,17 +87,20 @@ struct FwdLayout {
   // In the dual stream tile B reads tile A's Q, and (bf16 Q, where a Q tile is
   // exactly a V tile) tile B's Q buffer becomes a third V slot: each step then
   // uses two V blocks and a third can be loading.
-  static constexpr int VST_DUAL = QK8 ? 2 : 3;
+  static constexpr int VST_DUAL = (QK8 && !PV8) ? 2 : 3;
   static constexpr int NBOX = D / 64;            // 64-element (128 B) TMA boxes per row block
   static constexpr int BOX_BYTES = 128 * 128;    // one 128 x 64 bf16 box
   static constexpr int TILE_BYTES = 128 * D * 2; // one 128 x D bf16 tile
   static_assert(!QK8 || D == 128, "8-bit Q/K: head dim 128 (one 128-byte row per key)");
   static constexpr int QK_BYTES = QK8 ? 128 * D : TILE_BYTES;  // one Q or K tile
   static constexpr int QK_NBOX = QK8 ? 1 : NBOX;                // 128-byte TMA boxes per Q / K row
+  static_assert(!PV8 || QK8, "8-bit V and P come with 8-bit Q and K");
+  static constexpr int V_BYTES = PV8 ? 128 * D : TILE_BYTES;    // one V tile
+  static constexpr int V_NBOX = PV8 ? 1 : NBOX;                 // 128-byte TMA boxes per V row
   static constexpr int Q_OFF = 0;                // two Q tiles
   static constexpr int K_OFF = Q_OFF + 2 * QK_BYTES;
   static constexpr int V_OFF = K_OFF + KST * QK_BYTES;
-  static constexpr int BAR_OFF = V_OFF + VST * TILE_BYTES;
+  static constexpr int BAR_OFF = V_OFF + VST * V_BYTES;
   // barrier slots (8 bytes each); [t] = per Q tile, [s] = per ring stage
   static constexpr int B_Q_FULL = 0;                    // [t]
   static constexpr int B_K_FULL = B_Q_FULL + 2;        // [ks]
@@ -122,7 +126,7 @@ struct FwdLayout {
   __device__ static constexpr uint32_t s_col(int t) { return static_cast<uint32_t>(t) * 128u; }
   __device__ static constexpr uint32_t o_col(int t) { return 256u + static_cast<uint32_t>(t) * D; }
   // shared-memory offset of V slot s (slot 2 only in the dual stream: tile B's Q buffer)
-  __device__ static constexpr int v_off(int s) { return s < 2 ? V_OFF + s * TILE_BYTES : Q_OFF + QK_BYTES; }
+  __device__ static constexpr int v_off(int s) { return s < 2 ? V_OFF + s * V_BYTES : Q_OFF + QK_BYTES; }
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int THREADS = 384;
   static constexpr int WARP_TMA = 8, WARP_MMA = 9, WARP_TMA_V = 10;
@@ -135,11 +139,14 @@ struct FwdLayout {
 // p = 2^(s * c - m) for one 128-column score row, packed to bf16 pairs; returns
 // the fp32 sum of the unrounded p.  Column pair cp (columns 2cp, 2cp+1) takes
 // the FMA-pipe cubic when cp % POLY_EVERY == POLY_EVERY - 1, MUFU ex2 otherwise.
-template <int POLY_EVERY>
+// P8: the p values are packed as e4m3, four per word (16 words per half) instead
+// of bf16 pairs (32 words).
+template <int POLY_EVERY, bool P8 = false>
 __device__ __forceinline__ float exp_half(const uint32_t* sr, float c, float m, uint32_t* pk, int half) {
   const uint64_t c2 = f2_pack(c, c);
   const uint64_t nm2 = f2_pack(-m, -m);
   uint64_t acc[4];  // 4 independent packed partial sums (8 lanes of accumulation)
+  float pe0 = 0.f, pe1 = 0.f;  // P8: the previous pair, packed with the next one
 #pragma unroll
   for (int i = 0; i < 4; ++i) acc[i] = 0ull;
 #pragma unroll
@@ -155,7 +162,13 @@ __device__ __forceinline__ float exp_half(const uint32_t* sr, float c, float m, 
       e1 = exp2_mufu(x1);
     }
     acc[q & 3] = f2_add(acc[q & 3], f2_pack(e0, e1));
-    pk[q] = pack_bf16x2(e0, e1);
+    if constexpr (P8) {
+      if (q & 1) pk[q >> 1] = pack_e4m3x4(pe0, pe1, e0, e1);
+      pe0 = e0;
+      pe1 = e1;
+    } else {
+      pk[q] = pack_bf16x2(e0, e1);
+    }
   }
   float a0, a1;
   f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a0, a1);
@@ -186,11 +199,11 @@ __device__ __forceinline__ int tile_blocks(int row0, int rows, int S_q, int S_k,
   return last_key < 0 ? 0 : min(n_kv, last_key / BN + 1);
 }
 
-template <int D, bool CAUSAL, int POLY_EVERY, bool QK8 = false>
-__global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
+template <int D, bool CAUSAL, int POLY_EVERY, bool QK8 = false, bool PV8 = false>
+__global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using L = FwdLayout<D, QK8>;
+  using L = FwdLayout<D, QK8, PV8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -308,9 +321,9 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
       for (int j = 0; j < n_loads; ++j) {
         const int s = j % nv;
         if (j >= nv && !mbar_wait(bar(L::B_V_EMPTY + s), ((j / nv) - 1) & 1, ctl)) break;
-        mbar_arrive_expect_tx(bar(L::B_V_FULL + s), L::TILE_BYTES);
+        mbar_arrive_expect_tx(bar(L::B_V_FULL + s), L::V_BYTES);
 #pragma unroll
-        for (int x = 0; x < L::NBOX; ++x)
+        for (int x = 0; x < L::V_NBOX; ++x)
           tma_load_4d(sbase + L::v_off(s) + x * L::BOX_BYTES, &tm_v, bar(L::B_V_FULL + s),
                       x * 64, hkv, (j0 + j) * L::BN, b);
         issued = j + 1;
@@ -346,6 +359,18 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
       // PV_t(j) in two halves of 64 keys, each issued once its half of P_t(j) is in TMEM
       auto issue_pv_half = [&](int t, int stage, bool acc, int hf) {
         const uint32_t v_base = sbase + L::v_off(stage);
+        if constexpr (PV8) {
+          // 32 keys per MMA: 8 columns of e4m3 P (4 per column), 32 rows of 128 B of V
+          // (MN-major, one 128-byte column block: LBO unused)
+          constexpr uint32_t IDESC_PV8 = idesc_e4m3_f32(128, D) | (1u << 16);
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2) {
+            const int kk = 2 * hf + k2;
+            umma_ts_f8(tmem + L::o_col(t), tmem + L::s_col(t) + kk * 8, sdesc_sw128(v_base + kk * 4096, 16, 1024),
+                       IDESC_PV8, (acc || kk > 0) ? 1u : 0u);
+          }
+          return;
+        }
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
           const int kk = 4 * hf + k4;
@@ -517,14 +542,18 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8>::THREADS, 1)
           tmem_st32(o_addr + ch * 32, orr);
         }
       }
-      // P_t(j) over the first 64 columns of S_t, published in two halves (keys 0-63,
-      // then 64-127) so the PV MMA starts on the first while the second is computed.
+      // P_t(j) over the first 64 columns of S_t (32 for e4m3 P), published in two
+      // halves (keys 0-63, then 64-127) so the PV MMA starts on the first while the
+      // second is computed.
       // Masked blocks take MUFU ex2 only: it maps -inf to an exact 0.
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         uint32_t pk[32];
-        l += need_mask ? exp_half<0>(sr, c, m_eff, pk, hf) : exp_half<POLY_EVERY>(sr, c, m_eff, pk, hf);
-        tmem_st32(s_addr + 32 * hf, pk);
+        l += need_mask ? exp_half<0, PV8>(sr, c, m_eff, pk, hf) : exp_half<POLY_EVERY, PV8>(sr, c, m_eff, pk, hf);
+        if constexpr (PV8)
+          tmem_st16(s_addr + 16 * hf, pk);  // 64 keys as e4m3: 16 columns
+        else
+          tmem_st32(s_addr + 32 * hf, pk);
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive_warp(bar(L::B_P_FULL + 2 * t + hf));

@@ -506,6 +506,24 @@ def run_configs(attn, dev, flush, peaks):
     for w in (workloads.FWD_NONCAUSAL, workloads.FWD_CAUSAL, workloads.FWD_CAUSAL_SPIKY, workloads.FWD_CAUSAL_GQA):
         fwd_entry(w)
 
+    # the causal forward workload with 8-bit inputs: e4m3 Q, K (bf16 V, P), and e4m3 Q, K, V (e4m3 P)
+    w = workloads.FWD_CAUSAL
+    x = workloads.make_inputs(w)
+    q8, k8, v8 = (x[n].to(dev).to(torch.float8_e4m3fn) for n in ("q", "k", "v"))
+    v16 = x["v"].to(dev)
+    o = torch.empty((w.B, w.S_q, w.H_q, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.H_q, w.S_q), dtype=torch.float32, device=dev)
+    for tag, vv in (("e4m3_qk", v16), ("e4m3_qkv", v8)):
+        with ClockSampler(dev.index) as clk:
+            ms, reps = timed_calls(lambda: attn.fwd_qk8(q8, k8, vv, causal=True, scale=w.scale, out=o, lse=lse),
+                                   flush, stream)
+        c = clk.summary()
+        tf = w.fwd_flops() / (ms * 1e-3) / 1e12
+        # fraction of the measured bf16 peak (the 8-bit products themselves run at up to twice that rate)
+        out[f"{w.name}_{tag}"] = {"ms": round(ms, 4), "tflops": round(tf, 1), "frac_of_measured_bf16": round(tf / peak, 4),
+                                  "reps": reps, "sm_mhz": c["sm_mhz"], "clock_samples": c.get("samples")}
+    del q8, k8, v8, v16, o, lse, x
+
     # decode: one query row per head against 32768 keys, split-KV forward (bytes-bound: K and V stream once)
     w = workloads.small(B=1, H_q=32, H_kv=8, S_q=1, S_k=32768, D=128, causal=True, seed=1)
     x = workloads.make_inputs(w)

@@ -58,7 +58,8 @@ typedef enum {
 } attn_status_t;
 
 /* Version of this ABI (bumped on any incompatible change; 2: attn_bwd_options_t gained
- * `deterministic`, the split-KV and 8-bit Q/K forwards were added). */
+ * `deterministic`, the split-KV and 8-bit Q/K forwards were added; 3: the backward
+ * workspace gained the deterministic mode's work-item counter, attn_fwd_qkv8). */
 int attn_abi_version(void);
 
 /* Human-readable name of a status code (static storage). */
@@ -116,6 +117,26 @@ attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, 
 attn_status_t attn_fwd_qk8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H_q,
                            int H_kv, int S_q, int S_k, int D, int causal, float scale,
                            const attn_fwd_options_t* opt, void* stream);
+
+/*
+ * Forward with 8-bit Q, K and V: q, k and v hold float8 e4m3 values (one byte per
+ * element, BSHD); o is bf16, lse fp32.  Both products run on the tensor cores'
+ * 8-bit path (kind::f8f6f4): S = scale * Q K^T as in attn_fwd_qk8, and O += P V
+ * with the unnormalised weights p = 2^(scale log2(e) s - m) (m the row's running
+ * max, p <= 2^rescale_threshold) rounded to e4m3 in tensor memory.  The row sums
+ * and lse use the unrounded p, so lse is as accurate as attn_fwd_qk8's; O differs
+ * from the exact attention of the e4m3 inputs by the rounding of p: per element
+ * at most 2^-4 sum_k P_ik |v_k| (three mantissa bits, round to nearest) plus
+ * 2^-10 sum_k |v_k| / L_i for weights in e4m3's subnormal range (L_i = sum_k
+ * exp(s_ik - max_k s_ik)), plus the bf16 rounding of O (the "reduce precision"
+ * lever of AI Infra series ch. 6, GPU performance engineering (II), section 5,
+ * applied to the whole forward).  Head dim 128 only; options and errors as
+ * attn_fwd_ex, except that rescale_threshold must be <= 8 (ATTN_ERR_INVALID_ARG
+ * otherwise): p <= 2^rescale_threshold must stay below e4m3's largest value, 448.
+ */
+attn_status_t attn_fwd_qkv8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H_q,
+                            int H_kv, int S_q, int S_k, int D, int causal, float scale,
+                            const attn_fwd_options_t* opt, void* stream);
 
 /*
  * Split-KV forward for shapes with few query rows and many keys (decoding

@@ -9,7 +9,7 @@
 int main(void) {
   void* entry_points[] = {
       (void*)attn_abi_version,      (void*)attn_status_string,   (void*)attn_fwd,
-      (void*)attn_fwd_default_options, (void*)attn_fwd_ex,       (void*)attn_fwd_qk8,
+      (void*)attn_fwd_default_options, (void*)attn_fwd_ex,       (void*)attn_fwd_qk8, (void*)attn_fwd_qkv8,
       (void*)attn_fwd_split,        (void*)attn_fwd_split_qk8,   (void*)attn_fwd_split_count,
       (void*)attn_fwd_split_workspace_size, (void*)attn_bwd_workspace_size, (void*)attn_bwd,
       (void*)attn_bwd_ex,           (void*)attn_bwd_noalloc,     (void*)attn_device_status,
