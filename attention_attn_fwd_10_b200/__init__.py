@@ -74,7 +74,8 @@ def _shapes(q, k):
 
 
 def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
-        rescale_threshold: float = 8.0, poly_exp_every: int = 8, rescale_count=None, stream=None):
+        rescale_threshold: float = 8.0, poly_exp_every: int = 8, rescale_count=None, stream=None,
+        persistent: bool = True):
     """Forward attention.  Returns (o bf16 [B,S_q,H_q,D], lse fp32 [B,H_q,S_q]).
 
     CPU inputs are copied to the current CUDA device and the outputs are
@@ -98,7 +99,7 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse
     _check_tensor("lse", lse, (B, H_q, S_q), torch.float32)
     dev = _device_of(q, k, v, out, lse, rescale_count)
     opt = FwdOptions(float(rescale_threshold), int(poly_exp_every),
-                     rescale_count.data_ptr() if rescale_count is not None else None)
+                     rescale_count.data_ptr() if rescale_count is not None else None, int(bool(persistent)))
     with torch.cuda.device(dev):
         code = load().attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                                   B, H_q, H_kv, S_q, S_k, D, int(bool(causal)), scale, ctypes.byref(opt),
@@ -110,7 +111,7 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse
 
 
 def fwd_qk8(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
-            rescale_threshold: float = 8.0, poly_exp_every: int = 8, stream=None):
+            rescale_threshold: float = 8.0, poly_exp_every: int = 8, stream=None, persistent: bool = True):
     """Forward with 8-bit Q and K (attn_fwd_qk8): q, k torch.float8_e4m3fn, v bf16,
     head dim 128.  Returns (o bf16, lse fp32) of attention over the e4m3 values of
     q and k.  With v torch.float8_e4m3fn as well, both products run on the 8-bit
@@ -128,7 +129,7 @@ def fwd_qk8(q, k, v, causal: bool = False, scale: float | None = None, out=None,
     _check_tensor("out", out, (B, S_q, H_q, D))
     _check_tensor("lse", lse, (B, H_q, S_q), torch.float32)
     dev = _device_of(q, k, v, out, lse)
-    opt = FwdOptions(float(rescale_threshold), int(poly_exp_every), None)
+    opt = FwdOptions(float(rescale_threshold), int(poly_exp_every), None, int(bool(persistent)))
     with torch.cuda.device(dev):
         fn = load().attn_fwd_qkv8 if pv8 else load().attn_fwd_qk8
         code = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),

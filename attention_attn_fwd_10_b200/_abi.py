@@ -52,6 +52,7 @@ class FwdOptions(ctypes.Structure):
         ("rescale_threshold", ctypes.c_float),
         ("poly_exp_every", ctypes.c_int),
         ("rescale_count", ctypes.c_void_p),
+        ("persistent", ctypes.c_int),
     ]
 
 

@@ -318,6 +318,7 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   p.split_blocks = split_blocks;
   // one tile holds every query row: tile B takes half of the key blocks instead of idling
   p.dual = S_q <= 128 / gp ? 1 : 0;
+  p.persistent = (opt.persistent && !p.dual) ? 1 : 0;
   if (n_splits > 1) {
     const size_t rows = static_cast<size_t>(n_splits) * B * H_q * S_q;
     p.o_part = static_cast<float*>(workspace);
@@ -387,6 +388,7 @@ void attn_fwd_default_options(attn_fwd_options_t* opt) {
   opt->rescale_threshold = 8.0f;
   opt->poly_exp_every = 8;
   opt->rescale_count = nullptr;
+  opt->persistent = 1;
 }
 
 attn_status_t attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H_q,

@@ -316,22 +316,26 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, L::BQ, false, false);   // S^T, dP^T
       constexpr uint32_t IDESC_G = idesc_bf16_f32(128, D, false, true);        // dV, dK (A in TMEM)
       constexpr uint32_t IDESC_Q = idesc_bf16_f32(D, L::BQ, true, true);       // dQ^T
-      const uint32_t k_base = sbase + L::K_OFF, v_base = sbase + L::V_OFF;
+      // shared-memory descriptors as (low, high) halves: the descriptor of base + off is
+      // the base's low half plus off / 16 (one 32-bit add per MMA)
+      constexpr uint32_t HI = sdesc_sw128_hi(1024);
+      const uint32_t k_lo = sdesc_lo(sbase + L::K_OFF, 16), v_lo = sdesc_lo(sbase + L::V_OFF, 16);
+      const uint32_t kT_lo = sdesc_lo(sbase + L::K_OFF, L::KBOX_BYTES);  // K^T: MN-major view of K
       auto issue_s_dp = [&](int st) {
         const uint32_t sb = sbase + L::STAGE_OFF + st * L::STAGE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ao = (kk >> 2) * L::KBOX_BYTES + (kk & 3) * 32;
           const uint32_t bo = (kk >> 2) * L::QBOX_BYTES + (kk & 3) * 32;
-          umma_ss(tmem + L::X_COL, sdesc_sw128(k_base + ao, 16, 1024), sdesc_sw128(sb + L::ST_Q + bo, 16, 1024),
-                  IDESC_S, kk > 0 ? 1u : 0u);
+          umma_ss_h(tmem + L::X_COL, k_lo + (ao >> 4), HI, sdesc_lo(sb + L::ST_Q, 16) + (bo >> 4), HI, IDESC_S,
+                    kk > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ao = (kk >> 2) * L::KBOX_BYTES + (kk & 3) * 32;
           const uint32_t bo = (kk >> 2) * L::QBOX_BYTES + (kk & 3) * 32;
-          umma_ss(tmem + L::Y_COL, sdesc_sw128(v_base + ao, 16, 1024), sdesc_sw128(sb + L::ST_DO + bo, 16, 1024),
-                  IDESC_S, kk > 0 ? 1u : 0u);
+          umma_ss_h(tmem + L::Y_COL, v_lo + (ao >> 4), HI, sdesc_lo(sb + L::ST_DO, 16) + (bo >> 4), HI, IDESC_S,
+                    kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(L::B_S_FULL));
       };
@@ -360,12 +364,12 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
         // dV += P^T dO_i ; dK += dS^T Q_i   (16 queries per MMA: 8 TMEM columns, 2048 B of the stage)
 #pragma unroll
         for (int kk = 0; kk < L::BQ / 16; ++kk)
-          umma_ts(tmem + L::DV_COL, tmem + L::P_COL + kk * 8, sdesc_sw128(sb + L::ST_DO + kk * 2048, L::QBOX_BYTES, 1024),
-                  IDESC_G, (i > 0 || kk > 0) ? 1u : 0u);
+          umma_ts_h(tmem + L::DV_COL, tmem + L::P_COL + kk * 8, sdesc_lo(sb + L::ST_DO, L::QBOX_BYTES) + kk * 128,
+                    HI, IDESC_G, (i > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < L::BQ / 16; ++kk)
-          umma_ts(tmem + L::DK_COL, tmem + L::DS_COL + kk * 8, sdesc_sw128(sb + L::ST_Q + kk * 2048, L::QBOX_BYTES, 1024),
-                  IDESC_G, (i > 0 || kk > 0) ? 1u : 0u);
+          umma_ts_h(tmem + L::DK_COL, tmem + L::DS_COL + kk * 8, sdesc_lo(sb + L::ST_Q, L::QBOX_BYTES) + kk * 128,
+                    HI, IDESC_G, (i > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(L::B_PD_FREE));
         umma_commit(bar(L::B_QDO_EMPTY + st));
         if (i >= 1) {
@@ -376,8 +380,8 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
         const uint32_t ds = sbase + L::DS_OFF + db * L::DS_BYTES;
 #pragma unroll
         for (int kk = 0; kk < L::BN / 16; ++kk)
-          umma_ss(tmem + L::DQ_COL, sdesc_sw128(k_base + kk * 2048, L::KBOX_BYTES, 1024),
-                  sdesc_sw128(ds + kk * 2048, L::DS_BYTES, 1024), IDESC_Q, kk > 0 ? 1u : 0u);
+          umma_ss_h(tmem + L::DQ_COL, kT_lo + kk * 128, HI, sdesc_lo(ds, L::DS_BYTES) + kk * 128, HI, IDESC_Q,
+                    kk > 0 ? 1u : 0u);
         umma_commit(bar(L::B_DQ_FULL));
       }
       if (ok) umma_commit(bar(L::B_D_FINAL));

@@ -35,11 +35,10 @@
 //   wastes 60%", first move).
 #pragma once
 
+#include <type_traits>
+
 #include "sm100_common.cuh"
 
-#ifndef ATTN_FWD_PV_WAIT
-#define ATTN_FWD_PV_WAIT 0
-#endif
 
 namespace attn {
 
@@ -67,6 +66,10 @@ struct FwdParams {
   // the two tiles' softmax/MMA chains overlap; tile A merges the two partial
   // results by the log-sum-exp identity in the epilogue.
   int dual;
+  // Persistent CTAs: after its work item a CTA claims the item of a CTA that has
+  // not started yet (cluster launch control) and processes it with the barriers,
+  // rings and tensor memory it already holds.  Not with the dual stream.
+  int persistent;
   float scale_log2;  // scale * log2(e)
   float tau;         // rescale threshold (base-2 units); 0 = rescale on every increase
   int* status;       // device status word
@@ -109,13 +112,19 @@ struct FwdLayout {
   static constexpr int B_V_EMPTY = B_V_FULL + 3;       // [vs], up to 3
   static constexpr int B_S_FULL = B_V_EMPTY + 3;       // [t]
   static constexpr int B_P_FULL = B_S_FULL + 2;         // [t][half]  (one arrival per softmax warp)
-  static constexpr int B_PV_DONE = B_P_FULL + 4;        // [t]
-  static constexpr int B_O_FINAL = B_PV_DONE + 2;       // [t]
+  static constexpr int B_O_FINAL = B_P_FULL + 4;        // [t]
   static constexpr int B_DRAIN = B_O_FINAL + 2;
   static constexpr int B_XCHG = B_DRAIN + 1;            // dual stream: tile B's row statistics written (4 warps)
-  static constexpr int N_BARS = B_XCHG + 1;
+  static constexpr int B_Q_EMPTY = B_XCHG + 1;          // [t] the unit's last S_t has read Q_t
+  static constexpr int B_ITEM_FULL = B_Q_EMPTY + 2;     // [u % 2] the scheduler published unit u's work item
+  static constexpr int B_ITEM_READ = B_ITEM_FULL + 2;   // every role read the current item (11 arrivals)
+  static constexpr int B_CLC = B_ITEM_READ + 1;         // cluster launch control response written
+  static constexpr int N_BARS = B_CLC + 1;
+  static constexpr int ITEM_READERS = 11;  // 8 softmax warps, the two producers, the issuer
   static constexpr int XCHG_OFF = BAR_OFF + 8 * N_BARS;  // dual stream: tile B's running max, sum per row (2 x 128 fp32)
-  static constexpr int TMEM_SLOT_OFF = XCHG_OFF + 1024;
+  static constexpr int CLC_OFF = (XCHG_OFF + 1024 + 15) / 16 * 16;  // 16-byte cluster launch control response
+  static constexpr int ITEM_OFF = CLC_OFF + 16;                     // work items of units u % 2
+  static constexpr int TMEM_SLOT_OFF = ITEM_OFF + 8;
   static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 4;
   static constexpr int SMEM_USED = ABORT_OFF + 4;
   // 1 KiB of slack to align the base to 1024 bytes (128-byte swizzle atoms);
@@ -129,11 +138,11 @@ struct FwdLayout {
   __device__ static constexpr int v_off(int s) { return s < 2 ? V_OFF + s * V_BYTES : Q_OFF + QK_BYTES; }
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr int THREADS = 384;
-  static constexpr int WARP_TMA = 8, WARP_MMA = 9, WARP_TMA_V = 10;
+  static constexpr int WARP_TMA = 8, WARP_MMA = 9, WARP_TMA_V = 10, WARP_SCHED = 11;
   // Register split: launched at 168 per thread (384 x 168 = 64512); the two
-  // softmax warpgroups grow to 208 and the third (producers, MMA issuer) shrinks
-  // to 80: 2 x 128 x 208 + 128 x 80 = 63488, within the launch's total.
-  static constexpr int REG_SOFTMAX = 208, REG_OTHER = 80;
+  // softmax warpgroups grow to 216 and the third (producers, MMA issuer,
+  // scheduler) shrinks to 72: 2 x 128 x 216 + 128 x 72 = 64512, the launch's total.
+  static constexpr int REG_SOFTMAX = 216, REG_OTHER = 72;
 };
 
 // p = 2^(s * c - m) for one 128-column score row, packed to bf16 pairs; returns
@@ -210,59 +219,81 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
   uint8_t* const sptr = smem_raw + (sbase - raw);
   auto bar = [&](int slot) -> uint32_t { return sbase + L::BAR_OFF + 8u * slot; };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sptr + L::ABORT_OFF);
+  volatile int* item_slot = reinterpret_cast<volatile int*>(sptr + L::ITEM_OFF);
   const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // ---- work decode: groups of bh_group (batch, head) pairs run together, so the
-  // K / V rows they read stay in L2 (heads of one kv group are adjacent); inside a
-  // group, longest units first for causal (blocks are dispatched in index order)
-  const int BH = p.B * (p.H_q >> p.gp_log2);  // (batch, head pack) pairs
-  const int split = static_cast<int>(blockIdx.x) % p.n_splits;  // the splits of one unit are adjacent
-  const int cta = static_cast<int>(blockIdx.x) / p.n_splits;
-  const int per_group = p.bh_group * p.n_units;
-  const int grp = cta / per_group;
-  const int within = cta - grp * per_group;
-  const int gs = min(p.bh_group, BH - grp * p.bh_group);
-  int u = within / gs;
-  const int bh = grp * p.bh_group + (within - u * gs);
-  if (CAUSAL) u = p.n_units - 1 - u;
-  const int b = bh / (p.H_q >> p.gp_log2);
-  const int h0 = (bh - b * (p.H_q >> p.gp_log2)) << p.gp_log2;  // first query head of the pack
-  const int hkv = h0 / (p.H_q / p.H_kv);
-  const int tile_pos = L::BM >> p.gp_log2;  // query positions per tile
-  const int q0 = u * 2 * tile_pos;          // first query position of the unit
-  const int diag = p.S_k - p.S_q;  // bottom-right causal: key j visible to row i iff j <= i + diag
-  // Key block of tile t's step j: j0 + j (both tiles take the same blocks), or in the
-  // dual stream j0 + 2j + t.  nblk[t] steps per tile; the producers load n_loads
-  // blocks j0, j0 + 1, ... in order either way.
-  const int j0 = split * p.split_blocks;
   const bool dual = p.dual != 0;
-  int nblk[2];
-  int n_loads;
-  if (dual) {
-    const int nb_all = min(max(tile_blocks(q0, tile_pos, p.S_q, p.S_k, CAUSAL, L::BN) - j0, 0), p.split_blocks);
-    nblk[0] = (nb_all + 1) / 2;
-    nblk[1] = nb_all / 2;
-    n_loads = nb_all;
-  } else {
-#pragma unroll
-    for (int t = 0; t < 2; ++t)
-      nblk[t] = min(max(tile_blocks(q0 + t * tile_pos, tile_pos, p.S_q, p.S_k, CAUSAL, L::BN) - j0, 0),
-                    p.split_blocks);
-    n_loads = max(nblk[0], nblk[1]);
-  }
-  const int n_blocks = max(nblk[0], nblk[1]);
-  // Q tiles loaded: one per tile, or only tile A's in the dual stream (both tiles read it)
-  const bool q_loaded[2] = {nblk[0] > 0, nblk[1] > 0 && !dual};
+  const int tile_pos = L::BM >> p.gp_log2;  // query positions per tile
+  const int diag = p.S_k - p.S_q;           // bottom-right causal: key j visible to row i iff j <= i + diag
+
+  // ---- work items.  Item n is the work of block n of a one-CTA-per-unit grid:
+  // groups of bh_group (batch, head pack) pairs run together, so the K / V rows
+  // they read stay in L2 (heads of one kv group are adjacent); inside a group the
+  // longest units come first for causal (the hardware starts blocks, and hands
+  // out pending blocks to persistent CTAs, in index order: longest first); the
+  // splits of one unit are adjacent.
+  struct Unit {
+    int b, h0, hkv, q0, j0, split;
+    int nb0, nb1;     // steps of tile A, tile B
+    int n_loads;      // K / V blocks the producers load, in order j0, j0 + 1, ...
+    int n_blocks;     // max(nb0, nb1)
+    bool ql0, ql1;    // Q tiles loaded: one per tile, or only tile A's in the dual stream
+    __device__ int nblk(int t) const { return t == 0 ? nb0 : nb1; }
+    __device__ bool q_loaded(int t) const { return t == 0 ? ql0 : ql1; }
+  };
+  auto decode = [&](int item) {
+    Unit w;
+    const int BH = p.B * (p.H_q >> p.gp_log2);  // (batch, head pack) pairs
+    w.split = item % p.n_splits;
+    const int cta = item / p.n_splits;
+    const int per_group = p.bh_group * p.n_units;
+    const int grp = cta / per_group;
+    const int within = cta - grp * per_group;
+    const int gs = min(p.bh_group, BH - grp * p.bh_group);
+    int u = within / gs;
+    const int bh = grp * p.bh_group + (within - u * gs);
+    if (CAUSAL) u = p.n_units - 1 - u;
+    w.b = bh / (p.H_q >> p.gp_log2);
+    w.h0 = (bh - w.b * (p.H_q >> p.gp_log2)) << p.gp_log2;  // first query head of the pack
+    w.hkv = w.h0 / (p.H_q / p.H_kv);
+    w.q0 = u * 2 * tile_pos;  // first query position of the unit
+    // Key block of tile t's step j: j0 + j (both tiles take the same blocks), or in the
+    // dual stream j0 + 2j + t.
+    w.j0 = w.split * p.split_blocks;
+    if (dual) {
+      const int nb_all = min(max(tile_blocks(w.q0, tile_pos, p.S_q, p.S_k, CAUSAL, L::BN) - w.j0, 0), p.split_blocks);
+      w.nb0 = (nb_all + 1) / 2;
+      w.nb1 = nb_all / 2;
+      w.n_loads = nb_all;
+    } else {
+      w.nb0 = min(max(tile_blocks(w.q0, tile_pos, p.S_q, p.S_k, CAUSAL, L::BN) - w.j0, 0), p.split_blocks);
+      w.nb1 = min(max(tile_blocks(w.q0 + tile_pos, tile_pos, p.S_q, p.S_k, CAUSAL, L::BN) - w.j0, 0), p.split_blocks);
+      w.n_loads = max(w.nb0, w.nb1);
+    }
+    w.n_blocks = max(w.nb0, w.nb1);
+    w.ql0 = w.nb0 > 0;
+    w.ql1 = w.nb1 > 0 && !dual;
+    return w;
+  };
+  // Unit u's item (-1 = no more work) sits in slot u % 2 once ITEM_FULL[u % 2]
+  // completes; every role arrives on ITEM_READ when it has read it, and only then
+  // does the scheduler claim the next unit (one unit ahead of the slowest role).
+  auto read_item = [&](int u) -> int {
+    if (!mbar_wait(bar(L::B_ITEM_FULL + (u & 1)), (u >> 1) & 1, ctl)) return -2;
+    return item_slot[u & 1];
+  };
 
   // ---- setup
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::N_BARS; ++i)
-      mbar_init(bar(i), ((i >= L::B_P_FULL && i < L::B_P_FULL + 4) || i == L::B_XCHG) ? 4u : 1u);
+      mbar_init(bar(i), ((i >= L::B_P_FULL && i < L::B_P_FULL + 4) || i == L::B_XCHG) ? 4u
+                        : i == L::B_ITEM_READ ? static_cast<uint32_t>(L::ITEM_READERS) : 1u);
     *abort_flag = 0;
+    item_slot[0] = static_cast<int>(blockIdx.x);  // unit 0: this block's own item
     fence_mbar_init();
+    mbar_arrive(bar(L::B_ITEM_FULL));
   }
   if (warp == L::WARP_MMA) {
     tmem_alloc(sbase + L::TMEM_SLOT_OFF, L::TMEM_COLS);
@@ -286,357 +317,469 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
   }
   if (warp == L::WARP_TMA) {
     // ===================== TMA producer: Q, K =====================
-    if (lane == 0 && n_blocks > 0) {
+    if (lane == 0) {
+      int kn = 0;              // K blocks loaded (all units)
+      int qn0 = 0, qn1 = 0;    // Q_A, Q_B tiles loaded
+      bool ok = true;
+      for (int u = 0; ok; ++u) {
+        const int item = read_item(u);
+        mbar_arrive(bar(L::B_ITEM_READ));
+        if (item < 0) break;
+        const Unit w = decode(item);
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (!q_loaded[t]) continue;
-        mbar_arrive_expect_tx(bar(L::B_Q_FULL + t), L::QK_BYTES);
+        for (int t = 0; t < 2; ++t) {
+          if (!ok || !w.q_loaded(t)) continue;
+          int& qn = t == 0 ? qn0 : qn1;
+          // the previous unit's last S_t has read Q_t
+          if (qn > 0 && !(ok = mbar_wait(bar(L::B_Q_EMPTY + t), (qn - 1) & 1, ctl))) break;
+          mbar_arrive_expect_tx(bar(L::B_Q_FULL + t), L::QK_BYTES);
 #pragma unroll
-        for (int x = 0; x < L::QK_NBOX; ++x)
-          tma_load_4d(sbase + L::Q_OFF + t * L::QK_BYTES + x * L::BOX_BYTES, &tm_q, bar(L::B_Q_FULL + t),
-                      x * 64, h0, q0 + t * tile_pos, b);
-      }
-      int issued = 0;
-      for (int j = 0; j < n_loads; ++j) {
-        const int s = j % L::KST;
-        if (j >= L::KST && !mbar_wait(bar(L::B_K_EMPTY + s), ((j / L::KST) - 1) & 1, ctl)) break;
-        mbar_arrive_expect_tx(bar(L::B_K_FULL + s), L::QK_BYTES);
+          for (int x = 0; x < L::QK_NBOX; ++x)
+            tma_load_4d(sbase + L::Q_OFF + t * L::QK_BYTES + x * L::BOX_BYTES, &tm_q, bar(L::B_Q_FULL + t),
+                        x * 64, w.h0, w.q0 + t * tile_pos, w.b);
+          ++qn;
+        }
+        for (int j = 0; ok && j < w.n_loads; ++j) {
+          const int s = kn % L::KST;
+          if (kn >= L::KST && !(ok = mbar_wait(bar(L::B_K_EMPTY + s), ((kn / L::KST) - 1) & 1, ctl))) break;
+          mbar_arrive_expect_tx(bar(L::B_K_FULL + s), L::QK_BYTES);
 #pragma unroll
-        for (int x = 0; x < L::QK_NBOX; ++x)
-          tma_load_4d(sbase + L::K_OFF + s * L::QK_BYTES + x * L::BOX_BYTES, &tm_k, bar(L::B_K_FULL + s),
-                      x * 64, hkv, (j0 + j) * L::BN, b);
-        issued = j + 1;
+          for (int x = 0; x < L::QK_NBOX; ++x)
+            tma_load_4d(sbase + L::K_OFF + s * L::QK_BYTES + x * L::BOX_BYTES, &tm_k, bar(L::B_K_FULL + s),
+                        x * 64, w.hkv, (w.j0 + j) * L::BN, w.b);
+          ++kn;
+        }
       }
       // Drain: every load this thread issued has landed before the CTA may exit.
-      for (int t = 0; t < 2; ++t)
-        if (q_loaded[t]) mbar_wait_drain(bar(L::B_Q_FULL + t), 0, 1000000000ull);
-      for (int s = 0; s < L::KST && s < issued; ++s)
-        mbar_wait_drain(bar(L::B_K_FULL + s), ((issued - 1 - s) / L::KST) & 1, 1000000000ull);
+      if (qn0 > 0) mbar_wait_drain(bar(L::B_Q_FULL), (qn0 - 1) & 1, 1000000000ull);
+      if (qn1 > 0) mbar_wait_drain(bar(L::B_Q_FULL + 1), (qn1 - 1) & 1, 1000000000ull);
+      for (int i = 0; i < L::KST && i < kn; ++i) {
+        const int n = kn - 1 - i;
+        mbar_wait_drain(bar(L::B_K_FULL + n % L::KST), (n / L::KST) & 1, 1000000000ull);
+      }
     }
   } else if (warp == L::WARP_TMA_V) {
     // ===================== TMA producer: V =====================
-    if (lane == 0 && n_blocks > 0) {
-      int issued = 0;
-      const int nv = dual ? L::VST_DUAL : L::VST;  // V slots in use
-      for (int j = 0; j < n_loads; ++j) {
-        const int s = j % nv;
-        if (j >= nv && !mbar_wait(bar(L::B_V_EMPTY + s), ((j / nv) - 1) & 1, ctl)) break;
-        mbar_arrive_expect_tx(bar(L::B_V_FULL + s), L::V_BYTES);
+    if (lane == 0) {
+      // V slots in use: VST, or VST_DUAL in the dual stream (the same for every unit)
+      auto load_v = [&](auto nv_c) {
+        constexpr int nv = decltype(nv_c)::value;
+        int vn = 0;  // V blocks loaded (all units)
+        bool ok = true;
+        for (int u = 0; ok; ++u) {
+          const int item = read_item(u);
+          mbar_arrive(bar(L::B_ITEM_READ));
+          if (item < 0) break;
+          const Unit w = decode(item);
+          for (int j = 0; ok && j < w.n_loads; ++j) {
+            const int s = vn % nv;
+            if (vn >= nv && !(ok = mbar_wait(bar(L::B_V_EMPTY + s), ((vn / nv) - 1) & 1, ctl))) break;
+            mbar_arrive_expect_tx(bar(L::B_V_FULL + s), L::V_BYTES);
 #pragma unroll
-        for (int x = 0; x < L::V_NBOX; ++x)
-          tma_load_4d(sbase + L::v_off(s) + x * L::BOX_BYTES, &tm_v, bar(L::B_V_FULL + s),
-                      x * 64, hkv, (j0 + j) * L::BN, b);
-        issued = j + 1;
-      }
-      for (int s = 0; s < nv && s < issued; ++s)
-        mbar_wait_drain(bar(L::B_V_FULL + s), ((issued - 1 - s) / nv) & 1, 1000000000ull);
+            for (int x = 0; x < L::V_NBOX; ++x)
+              tma_load_4d(sbase + L::v_off(s) + x * L::BOX_BYTES, &tm_v, bar(L::B_V_FULL + s),
+                          x * 64, w.hkv, (w.j0 + j) * L::BN, w.b);
+            ++vn;
+          }
+        }
+        for (int i = 0; i < nv && i < vn; ++i) {
+          const int n = vn - 1 - i;
+          mbar_wait_drain(bar(L::B_V_FULL + n % nv), (n / nv) & 1, 1000000000ull);
+        }
+      };
+      if (dual)
+        load_v(std::integral_constant<int, L::VST_DUAL>{});
+      else
+        load_v(std::integral_constant<int, L::VST>{});
     }
   } else if (warp == L::WARP_MMA) {
     // ===================== MMA issuer =====================
-    if (lane == 0 && n_blocks > 0) {
+    if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, false, true);
+      // The shared-memory base goes through an opaque move in each call, so the MMA
+      // descriptors are computed where they are used rather than hoisted out of the
+      // unit and block loops (this warp has 72 registers).
+      auto opaque = [](uint32_t x) {
+        uint32_t y;
+        asm volatile("mov.b32 %0, %1;" : "=r"(y) : "r"(x));
+        return y;
+      };
+      // Descriptors as (low, high) halves: the high half is a constant, and the
+      // descriptor of base + off is the base's low half plus off / 16, one 32-bit add
+      // per MMA.
+      constexpr uint32_t HI = sdesc_sw128_hi(1024);
       auto issue_s = [&](int t, int stage) {
-        const uint32_t q_base = sbase + L::Q_OFF + (dual ? 0 : t) * L::QK_BYTES;
-        const uint32_t k_base = sbase + L::K_OFF + stage * L::QK_BYTES;
+        const uint32_t base = opaque(sbase);
+        const uint32_t qd = sdesc_lo(base + L::Q_OFF + (dual ? 0 : t) * L::QK_BYTES, 16);
+        const uint32_t kd = sdesc_lo(base + L::K_OFF + stage * L::QK_BYTES, 16);
         if constexpr (QK8) {
           // 32 head dims (32 bytes of the 128-byte row) per MMA
 #pragma unroll
           for (int kk = 0; kk < D / 32; ++kk)
-            umma_ss_f8(tmem + L::s_col(t), sdesc_sw128(q_base + kk * 32, 16, 1024),
-                       sdesc_sw128(k_base + kk * 32, 16, 1024), idesc_e4m3_f32(128, 128), kk > 0 ? 1u : 0u);
+            umma_ss_f8_h(tmem + L::s_col(t), qd + (kk * 32 >> 4), HI, kd + (kk * 32 >> 4), HI,
+                         idesc_e4m3_f32(128, 128), kk > 0 ? 1u : 0u);
           umma_commit(bar(L::B_S_FULL + t));
           return;
         }
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::BOX_BYTES + (kk & 3) * 32;
-          umma_ss(tmem + L::s_col(t), sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(k_base + off, 16, 1024),
-                  IDESC_S, kk > 0 ? 1u : 0u);
+          umma_ss_h(tmem + L::s_col(t), qd + (off >> 4), HI, kd + (off >> 4), HI, IDESC_S, kk > 0 ? 1u : 0u);
         }
         umma_commit(bar(L::B_S_FULL + t));
       };
       // PV_t(j) in two halves of 64 keys, each issued once its half of P_t(j) is in TMEM
       auto issue_pv_half = [&](int t, int stage, bool acc, int hf) {
-        const uint32_t v_base = sbase + L::v_off(stage);
+        const uint32_t v_base = opaque(sbase) + L::v_off(stage);
         if constexpr (PV8) {
           // 32 keys per MMA: 8 columns of e4m3 P (4 per column), 32 rows of 128 B of V
           // (MN-major, one 128-byte column block: LBO unused)
           constexpr uint32_t IDESC_PV8 = idesc_e4m3_f32(128, D) | (1u << 16);
+          const uint32_t vd = sdesc_lo(v_base, 16);
 #pragma unroll
           for (int k2 = 0; k2 < 2; ++k2) {
             const int kk = 2 * hf + k2;
-            umma_ts_f8(tmem + L::o_col(t), tmem + L::s_col(t) + kk * 8, sdesc_sw128(v_base + kk * 4096, 16, 1024),
-                       IDESC_PV8, (acc || kk > 0) ? 1u : 0u);
+            umma_ts_f8_h(tmem + L::o_col(t), tmem + L::s_col(t) + kk * 8, vd + (kk * 4096 >> 4), HI, IDESC_PV8,
+                         (acc || kk > 0) ? 1u : 0u);
           }
           return;
         }
+        const uint32_t vd = sdesc_lo(v_base, L::BOX_BYTES);
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
           const int kk = 4 * hf + k4;
           // 16 keys = 16 rows of 128 B = 2048 bytes; 64-wide d blocks are BOX_BYTES apart.
-          umma_ts(tmem + L::o_col(t), tmem + L::s_col(t) + kk * 8,
-                  sdesc_sw128(v_base + kk * 2048, L::BOX_BYTES, 1024), IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+          umma_ts_h(tmem + L::o_col(t), tmem + L::s_col(t) + kk * 8, vd + (kk * 2048 >> 4), HI, IDESC_PV,
+                    (acc || kk > 0) ? 1u : 0u);
         }
-#if ATTN_FWD_PV_WAIT
-        if (hf == 1) umma_commit(bar(L::B_PV_DONE + t));
-#endif
       };
-      if (dual) {
-        // Dual stream: tile t takes key blocks j0 + 2j + t.  Load n = 2j + t sits in K
-        // slot n % KST and V slot n % VST_DUAL; the S and the PV MMAs each consume
-        // their loads in order n = 0, 1, 2, ..., so a running (slot, phase) pair per
-        // ring tracks them.  Each load is used by one tile only.
-        bool ok = true;
-        int ks = 0, kph = 0;  // K slot and phase of the next S MMA
-        int vs = 0, vph = 0;  // V slot and phase of the next PV MMA (V loads are consumed in order too)
-        for (int t = 0; ok && t < 2; ++t) {
-          if (nblk[t] == 0) continue;
-          ok = mbar_wait(bar(L::B_K_FULL + ks), kph, ctl);
-          if (ok && t == 0) ok = mbar_wait(bar(L::B_Q_FULL), 0, ctl);
-          if (ok) {
+      // K / V blocks consumed (all units): ring slot n % KST and n % VST (VST_DUAL in the
+      // dual stream), phase n / KST and n / VST
+      int kc = 0, vc = 0;
+      int qc0 = 0, qc1 = 0;  // Q_A, Q_B tiles consumed
+      int pc0 = 0, pc1 = 0;  // blocks of tile A, tile B processed (S_FULL / P_FULL phases)
+      bool ok = true;
+      for (int u = 0; ok; ++u) {
+        const int item = read_item(u);
+        mbar_arrive(bar(L::B_ITEM_READ));
+        if (item < 0) break;
+        const Unit w = decode(item);
+        if (w.n_blocks == 0) continue;
+        if (dual) {
+          // Dual stream: tile t takes key blocks j0 + 2j + t.  Load n = 2j + t of the unit
+          // is used by one tile only; the S and the PV MMAs each consume their ring in
+          // load order.
+          for (int t = 0; ok && t < 2; ++t) {
+            if (w.nblk(t) == 0) continue;
+            ok = mbar_wait(bar(L::B_K_FULL + kc % L::KST), (kc / L::KST) & 1, ctl);
+            if (ok && t == 0) ok = mbar_wait(bar(L::B_Q_FULL), qc0 & 1, ctl);
+            if (!ok) break;
             tc_fence_after();
-            issue_s(t, ks);
-            umma_commit(bar(L::B_K_EMPTY + ks));
+            issue_s(t, kc % L::KST);
+            umma_commit(bar(L::B_K_EMPTY + kc % L::KST));
+            ++kc;
           }
-          if (++ks == L::KST) { ks = 0; kph ^= 1; }
-        }
-        for (int j = 0; ok && j < n_blocks; ++j) {
+          // both tiles read Q_A: release it after the unit's last S
+          if (ok && w.n_loads <= 2) umma_commit(bar(L::B_Q_EMPTY));
+          for (int j = 0; ok && j < w.n_blocks; ++j) {
 #pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (!ok || j >= nblk[t]) continue;
-            ok = mbar_wait(bar(L::B_V_FULL + vs), vph, ctl) && mbar_wait(bar(L::B_P_FULL + 2 * t), j & 1, ctl);
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv_half(t, vs, j > 0, 0);
-            ok = mbar_wait(bar(L::B_P_FULL + 2 * t + 1), j & 1, ctl);
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv_half(t, vs, j > 0, 1);
-            if (j == nblk[t] - 1) umma_commit(bar(L::B_O_FINAL + t));
-            umma_commit(bar(L::B_V_EMPTY + vs));
-            if (++vs == L::VST_DUAL) { vs = 0; vph ^= 1; }
-            if (j + 1 < nblk[t]) {
-              ok = mbar_wait(bar(L::B_K_FULL + ks), kph, ctl);
-              if (!ok) break;
-              issue_s(t, ks);
-              umma_commit(bar(L::B_K_EMPTY + ks));
-              if (++ks == L::KST) { ks = 0; kph ^= 1; }
-            }
-          }
-        }
-      } else {
-        bool ok = mbar_wait(bar(L::B_K_FULL), 0, ctl);
-        for (int t = 0; ok && t < 2; ++t) {
-          if (nblk[t] == 0) continue;
-          ok = mbar_wait(bar(L::B_Q_FULL + t), 0, ctl);
-          if (ok) {
-            tc_fence_after();
-            issue_s(t, 0);
-          }
-        }
-        if (ok) umma_commit(bar(L::B_K_EMPTY));  // K_0 released once both S(0) complete
-        // Per key block j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1).  S_t(j+1) overwrites
-        // P_t(j), which PV_t(j) reads: the MMAs of this one issuing thread execute
-        // in issue order, so PV_t(j) has read P_t(j) before S_t(j+1) writes there
-        // (ATTN_FWD_PV_WAIT=1 makes the issuer wait for PV_t(j) to complete instead).
-        for (int j = 0; ok && j < n_blocks; ++j) {
-          const int vs = j % L::VST;
-          const int ks1 = (j + 1) % L::KST;
-          if (!mbar_wait(bar(L::B_V_FULL + vs), (j / L::VST) & 1, ctl)) break;
-          bool k_next_ready = false;
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (!ok || j >= nblk[t]) continue;
-            ok = mbar_wait(bar(L::B_P_FULL + 2 * t), j & 1, ctl);
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv_half(t, vs, j > 0, 0);
-            ok = mbar_wait(bar(L::B_P_FULL + 2 * t + 1), j & 1, ctl);
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv_half(t, vs, j > 0, 1);
-            if (j == nblk[t] - 1) umma_commit(bar(L::B_O_FINAL + t));
-            if (j + 1 < nblk[t]) {
-              if (!k_next_ready) {
-                ok = mbar_wait(bar(L::B_K_FULL + ks1), ((j + 1) / L::KST) & 1, ctl);
-                if (!ok) break;
-                k_next_ready = true;
-              }
-#if ATTN_FWD_PV_WAIT
-              ok = mbar_wait(bar(L::B_PV_DONE + t), j & 1, ctl);
+            for (int t = 0; t < 2; ++t) {
+              if (!ok || j >= w.nblk(t)) continue;
+              const int vs = vc % L::VST_DUAL;
+              ok = mbar_wait(bar(L::B_V_FULL + vs), (vc / L::VST_DUAL) & 1, ctl) &&
+                   mbar_wait(bar(L::B_P_FULL + 2 * t), ((t == 0 ? pc0 : pc1) + j) & 1, ctl);
               if (!ok) break;
               tc_fence_after();
-#endif
-              issue_s(t, ks1);
+              issue_pv_half(t, vs, j > 0, 0);
+              ok = mbar_wait(bar(L::B_P_FULL + 2 * t + 1), ((t == 0 ? pc0 : pc1) + j) & 1, ctl);
+              if (!ok) break;
+              tc_fence_after();
+              issue_pv_half(t, vs, j > 0, 1);
+              if (j == w.nblk(t) - 1) umma_commit(bar(L::B_O_FINAL + t));
+              umma_commit(bar(L::B_V_EMPTY + vs));
+              ++vc;
+              if (j + 1 < w.nblk(t)) {
+                const int ks = kc % L::KST;
+                ok = mbar_wait(bar(L::B_K_FULL + ks), (kc / L::KST) & 1, ctl);
+                if (!ok) break;
+                issue_s(t, ks);
+                umma_commit(bar(L::B_K_EMPTY + ks));
+                // the unit's last S reads Q_A (both tiles use it): release it after that one
+                if (2 * (j + 1) + t == w.n_loads - 1) umma_commit(bar(L::B_Q_EMPTY));
+                ++kc;
+              }
             }
           }
+        } else {
+          // S_t(0) of both tiles on K_0 of the unit.  This overwrites S_t / P_t of the
+          // previous unit, whose PV MMAs this thread issued first.
+          ok = mbar_wait(bar(L::B_K_FULL + kc % L::KST), (kc / L::KST) & 1, ctl);
+          for (int t = 0; ok && t < 2; ++t) {
+            if (w.nblk(t) == 0) continue;
+            ok = mbar_wait(bar(L::B_Q_FULL + t), (t == 0 ? qc0 : qc1) & 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(t, kc % L::KST);
+            if (w.nblk(t) == 1) umma_commit(bar(L::B_Q_EMPTY + t));  // the unit's last S_t has been issued
+          }
           if (!ok) break;
-          umma_commit(bar(L::B_V_EMPTY + vs));
-          if (k_next_ready) umma_commit(bar(L::B_K_EMPTY + ks1));
+          umma_commit(bar(L::B_K_EMPTY + kc % L::KST));  // K_0 released once both S(0) complete
+          ++kc;
+          // Per key block j: PV_A(j), S_A(j+1), PV_B(j), S_B(j+1).  S_t(j+1) overwrites
+          // P_t(j), which PV_t(j) reads: the MMAs of this one issuing thread execute
+          // in issue order, so PV_t(j) has read P_t(j) before S_t(j+1) writes there.
+          // The first PV_t of a unit overwrites O_t: the softmax publishes P_t(0) only
+          // after its epilogue has read the previous unit's O_t.
+          for (int j = 0; ok && j < w.n_blocks; ++j) {
+            const int vs = vc % L::VST;
+            const int ks1 = kc % L::KST;
+            if (!(ok = mbar_wait(bar(L::B_V_FULL + vs), (vc / L::VST) & 1, ctl))) break;
+            bool k_next_ready = false;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (!ok || j >= w.nblk(t)) continue;
+              ok = mbar_wait(bar(L::B_P_FULL + 2 * t), ((t == 0 ? pc0 : pc1) + j) & 1, ctl);
+              if (!ok) break;
+              tc_fence_after();
+              issue_pv_half(t, vs, j > 0, 0);
+              ok = mbar_wait(bar(L::B_P_FULL + 2 * t + 1), ((t == 0 ? pc0 : pc1) + j) & 1, ctl);
+              if (!ok) break;
+              tc_fence_after();
+              issue_pv_half(t, vs, j > 0, 1);
+              if (j == w.nblk(t) - 1) umma_commit(bar(L::B_O_FINAL + t));
+              if (j + 1 < w.nblk(t)) {
+                if (!k_next_ready) {
+                  ok = mbar_wait(bar(L::B_K_FULL + ks1), (kc / L::KST) & 1, ctl);
+                  if (!ok) break;
+                  k_next_ready = true;
+                }
+                issue_s(t, ks1);
+                if (j + 2 == w.nblk(t)) umma_commit(bar(L::B_Q_EMPTY + t));  // the unit's last S_t
+              }
+            }
+            if (!ok) break;
+            umma_commit(bar(L::B_V_EMPTY + vs));
+            ++vc;
+            if (k_next_ready) {
+              umma_commit(bar(L::B_K_EMPTY + ks1));
+              ++kc;
+            }
+          }
         }
+        pc0 += w.nb0;
+        pc1 += w.nb1;
+        qc0 += w.ql0 ? 1 : 0;
+        qc1 += w.ql1 ? 1 : 0;
       }
       // Drain: no MMA may still be writing TMEM when it is released.
       umma_commit(bar(L::B_DRAIN));
       mbar_wait_drain(bar(L::B_DRAIN), 0, 1000000000ull);
+    }
+  } else if (warp == L::WARP_SCHED) {
+    // ===================== work scheduler =====================
+    // Unit u + 1's item: once every role has read unit u's, the next pending block of
+    // the grid (the hardware's launch order) is cancelled and its item taken over.
+    // Without the persistent mode, or once no block is left, the item is -1.
+    if (lane == 0) {
+      int item = static_cast<int>(blockIdx.x);
+      uint32_t clc_phase = 0;
+      for (int u = 0;; ++u) {
+        if (!mbar_wait(bar(L::B_ITEM_READ), u & 1, ctl)) break;
+        int next = -1;
+        if (p.persistent && item >= 0) {
+          mbar_arrive_expect_tx(bar(L::B_CLC), 16);
+          clc_try_cancel(sbase + L::CLC_OFF, bar(L::B_CLC));
+          if (!mbar_wait(bar(L::B_CLC), clc_phase, ctl)) break;
+          clc_phase ^= 1;
+          next = clc_cancelled_block(sbase + L::CLC_OFF);
+        }
+        item_slot[(u + 1) & 1] = next;
+        mbar_arrive(bar(L::B_ITEM_FULL + ((u + 1) & 1)));
+        item = next;
+        if (next < 0) break;
+      }
     }
   } else if (warp < 8) {
     // ===================== softmax warpgroups (warps 0-3: tile A, 4-7: tile B) =====================
     setmaxnreg_inc<L::REG_SOFTMAX>();
     const int t = warp >> 2;
     const int row = threadIdx.x & 127;  // == TMEM lane
-    const int row0 = q0 + (dual ? 0 : t * tile_pos);  // first query position of the tile
-    const int qi = row0 + (row >> p.gp_log2);     // this row's query position
-    const int h = h0 + (row & (p.gp - 1));        // and query head
-    const int nb = nblk[t];
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float c = p.scale_log2;
-    const int lim = min(qi + (CAUSAL ? diag : p.S_k), p.S_k - 1);  // last visible key of this row
-    const int lim_tile = CAUSAL ? row0 + diag : p.S_k - 1;         // last key every row of the tile sees
-    float m_used = -INFINITY;
-    float l = 0.f;
-    unsigned rescales = 0;
+    int sc = 0;  // blocks of this tile processed (S_FULL / P_FULL phases)
+    int oc = 0;  // O_FINAL phases consumed
     bool ok = true;
-    for (int j = 0; j < nb; ++j) {
-      ok = mbar_wait(bar(L::B_S_FULL + t), j & 1, ctl);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[128];
-      const uint32_t s_addr = tmem + lane_addr + L::s_col(t);
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) tmem_ld32(s_addr + ch * 32, sr + ch * 32);
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) tmem_ld_wait(sr + ch * 32);
-
-      float* s = reinterpret_cast<float*>(sr);
-      const int kbase = (j0 + (dual ? 2 * j + t : j)) * L::BN;
-      const bool need_mask = (kbase + L::BN - 1 > lim_tile) || (kbase + L::BN > p.S_k);
-      if (need_mask) {
-        const int lim_c = lim - kbase;
-#pragma unroll
-        for (int cc = 0; cc < 128; ++cc)
-          if (cc > lim_c) s[cc] = -INFINITY;
+    for (int u = 0; ok; ++u) {
+      const int item = read_item(u);
+      if (item < 0) {
+        mbar_arrive_warp(bar(L::B_ITEM_READ));
+        break;
       }
-      const float mx = row_max128(sr);
-      const float m_new = fmaxf(m_used, mx * c);
-      const bool resc = (m_new - m_used) > p.tau;  // false for NaN (-inf - -inf)
-      float alpha = 1.f;
-      if (resc) {
-        alpha = exp2_mufu(m_used - m_new);  // 0 when m_used = -inf
-        m_used = m_new;
-        l *= alpha;
-        if (j > 0) ++rescales;
+      int nb, kb0, lim, lim_tile;  // the key-block loop needs only these (the rest is decoded again after it)
+      {
+        const Unit w = decode(item);
+        const int row0 = w.q0 + (dual ? 0 : t * tile_pos);  // first query position of the tile
+        const int qi = row0 + (row >> p.gp_log2);           // this row's query position
+        nb = w.nblk(t);
+        kb0 = w.j0 * L::BN;
+        lim = min(qi + (CAUSAL ? diag : p.S_k), p.S_k - 1);  // last visible key of this row
+        lim_tile = CAUSAL ? row0 + diag : p.S_k - 1;         // last key every row of the tile sees
       }
-      const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
-      if (j > 0 && __any_sync(0xffffffffu, resc)) {
-        // PV_t(j-1) completed before S_t(j) was issued, so O_t is final up to block
-        // j-1; it is rescaled before any part of P_t(j) is published.
-        const uint32_t o_addr = tmem + lane_addr + L::o_col(t);
-#pragma unroll 1
-        for (int ch = 0; ch < D / 32; ++ch) {
-          uint32_t orr[32];
-          tmem_ld32(o_addr + ch * 32, orr);
-          tmem_ld_wait(orr);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
-          tmem_st32(o_addr + ch * 32, orr);
-        }
-      }
-      // P_t(j) over the first 64 columns of S_t (32 for e4m3 P), published in two
-      // halves (keys 0-63, then 64-127) so the PV MMA starts on the first while the
-      // second is computed.
-      // Masked blocks take MUFU ex2 only: it maps -inf to an exact 0.
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t pk[32];
-        l += need_mask ? exp_half<0, PV8>(sr, c, m_eff, pk, hf) : exp_half<POLY_EVERY, PV8>(sr, c, m_eff, pk, hf);
-        if constexpr (PV8)
-          tmem_st16(s_addr + 16 * hf, pk);  // 64 keys as e4m3: 16 columns
-        else
-          tmem_st32(s_addr + 32 * hf, pk);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive_warp(bar(L::B_P_FULL + 2 * t + hf));
-      }
-    }
-    if (p.rescale_count != nullptr && rescales) atomicAdd(p.rescale_count, (unsigned long long)rescales);
-
-    // ---- epilogue: O / l -> bf16 (or the split's fp32 O_s), lse
-    if (ok && nb > 0) {
-      ok = mbar_wait(bar(L::B_O_FINAL + t), 0, ctl);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    float* xch = reinterpret_cast<float*>(sptr + L::XCHG_OFF);
-    if (dual && t == 1) {
-      // tile B hands its row statistics to tile A, which merges both halves
-      xch[row] = m_used;
-      xch[128 + row] = l;
-      mbar_arrive_warp(bar(L::B_XCHG));
-    } else if (ok) {
-      // Row result = (w_A O_A + w_B O_B) / (w_A l_A + w_B l_B), w = 2^(m - max m): the
-      // log-sum-exp merge of the two key halves in the dual stream; only this tile's
-      // O (w = 1) otherwise.  A half that saw no key has l = 0 and weight 0, and its O
-      // columns are never read into the result (select, not multiply).
-      float m_b = -INFINITY, l_b = 0.f;
-      const bool have_b = dual && nblk[1] > 0;
-      if (dual) {
-        ok = mbar_wait(bar(L::B_XCHG), 0, ctl);
-        if (ok && have_b) ok = mbar_wait(bar(L::B_O_FINAL + 1), 0, ctl);
-        ok = __all_sync(0xffffffffu, ok);
-        m_b = xch[row];
-        l_b = xch[128 + row];
-      }
-      if (ok) {
+      float m_used = -INFINITY;
+      float l = 0.f;
+      unsigned rescales = 0;
+      // The next unit is claimed once every role has read this one; the softmax
+      // warps count as having read it only when they start the unit's last block,
+      // so a CTA does not hold on to pending work while it still has much of its own.
+      if (nb == 0) mbar_arrive_warp(bar(L::B_ITEM_READ));
+      for (int j = 0; j < nb; ++j) {
+        if (j == nb - 1) mbar_arrive_warp(bar(L::B_ITEM_READ));
+        ok = mbar_wait(bar(L::B_S_FULL + t), (sc + j) & 1, ctl);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
-        const float mx = fmaxf(m_used, m_b);
-        const float w_a = l > 0.f ? exp2_mufu(m_used - mx) : 0.f;
-        const float w_b = l_b > 0.f ? exp2_mufu(m_b - mx) : 0.f;
-        const float lsum = l * w_a + l_b * w_b;
-        const float inv_l = lsum > 0.f ? 1.f / lsum : 0.f;
-        const float c_a = w_a * inv_l, c_b = w_b * inv_l;
-        const float lse_v = lsum > 0.f ? (mx + __log2f(lsum)) * 0.69314718055994531f : -INFINITY;
-        const bool valid = qi < p.S_q;
-        const uint32_t oa_addr = tmem + lane_addr + L::o_col(t);
-        const uint32_t ob_addr = tmem + lane_addr + L::o_col(1);
-        const size_t part = static_cast<size_t>(split) * p.B + b;
+        uint32_t sr[128];
+        const uint32_t s_addr = tmem + lane_addr + L::s_col(t);
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) tmem_ld32(s_addr + ch * 32, sr + ch * 32);
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) tmem_ld_wait(sr + ch * 32);
+
+        float* s = reinterpret_cast<float*>(sr);
+        const int kbase = kb0 + (dual ? 2 * j + t : j) * L::BN;
+        const bool need_mask = (kbase + L::BN - 1 > lim_tile) || (kbase + L::BN > p.S_k);
+        if (need_mask) {
+          const int lim_c = lim - kbase;
+#pragma unroll
+          for (int cc = 0; cc < 128; ++cc)
+            if (cc > lim_c) s[cc] = -INFINITY;
+        }
+        const float mx = row_max128(sr);
+        const float m_new = fmaxf(m_used, mx * c);
+        const bool resc = (m_new - m_used) > p.tau;  // false for NaN (-inf - -inf)
+        float alpha = 1.f;
+        if (resc) {
+          alpha = exp2_mufu(m_used - m_new);  // 0 when m_used = -inf
+          m_used = m_new;
+          l *= alpha;
+          if (j > 0) ++rescales;
+        }
+        const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
+        if (j > 0 && __any_sync(0xffffffffu, resc)) {
+          // PV_t(j-1) completed before S_t(j) was issued, so O_t is final up to block
+          // j-1; it is rescaled before any part of P_t(j) is published.
+          const uint32_t o_addr = tmem + lane_addr + L::o_col(t);
 #pragma unroll 1
-        for (int ch = 0; ch < D / 16; ++ch) {  // 16 columns at a time
-          uint32_t orr[16], obr[16];
-          if (nb > 0) {
-            tmem_ld16(oa_addr + ch * 16, orr);
-            tmem_ld_wait16(orr);
-          }
-          if (have_b) {
-            tmem_ld16(ob_addr + ch * 16, obr);
-            tmem_ld_wait16(obr);
-          }
-          float* ov = reinterpret_cast<float*>(orr);  // the result, in place
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t orr[32];
+            tmem_ld32(o_addr + ch * 32, orr);
+            tmem_ld_wait(orr);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float v = (nb > 0 && w_a > 0.f) ? __uint_as_float(orr[i]) * c_a : 0.f;
-            if (have_b && w_b > 0.f) v += __uint_as_float(obr[i]) * c_b;
-            ov[i] = v;
-          }
-          if (!valid) continue;
-          if (p.n_splits > 1) {
-            // partial result of this split: fp32 O_s
-            float4* dst = reinterpret_cast<float4*>(p.o_part + ((part * p.S_q + qi) * p.H_q + h) * D + ch * 16);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) dst[i] = make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
-          } else {
-            uint32_t pkd[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) pkd[i] = pack_bf16x2(ov[2 * i], ov[2 * i + 1]);
-            uint4* dst = reinterpret_cast<uint4*>(p.o + ((static_cast<size_t>(b) * p.S_q + qi) * p.H_q + h) * D + ch * 16);
-            dst[0] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
-            dst[1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
+            for (int i = 0; i < 32; ++i) orr[i] = __float_as_uint(__uint_as_float(orr[i]) * alpha);
+            tmem_st32(o_addr + ch * 32, orr);
           }
         }
-        if (valid) {
-          if (p.n_splits > 1)
-            p.lse_part[(part * p.H_q + h) * p.S_q + qi] = lse_v;
+        // P_t(j) over the first 64 columns of S_t (32 for e4m3 P), published in two
+        // halves (keys 0-63, then 64-127) so the PV MMA starts on the first while the
+        // second is computed.
+        // Masked blocks take MUFU ex2 only: it maps -inf to an exact 0.
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t pk[32];
+          l += need_mask ? exp_half<0, PV8>(sr, c, m_eff, pk, hf) : exp_half<POLY_EVERY, PV8>(sr, c, m_eff, pk, hf);
+          if constexpr (PV8)
+            tmem_st16(s_addr + 16 * hf, pk);  // 64 keys as e4m3: 16 columns
           else
-            p.lse[(static_cast<size_t>(b) * p.H_q + h) * p.S_q + qi] = lse_v;
+            tmem_st32(s_addr + 32 * hf, pk);
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive_warp(bar(L::B_P_FULL + 2 * t + hf));
+        }
+      }
+      sc += nb;
+      if (p.rescale_count != nullptr && rescales) atomicAdd(p.rescale_count, (unsigned long long)rescales);
+      const Unit w = decode(item);
+      const int qi = w.q0 + (dual ? 0 : t * tile_pos) + (row >> p.gp_log2);  // this row's query position
+      const int h = w.h0 + (row & (p.gp - 1));                                 // and query head
+
+      // ---- epilogue: O / l -> bf16 (or the split's fp32 O_s), lse
+      if (ok && nb > 0) {
+        ok = mbar_wait(bar(L::B_O_FINAL + t), oc & 1, ctl);
+        ok = __all_sync(0xffffffffu, ok);
+        ++oc;
+      }
+      float* xch = reinterpret_cast<float*>(sptr + L::XCHG_OFF);
+      if (dual && t == 1) {
+        // tile B hands its row statistics to tile A, which merges both halves
+        xch[row] = m_used;
+        xch[128 + row] = l;
+        mbar_arrive_warp(bar(L::B_XCHG));
+      } else if (ok) {
+        // Row result = (w_A O_A + w_B O_B) / (w_A l_A + w_B l_B), w = 2^(m - max m): the
+        // log-sum-exp merge of the two key halves in the dual stream; only this tile's
+        // O (w = 1) otherwise.  A half that saw no key has l = 0 and weight 0, and its O
+        // columns are never read into the result (select, not multiply).
+        float m_b = -INFINITY, l_b = 0.f;
+        const bool have_b = dual && w.nblk(1) > 0;
+        if (dual) {
+          ok = mbar_wait(bar(L::B_XCHG), 0, ctl);
+          if (ok && have_b) ok = mbar_wait(bar(L::B_O_FINAL + 1), 0, ctl);
+          ok = __all_sync(0xffffffffu, ok);
+          m_b = xch[row];
+          l_b = xch[128 + row];
+        }
+        if (ok) {
+          tc_fence_after();
+          const float mx = fmaxf(m_used, m_b);
+          const float w_a = l > 0.f ? exp2_mufu(m_used - mx) : 0.f;
+          const float w_b = l_b > 0.f ? exp2_mufu(m_b - mx) : 0.f;
+          const float lsum = l * w_a + l_b * w_b;
+          const float inv_l = lsum > 0.f ? 1.f / lsum : 0.f;
+          const float c_a = w_a * inv_l, c_b = w_b * inv_l;
+          const float lse_v = lsum > 0.f ? (mx + __log2f(lsum)) * 0.69314718055994531f : -INFINITY;
+          const bool valid = qi < p.S_q;
+          const uint32_t oa_addr = tmem + lane_addr + L::o_col(t);
+          const uint32_t ob_addr = tmem + lane_addr + L::o_col(1);
+          const size_t part = static_cast<size_t>(w.split) * p.B + w.b;
+#pragma unroll 1
+          for (int ch = 0; ch < D / 16; ++ch) {  // 16 columns at a time
+            uint32_t orr[16], obr[16];
+            if (nb > 0) {
+              tmem_ld16(oa_addr + ch * 16, orr);
+              tmem_ld_wait16(orr);
+            }
+            if (have_b) {
+              tmem_ld16(ob_addr + ch * 16, obr);
+              tmem_ld_wait16(obr);
+            }
+            float* ov = reinterpret_cast<float*>(orr);  // the result, in place
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float v = (nb > 0 && w_a > 0.f) ? __uint_as_float(orr[i]) * c_a : 0.f;
+              if (have_b && w_b > 0.f) v += __uint_as_float(obr[i]) * c_b;
+              ov[i] = v;
+            }
+            if (!valid) continue;
+            if (p.n_splits > 1) {
+              // partial result of this split: fp32 O_s
+              float4* dst = reinterpret_cast<float4*>(p.o_part + ((part * p.S_q + qi) * p.H_q + h) * D + ch * 16);
+#pragma unroll
+              for (int i = 0; i < 4; ++i) dst[i] = make_float4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
+            } else {
+              uint32_t pkd[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) pkd[i] = pack_bf16x2(ov[2 * i], ov[2 * i + 1]);
+              uint4* dst = reinterpret_cast<uint4*>(p.o + ((static_cast<size_t>(w.b) * p.S_q + qi) * p.H_q + h) * D + ch * 16);
+              dst[0] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
+              dst[1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
+            }
+          }
+          if (valid) {
+            if (p.n_splits > 1)
+              p.lse_part[(part * p.H_q + h) * p.S_q + qi] = lse_v;
+            else
+              p.lse[(static_cast<size_t>(w.b) * p.H_q + h) * p.S_q + qi] = lse_v;
+          }
         }
       }
     }

@@ -484,10 +484,14 @@ def run_configs(attn, dev, flush, peaks):
             ms, reps = timed_calls(lambda: attn.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse),
                                    flush, stream)
         c = clk.summary()
+        # the same forward with one CTA per work unit instead of persistent CTAs
+        ms1, _ = timed_calls(lambda: attn.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse,
+                                              persistent=False), flush, stream)
         tf = w.fwd_flops() / (ms * 1e-3) / 1e12
         e = {"ms": round(ms, 4), "tflops": round(tf, 1), "frac_of_measured": round(tf / peak, 4),
              "frac_of_spec_2250": round(tf / SPEC_PEAK_TFLOPS, 4), "reps": reps,
-             "sm_mhz": c["sm_mhz"], "clock_samples": c.get("samples"), "clock_reasons": c["reasons"]}
+             "sm_mhz": c["sm_mhz"], "clock_samples": c.get("samples"), "clock_reasons": c["reasons"],
+             "one_cta_per_unit": {"ms": round(ms1, 4), "tflops": round(w.fwd_flops() / (ms1 * 1e-3) / 1e12, 1)}}
         # O rescales counted at the default threshold (tau = 8) and with a rescale on
         # every increase of the running max (tau = 0)
         counts = {}

@@ -88,11 +88,22 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
  *   rescale_count     : optional device pointer to an unsigned 64-bit counter;
  *                       the kernel adds the number of (row, key block) O rescales
  *                       it performed after a row's first block.  NULL = off.
+ *   persistent        : 1 (default) = persistent CTAs: a CTA that finishes its
+ *                       work unit (256 query rows of one head, or a key range of
+ *                       one in the split forward) claims the unit of a CTA that
+ *                       has not started yet -- the grid lists units longest first
+ *                       for causal -- and runs it with the barriers, rings and
+ *                       tensor memory it holds, loading the next unit's tiles
+ *                       while it finishes the current one (a persistent tile
+ *                       scheduler; Blackwell cluster launch control).  0 = one
+ *                       CTA per unit.  Ignored when one tile holds every query
+ *                       row (the two tiles then split the keys instead).
  */
 typedef struct {
   float rescale_threshold;
   int poly_exp_every;
   unsigned long long* rescale_count;
+  int persistent;
 } attn_fwd_options_t;
 
 /* Fills `opt` with the defaults above. */

@@ -58,6 +58,7 @@ def test_fwd_options_validation(lib):
     opt = _abi.FwdOptions()
     lib.attn_fwd_default_options(ctypes.byref(opt))
     assert opt.rescale_threshold == 8.0 and opt.poly_exp_every == 8 and opt.rescale_count is None
+    assert opt.persistent == 1
     for field, bad in (("rescale_threshold", -1.0), ("rescale_threshold", 17.0), ("poly_exp_every", 3)):
         o = _abi.FwdOptions(opt.rescale_threshold, opt.poly_exp_every, None)
         setattr(o, field, bad)

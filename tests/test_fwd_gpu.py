@@ -161,3 +161,26 @@ def test_packed_query_heads_d64():
     o_ref, lse_ref = ref.forward(x["q"], x["k"], x["v"], True, w.scale)
     parity.check_o(o, o_ref, w.name)
     parity.check_lse(lse, lse_ref, w.name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("B,H_q,H_kv,S,D", [(8, 16, 16, 640, 128), (4, 12, 4, 1000, 64), (2, 40, 8, 2304, 128)])
+def test_persistent_ctas_match_one_cta_per_unit(B, H_q, H_kv, S, D, causal):
+    # more work units than SMs: persistent CTAs take over the units of CTAs that have not
+    # started (several units each, of different lengths when causal).  Each unit's
+    # arithmetic is the same either way, so the results are bitwise equal; and they
+    # match the oracle.
+    w = workloads.small(B=B, H_q=H_q, H_kv=H_kv, S_q=S, S_k=S, D=D, causal=causal, seed=B * S + H_q)
+    x = workloads.make_inputs(w)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    o1, l1 = _attn().fwd(q, k, v, causal=causal, scale=w.scale, persistent=True)
+    o2, l2 = _attn().fwd(q, k, v, causal=causal, scale=w.scale, persistent=False)
+    torch.cuda.synchronize()
+    assert _attn().device_status() == 0
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    o_c, l_c = o1.cpu(), l1.cpu()
+    for (b, h) in [(0, 0), (B - 1, H_q - 1), (B // 2, H_q // 2)]:
+        rows = sorted(set(range(0, min(S, 300))) | set(range(max(0, S - 300), S)))
+        o_ref, lse_ref = ref.forward_rows(x["q"], x["k"], x["v"], causal, w.scale, b, h, rows)
+        parity.check_o(o_c[b, rows, h, :], o_ref, f"{w.name} b={b} h={h}")
+        parity.check_lse(l_c[b, h, rows], lse_ref, f"{w.name} b={b} h={h}")
