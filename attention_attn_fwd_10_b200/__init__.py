@@ -184,12 +184,14 @@ def bwd_workspace_size(B, H_q, S_q, D) -> int:
 
 
 def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, dq=None, dk=None, dv=None,
-        workspace=None, stream=None, main_pass_events=None, deterministic: bool = False):
+        workspace=None, stream=None, main_pass_events=None, deterministic: bool = False, cta_mode: int = 0):
     """Backward attention.  Returns (dq, dk, dv) bf16 with the shapes of q, k, v.
 
     ``main_pass_events``: optional (start, stop) torch.cuda.Event pair recorded
     around the main-pass kernel (diagnostic timing).  ``deterministic``: add the
-    dQ parts of each query block in key-tile order (bitwise reproducible dQ)."""
+    dQ parts of each query block in key-tile order (bitwise reproducible dQ).
+    ``cta_mode``: 0 / 1 = one CTA per key tile (default), 2 = CTA pairs whose
+    tensor cores execute each MMA together (head dim 128)."""
     on_host = not q.is_cuda
     if on_host:
         dev = torch.device("cuda", torch.cuda.current_device())
@@ -215,7 +217,7 @@ def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, d
     dev = _device_of(q, k, v, o, lse, do, dq, dk, dv, workspace)
     opt = None
     with torch.cuda.device(dev):
-        if main_pass_events is not None or deterministic:
+        if main_pass_events is not None or deterministic or cta_mode:
             ev = (None, None)
             if main_pass_events is not None:
                 s = torch.cuda.current_stream(dev) if stream is None else stream
@@ -223,7 +225,7 @@ def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, d
                     if e.cuda_event == 0:  # torch creates the CUDA event lazily, on its first record
                         e.record(s)
                 ev = (main_pass_events[0].cuda_event, main_pass_events[1].cuda_event)
-            opt = ctypes.byref(_abi.BwdOptions(ev[0], ev[1], int(bool(deterministic))))
+            opt = ctypes.byref(_abi.BwdOptions(ev[0], ev[1], int(bool(deterministic)), int(cta_mode)))
         code = load().attn_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                                   do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
                                   B, H_q, H_kv, S_q, S_k, D, int(bool(causal)), scale, opt,

@@ -60,7 +60,7 @@ class BwdOptions(ctypes.Structure):
     """attn_bwd_options_t"""
 
     _fields_ = [("main_pass_start", ctypes.c_void_p), ("main_pass_stop", ctypes.c_void_p),
-                ("deterministic", ctypes.c_int)]
+                ("deterministic", ctypes.c_int), ("cta_mode", ctypes.c_int)]
 
 
 _vp = ctypes.c_void_p

@@ -11,6 +11,7 @@
 
 #include "../../include/attn.h"
 #include "bwd_kernels.cuh"
+#include "bwd_pair_kernel.cuh"
 #include "fwd_kernel.cuh"
 #include "sm100_common.cuh"
 
@@ -84,16 +85,17 @@ bool make_bshd_map(CUtensorMap* map, const void* ptr, int B, int S, int H, int D
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// fp32 [B, S, H, D] dQ accumulator viewed as (D, H, S, B); boxes of D x 1 x 64 x 1
-// (whole 64-query blocks), no swizzle: the target of the backward's TMA reduce-adds.
-bool make_dqacc_map(CUtensorMap* map, void* ptr, int B, int S, int H, int D) {
+// fp32 [B, S, H, D] dQ accumulator viewed as (D, H, S, B); boxes of box_d x 1 x 64 x 1
+// (whole 64-query blocks; all D dims, or half of them for a CTA of a pair), no
+// swizzle: the target of the backward's TMA reduce-adds.
+bool make_dqacc_map(CUtensorMap* map, void* ptr, int B, int S, int H, int D, int box_d) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
                               static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(B)};
   const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 4, static_cast<cuuint64_t>(H) * D * 4,
                                  static_cast<cuuint64_t>(S) * H * D * 4};
-  const cuuint32_t box[4] = {static_cast<cuuint32_t>(D), 1, 64, 1};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(box_d), 1, 64, 1};
   const cuuint32_t estride[4] = {1, 1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ptr, dims, strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -238,6 +240,20 @@ cudaError_t launch_bwd(const CUtensorMap& mk, const CUtensorMap& mv, const CUten
   return cudaGetLastError();
 }
 
+template <bool CAUSAL, bool DET>
+cudaError_t launch_bwd_pair(const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mq32,
+                            const CUtensorMap& mdo32, const CUtensorMap& mq64, const CUtensorMap& mdo64,
+                            const CUtensorMap& mdq, const BwdParams& p, unsigned grid, cudaStream_t st) {
+  using L = BwdPairLayout<DET>;
+  auto kern = attn_bwd_pair_kernel<CAUSAL, DET>;
+  static CUcontext seen[kMaxDevices] = {};
+  const cudaError_t attr_err = smem_opt_in(kern, L::SMEM_BYTES, seen);
+  if (attr_err != cudaSuccess) return attr_err;
+  // the kernel is declared with a cluster size of two: grid is a multiple of two
+  kern<<<grid, L::THREADS, L::SMEM_BYTES, st>>>(mk, mv, mq32, mdo32, mq64, mdo64, mdq, p);
+  return cudaGetLastError();
+}
+
 // Reads and clears the status word in one atomic step (a timeout recorded by a
 // kernel on another stream is never lost between a read and a clear).
 __global__ void take_status_kernel(int* status, int* taken) { *taken = atomicExch(status, 0); }
@@ -367,7 +383,7 @@ using namespace attn;
 
 extern "C" {
 
-int attn_abi_version(void) { return 3; }
+int attn_abi_version(void) { return 4; }
 
 const char* attn_status_string(attn_status_t s) {
   switch (s) {
@@ -500,6 +516,9 @@ attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const voi
   const size_t sem_bytes = (static_cast<size_t>(B) * H_q * (s_pad / 64) * sizeof(int) + 255) / 256 * 256;
   p.ticket = reinterpret_cast<int*>(ws + dq_bytes + 2 * row_bytes + sem_bytes);
   const bool det = opt && opt->deterministic;
+  const int cta_mode = opt ? opt->cta_mode : 0;
+  if (cta_mode < 0 || cta_mode > 2 || (cta_mode == 2 && D != 128)) return ATTN_ERR_INVALID_ARG;
+  const bool pairs = cta_mode == 2;  // default: one CTA per tile (the faster kernel on B200)
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
@@ -516,10 +535,12 @@ attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const voi
   p.status = status;
   p.wait_limit_ns = g_wait_limit_ns.load();
 
-  CUtensorMap mk, mv, mq, mdo, mdq;
+  CUtensorMap mk, mv, mq, mdo, mdq, mq32, mdo32;
   if (!make_bshd_map(&mk, k, B, S_k, H_kv, D, 128) || !make_bshd_map(&mv, v, B, S_k, H_kv, D, 128) ||
       !make_bshd_map(&mq, q, B, S_q, H_q, D, 64) || !make_bshd_map(&mdo, dO, B, S_q, H_q, D, 64) ||
-      !make_dqacc_map(&mdq, p.dq_acc, B, S_q, H_q, D))
+      !make_dqacc_map(&mdq, p.dq_acc, B, S_q, H_q, D, pairs ? D / 2 : D))
+    return ATTN_ERR_CUDA;
+  if (pairs && (!make_bshd_map(&mq32, q, B, S_q, H_q, D, 32) || !make_bshd_map(&mdo32, dO, B, S_q, H_q, D, 32)))
     return ATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
@@ -539,8 +560,14 @@ attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const voi
     return ATTN_ERR_CUDA;
   {
     const unsigned grid = static_cast<unsigned>(p.n_kv_tiles) * B * H_kv;
+    const unsigned grid_pairs = 2u * static_cast<unsigned>((p.n_kv_tiles + 1) / 2) * B * H_kv;
     cudaError_t err;
-    if (D == 128)
+    if (pairs)
+      err = det ? (causal ? launch_bwd_pair<true, true>(mk, mv, mq32, mdo32, mq, mdo, mdq, p, grid_pairs, s)
+                          : launch_bwd_pair<false, true>(mk, mv, mq32, mdo32, mq, mdo, mdq, p, grid_pairs, s))
+                : (causal ? launch_bwd_pair<true, false>(mk, mv, mq32, mdo32, mq, mdo, mdq, p, grid_pairs, s)
+                          : launch_bwd_pair<false, false>(mk, mv, mq32, mdo32, mq, mdo, mdq, p, grid_pairs, s));
+    else if (D == 128)
       err = det ? (causal ? launch_bwd<128, true, true>(mk, mv, mq, mdo, mdq, p, grid, s)
                           : launch_bwd<128, false, true>(mk, mv, mq, mdo, mdq, p, grid, s))
                 : (causal ? launch_bwd<128, true, false>(mk, mv, mq, mdo, mdq, p, grid, s)

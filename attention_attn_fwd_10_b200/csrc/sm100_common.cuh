@@ -124,6 +124,25 @@ __device__ __forceinline__ bool sem_wait_eq(const int* sem, int want, const Wait
   }
 }
 
+// Waits until the global int at `sem` is at least `want` (acquire at GPU scope),
+// with the same bound and abort protocol as mbar_wait.
+__device__ __forceinline__ bool sem_wait_ge(const int* sem, int want, const WaitCtl& ctl) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(sem) : "memory");
+    if (v >= want) return true;
+    if ((it & 15u) == 0) {
+      if (*ctl.abort_flag) return false;
+      if (globaltimer_ns() - t0 > ctl.limit_ns) {
+        *ctl.abort_flag = 1;
+        atomicExch(ctl.status, kDevWaitTimeout);
+        return false;
+      }
+    }
+  }
+}
+
 // Adds 1 to the global int at `sem` with release semantics at GPU scope.
 __device__ __forceinline__ void sem_release_add(int* sem) {
   asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(sem) : "memory");
@@ -382,6 +401,156 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");
+}
+
+// ----------------------------------------------------------------------------
+// CTA pairs: clusters of two CTAs whose tensor cores execute one MMA together
+// (cta_group::2).  The even CTA (rank 0) issues every MMA of the pair; an MMA
+// of M rows takes rows [0, M/2) of A from rank 0 and [M/2, M) from rank 1, and
+// the first / second half of B's N columns from rank 0 / rank 1, each at the
+// same shared-memory (or tensor-memory) address in its own CTA, and leaves rank
+// r's M/2 output rows (all N columns) in rank r's tensor memory.
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// The shared::cluster address of the same shared-memory location in cluster CTA `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+// Every thread of both CTAs (kernel start only: the pair is launched together).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Arrive on an mbarrier of either CTA of the cluster (shared::cluster address).
+// Default semantics (release at CTA scope), as the pair's hand-offs use: the data
+// they order is tensor memory (tcgen05 fences around the arrival) or shared
+// memory written by TMA and read by the tensor cores.
+__device__ __forceinline__ void mbar_arrive_cl(uint32_t bar_cl) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cl) : "memory");
+}
+// One such arrival for the whole warp, after every lane has reached this point.
+__device__ __forceinline__ void mbar_arrive_cl_warp(uint32_t bar_cl) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive_cl(bar_cl);
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cl(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait with acquire at cluster scope: for barriers that the other CTA of
+// the pair arrives on (or commits to).
+__device__ __forceinline__ bool mbar_wait_cl(uint32_t bar, uint32_t parity, const WaitCtl& ctl) {
+  if (mbar_try_wait_cl(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait_cl(bar, parity)) return true;
+    if ((it & 15u) == 0) {
+      if (*ctl.abort_flag) return false;
+      if (globaltimer_ns() - t0 > ctl.limit_ns) {
+        *ctl.abort_flag = 1;
+        atomicExch(ctl.status, kDevWaitTimeout);
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ bool mbar_wait_cl_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait_cl(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from this
+// CTA's shared memory into the shared memory of a cluster CTA (`dst_cl`); the
+// transaction bytes complete on that CTA's mbarrier `bar_cl`.  Joins the issuing
+// thread's current bulk group.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t dst_cl, uint32_t src, uint32_t bytes, uint32_t bar_cl) {
+  asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   dst_cl),
+               "r"(src), "r"(bytes), "r"(bar_cl)
+               : "memory");
+}
+
+// 16-byte store into the shared memory of either CTA of the cluster.
+__device__ __forceinline__ void st_shared_cl_v4(uint32_t addr_cl, uint4 v) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr_cl), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_shared_cl_u32(uint32_t addr_cl, uint32_t v) {
+  asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(addr_cl), "r"(v) : "memory");
+}
+
+// Make this thread's generic-proxy writes to the shared memory of the cluster's
+// CTAs visible to the async proxy (tensor-core operand reads).
+__device__ __forceinline__ void fence_proxy_async_smem_cl() {
+  asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
+
+// Tensor memory of a pair: one warp (same warp index) in each CTA executes these.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Pair MMAs (issued by rank 0), descriptors as (low, high) halves.
+__device__ __forceinline__ void umma2_ss_h(uint32_t d_tmem, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo,
+                                           uint32_t b_hi, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 a, b;\n\t"
+      "mov.b64 a, {%1, %2};\n\tmov.b64 b, {%3, %4};\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], a, b, %5, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma2_ts_h(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 b;\n\t"
+      "mov.b64 b, {%2, %3};\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], b, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive (once) on the mbarrier at shared::cluster address `bar_cl` (either CTA
+// of the pair) when every pair MMA issued so far by this thread completes.
+__device__ __forceinline__ void umma2_commit(uint32_t bar_cl) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cl)
+               : "memory");
+}
+
+// High half of a 64-byte-swizzle descriptor (layout code 4): for MN-major
+// operands whose rows are 32 bf16 (64 B); SBO = next group of 8 contraction rows.
+__host__ __device__ constexpr uint32_t sdesc_sw64_hi(uint32_t sbo_bytes) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (4u << 29);
 }
 
 // ----------------------------------------------------------------------------

@@ -548,21 +548,23 @@ def run_configs(attn, dev, flush, peaks):
         "algorithmic_bytes": bytes_alg, "reps": reps, "sm_mhz": c["sm_mhz"], "clock_samples": c.get("samples")}
     del q, k, v, o, lse, ws, x
 
-    # the backward workload in its deterministic mode (fixed dQ order)
+    # the backward workload in its deterministic mode (fixed dQ order), and both modes
+    # with the main pass on CTA pairs (cta_group::2)
     wb = workloads.BWD_CAUSAL
     x = workloads.make_inputs(wb)
     q, k, v, do = (x[n].to(dev) for n in ("q", "k", "v", "do"))
     o, lse = attn.fwd(q, k, v, causal=True, scale=wb.scale)
     ws = torch.empty(attn.bwd_workspace_size(wb.B, wb.H_q, wb.S_q, wb.D), dtype=torch.uint8, device=dev)
     g = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
-    for det in (False, True):
+    for det, mode in ((False, 1), (True, 1), (False, 2), (True, 2)):
         with ClockSampler(dev.index) as clk:
             ms, reps = timed_calls(lambda: attn.bwd(q, k, v, o, lse, do, causal=True, scale=wb.scale, dq=g[0],
-                                                    dk=g[1], dv=g[2], workspace=ws, deterministic=det),
+                                                    dk=g[1], dv=g[2], workspace=ws, deterministic=det,
+                                                    cta_mode=mode),
                                    flush, stream)
         c = clk.summary()
         tf = wb.bwd_flops() / (ms * 1e-3) / 1e12
-        out[wb.name + ("_deterministic" if det else "")] = {
+        out[wb.name + ("_deterministic" if det else "") + ("_cta_pairs" if mode == 2 else "")] = {
             "ms": round(ms, 4), "tflops": round(tf, 1), "frac_of_measured": round(tf / peak, 4), "reps": reps,
             "sm_mhz": c["sm_mhz"], "clock_samples": c.get("samples")}
     del q, k, v, do, o, lse, ws, g, x
@@ -605,7 +607,7 @@ def run_reference(args):
 
 
 def run_profile(args):
-    """Launch only one pass (--profile fwd|bwd) W + K times on the workload, no
+    """Launch only one pass (--profile fwd|bwd|bwd_pairs|decode) W + K times on the workload, no
     timing: the driver for ncu captures of a single kernel."""
     import torch
 
@@ -634,7 +636,8 @@ def run_profile(args):
         if args.profile == "fwd":
             attn.fwd(q, k, v, causal=wf.causal, scale=wf.scale, out=o, lse=lse)
         else:
-            attn.bwd(q, k, v, o, lse, do, causal=wb.causal, scale=wb.scale, workspace=ws)
+            attn.bwd(q, k, v, o, lse, do, causal=wb.causal, scale=wb.scale, workspace=ws,
+                     cta_mode=2 if args.profile == "bwd_pairs" else 0)
     torch.cuda.synchronize()
     st = attn.device_status()
     print(f"profile {args.profile}: {args.warmup + args.steps} launches, device status {st}")
@@ -725,7 +728,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle CPU time to sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration measurements")
-    ap.add_argument("--profile", choices=("fwd", "bwd", "decode"), default=None,
+    ap.add_argument("--profile", choices=("fwd", "bwd", "bwd_pairs", "decode"), default=None,
                     help="only launch one pass W+K times (driver for ncu captures); prints no JSON")
     ap.add_argument("--variants", action="store_true",
                     help="side measurements (bf16 / e4m3 Q-K forward, decode shapes, deterministic backward); "

@@ -59,7 +59,8 @@ typedef enum {
 
 /* Version of this ABI (bumped on any incompatible change; 2: attn_bwd_options_t gained
  * `deterministic`, the split-KV and 8-bit Q/K forwards were added; 3: the backward
- * workspace gained the deterministic mode's work-item counter, attn_fwd_qkv8). */
+ * workspace gained the deterministic mode's work-item counter, attn_fwd_qkv8; 4:
+ * attn_fwd_options_t gained `persistent`, attn_bwd_options_t gained `cta_mode`). */
 int attn_abi_version(void);
 
 /* Human-readable name of a status code (static storage). */
@@ -232,11 +233,22 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
  *       on the order in which the hardware dispatches the blocks.  dQ is then
  *       bitwise identical from run to run (the pages' atomic reductions, section
  *       7 item 3, leave the order open); dK, dV are deterministic in both modes.
+ *       With CTA pairs the order is over pairs of key tiles.
+ *   cta_mode : how the main pass maps key tiles to CTAs.  0 (default) and 1 =
+ *       one CTA per 128-key tile (every MMA on one SM); the faster of the two
+ *       on B200 at these tile shapes.  2 = CTA pairs (clusters of two CTAs on
+ *       adjacent key tiles whose tensor cores execute each MMA together,
+ *       cta_group::2: "AI Infra series ch. 6", section 7 item 3): half of each
+ *       B operand per CTA and half the dQ reduce-adds, at the cost of a dS^T
+ *       exchange between the two CTAs and a dQ^T product of M = 128 per pair.
+ *       D = 128 only; other D return ATTN_ERR_INVALID_ARG.  Results agree to
+ *       rounding; only the summation order of dQ differs.
  */
 typedef struct {
   void* main_pass_start;
   void* main_pass_stop;
   int deterministic;
+  int cta_mode;
 } attn_bwd_options_t;
 
 /* attn_bwd with explicit options (`opt` NULL = all fields 0). */

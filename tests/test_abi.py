@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(lib):
 def test_status_strings(lib):
     for code, name in _abi.STATUS_NAMES.items():
         assert _abi.status_string(code).startswith(name)
-    assert lib.attn_abi_version() == 3
+    assert lib.attn_abi_version() == 4
 
 
 def _fwd(lib, **kw):
@@ -153,4 +153,4 @@ def test_header_is_c99_and_links(lib, tmp_path):
     assert res.returncode == 0, res.stderr
     run = subprocess.run([str(exe)], capture_output=True, text=True)
     assert run.returncode == 0, (run.returncode, run.stdout, run.stderr)
-    assert "abi 3" in run.stdout
+    assert "abi 4" in run.stdout
