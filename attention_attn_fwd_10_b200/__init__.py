@@ -190,8 +190,10 @@ def bwd(q, k, v, o, lse, do, causal: bool = False, scale: float | None = None, d
     ``main_pass_events``: optional (start, stop) torch.cuda.Event pair recorded
     around the main-pass kernel (diagnostic timing).  ``deterministic``: add the
     dQ parts of each query block in key-tile order (bitwise reproducible dQ).
-    ``cta_mode``: 0 / 1 = one CTA per key tile (default), 2 = CTA pairs whose
-    tensor cores execute each MMA together (head dim 128)."""
+    ``cta_mode``: 0 = the faster kernel of each mode (CTA pairs for the
+    deterministic backward at head dim 128, else one CTA per key tile), 1 = one
+    CTA per key tile, 2 = CTA pairs whose tensor cores execute each MMA together
+    (head dim 128)."""
     on_host = not q.is_cuda
     if on_host:
         dev = torch.device("cuda", torch.cuda.current_device())

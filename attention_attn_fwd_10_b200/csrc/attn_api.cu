@@ -518,7 +518,10 @@ attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const voi
   const bool det = opt && opt->deterministic;
   const int cta_mode = opt ? opt->cta_mode : 0;
   if (cta_mode < 0 || cta_mode > 2 || (cta_mode == 2 && D != 128)) return ATTN_ERR_INVALID_ARG;
-  const bool pairs = cta_mode == 2;  // default: one CTA per tile (the faster kernel on B200)
+  // default: CTA pairs for the deterministic instance at D = 128 (its turn waits halve
+  // with the number of dQ adders), one CTA per tile otherwise -- the faster kernel of
+  // each mode on B200
+  const bool pairs = cta_mode == 2 || (cta_mode == 0 && det && D == 128);
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);

@@ -556,7 +556,7 @@ def run_configs(attn, dev, flush, peaks):
     o, lse = attn.fwd(q, k, v, causal=True, scale=wb.scale)
     ws = torch.empty(attn.bwd_workspace_size(wb.B, wb.H_q, wb.S_q, wb.D), dtype=torch.uint8, device=dev)
     g = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
-    for det, mode in ((False, 1), (True, 1), (False, 2), (True, 2)):
+    for det, mode in ((False, 1), (True, 1), (False, 2), (True, 2)):  # explicit kernels (0 picks per mode)
         with ClockSampler(dev.index) as clk:
             ms, reps = timed_calls(lambda: attn.bwd(q, k, v, o, lse, do, causal=True, scale=wb.scale, dq=g[0],
                                                     dk=g[1], dv=g[2], workspace=ws, deterministic=det,
@@ -564,8 +564,10 @@ def run_configs(attn, dev, flush, peaks):
                                    flush, stream)
         c = clk.summary()
         tf = wb.bwd_flops() / (ms * 1e-3) / 1e12
-        out[wb.name + ("_deterministic" if det else "") + ("_cta_pairs" if mode == 2 else "")] = {
+        default_kernel = mode == (2 if det else 1)  # what cta_mode 0 picks for this mode
+        out[wb.name + ("_deterministic" if det else "") + ("_cta_pairs" if mode == 2 else "_one_cta_per_tile")] = {
             "ms": round(ms, 4), "tflops": round(tf, 1), "frac_of_measured": round(tf / peak, 4), "reps": reps,
+            "default": default_kernel,
             "sm_mhz": c["sm_mhz"], "clock_samples": c.get("samples")}
     del q, k, v, do, o, lse, ws, g, x
     torch.cuda.synchronize()

@@ -234,9 +234,10 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
  *       bitwise identical from run to run (the pages' atomic reductions, section
  *       7 item 3, leave the order open); dK, dV are deterministic in both modes.
  *       With CTA pairs the order is over pairs of key tiles.
- *   cta_mode : how the main pass maps key tiles to CTAs.  0 (default) and 1 =
- *       one CTA per 128-key tile (every MMA on one SM); the faster of the two
- *       on B200 at these tile shapes.  2 = CTA pairs (clusters of two CTAs on
+ *   cta_mode : how the main pass maps key tiles to CTAs.  0 (default) = the
+ *       faster kernel of each mode on B200: CTA pairs for the deterministic
+ *       instance at D = 128, one CTA per tile otherwise.  1 = one CTA per
+ *       128-key tile (every MMA on one SM).  2 = CTA pairs (clusters of two CTAs on
  *       adjacent key tiles whose tensor cores execute each MMA together,
  *       cta_group::2: "AI Infra series ch. 6", section 7 item 3): half of each
  *       B operand per CTA and half the dQ reduce-adds, at the cost of a dS^T
