@@ -565,8 +565,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) {
-    mbar_arrive_cl(pbar(L::B_EXIT));
-    if (!mbar_wait_drain(bar(L::B_EXIT), 0, 2000000000ull)) atomicExch(p.status, kDevWaitTimeout);
+    mbar_arrive_cl_release(pbar(L::B_EXIT));
+    if (!mbar_wait_cl_drain(bar(L::B_EXIT), 0, 2000000000ull)) atomicExch(p.status, kDevWaitTimeout);
   }
   __syncthreads();
   if (warp == L::WARP_MMA) {

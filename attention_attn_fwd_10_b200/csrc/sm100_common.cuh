@@ -436,7 +436,13 @@ __device__ __forceinline__ void cluster_sync_all() {
 __device__ __forceinline__ void mbar_arrive_cl(uint32_t bar_cl) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(bar_cl) : "memory");
 }
-// One such arrival for the whole warp, after every lane has reached this point.
+// Arrival that releases at cluster scope everything this thread has observed
+// (after a CTA barrier: the whole CTA's earlier accesses to the other CTA), for
+// the pair's exit handshake.  ~1.3k clk: not for per-block hand-offs.
+__device__ __forceinline__ void mbar_arrive_cl_release(uint32_t bar_cl) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cl) : "memory");
+}
+// One mbar_arrive_cl for the whole warp, after every lane has reached this point.
 __device__ __forceinline__ void mbar_arrive_cl_warp(uint32_t bar_cl) {
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive_cl(bar_cl);

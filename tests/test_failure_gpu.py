@@ -31,16 +31,20 @@ def test_timeouts_are_reported_and_the_context_stays_usable():
         st_fwd = attn.device_status()
         attn.bwd(q, k, v, o, lse, do, causal=True)
         st_bwd = attn.device_status()
+        attn.bwd(q, k, v, o, lse, do, causal=True, cta_mode=2)  # the CTA-pair kernel's abort paths
+        st_pairs = attn.device_status()
     finally:
         attn.set_wait_limit_ns(0)  # back to the default limit
-    assert st_fwd == TIMEOUT and st_bwd == TIMEOUT
+    assert st_fwd == TIMEOUT and st_bwd == TIMEOUT and st_pairs == TIMEOUT
     # the context is intact: a normal run is correct and reports no error
     o, lse = attn.fwd(q, k, v, causal=True)
     dq, dk, dv = attn.bwd(q, k, v, o, lse, do, causal=True)
+    pairs = attn.bwd(q, k, v, o, lse, do, causal=True, cta_mode=2)
     assert attn.device_status() == 0
     o_ref, lse_ref = ref.forward(x["q"], x["k"], x["v"], True, w.scale)
     parity.check_o(o, o_ref)
     parity.check_lse(lse, lse_ref)
     g_ref = ref.backward(x["q"], x["k"], x["v"], x["do"], True, w.scale)
-    for g, gr in zip((dq, dk, dv), g_ref):
+    for g, gp, gr in zip((dq, dk, dv), pairs, g_ref):
         parity.check_grad(g, gr)
+        parity.check_grad(gp, gr)
