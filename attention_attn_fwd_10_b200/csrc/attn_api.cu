@@ -364,16 +364,57 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
                  : launch_fwd_poly<64, false>(opt.poly_exp_every, mq, mk, mv, p, grid, s);
   if (err != cudaSuccess) return ATTN_ERR_CUDA;
   if (n_splits > 1) {
-    const long long warps = static_cast<long long>(B) * S_q * H_q;
-    const long long blocks = (warps + 7) / 8;
-    const unsigned g = static_cast<unsigned>(blocks < kNumSms * 16 ? blocks : kNumSms * 16);
-    if (D == 128)
-      attn_fwd_combine_kernel<128><<<g, 256, 0, s>>>(p);
-    else
-      attn_fwd_combine_kernel<64><<<g, 256, 0, s>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    const long long rows = static_cast<long long>(B) * S_q * H_q;
+    if (rows <= kNumSms * 8) {
+      // few rows (decode): one CTA per row, launched as a programmatic dependent so its
+      // launch overlaps the forward's tail; it waits on the device for the results
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = dim3(static_cast<unsigned>(rows));
+      cfg.blockDim = dim3(256);
+      cfg.dynamicSmemBytes = 0;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[0].val.programmaticStreamSerializationAllowed = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      const cudaError_t me = D == 128 ? cudaLaunchKernelEx(&cfg, attn_fwd_merge_rows_kernel<128>, p)
+                                      : cudaLaunchKernelEx(&cfg, attn_fwd_merge_rows_kernel<64>, p);
+      if (me != cudaSuccess) return ATTN_ERR_CUDA;
+    } else {
+      const long long blocks = (rows + 7) / 8;  // one warp per row
+      const unsigned g = static_cast<unsigned>(blocks < kNumSms * 16 ? blocks : kNumSms * 16);
+      if (D == 128)
+        attn_fwd_combine_kernel<128><<<g, 256, 0, s>>>(p);
+      else
+        attn_fwd_combine_kernel<64><<<g, 256, 0, s>>>(p);
+      if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    }
   }
   return ATTN_OK;
+}
+
+// Range count of the tensor-core split-KV forward: time ~ waves of CTAs x (key
+// blocks per range + ~2 blocks of per-CTA fixed cost).
+int tc_split_count(int B, int H_q, int H_kv, int S_q, int S_k) {
+  if (B < 1 || H_q < 1 || H_kv < 1 || H_q % H_kv != 0 || S_q < 1 || S_k < 1) return 1;
+  const int gp = fwd_head_pack(H_q, H_kv, S_q);
+  const long long ctas = static_cast<long long>((S_q + 256 / gp - 1) / (256 / gp)) * B * (H_q / gp);
+  const int n_kv = (S_k + 127) / 128;
+  if (ctas >= kNumSms) return 1;
+  int best = 1;
+  long long best_cost = -1;
+  for (int n = 1; n <= std::min(kMaxSplits, n_kv); ++n) {
+    const long long per = (n_kv + n - 1) / n;
+    const long long ranges = (n_kv + per - 1) / per;
+    const long long waves = (ctas * ranges + kNumSms - 1) / kNumSms;
+    const long long cost = waves * (per + 2);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = static_cast<int>(ranges);
+    }
+  }
+  return best;
 }
 
 }  // namespace
@@ -421,24 +462,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
 int attn_fwd_split_count(int B, int H_q, int H_kv, int S_q, int S_k, int causal) {
   (void)causal;
   if (B < 1 || H_q < 1 || H_kv < 1 || H_q % H_kv != 0 || S_q < 1 || S_k < 1) return 1;
-  const int gp = fwd_head_pack(H_q, H_kv, S_q);
-  const long long ctas = static_cast<long long>((S_q + 256 / gp - 1) / (256 / gp)) * B * (H_q / gp);
-  const int n_kv = (S_k + 127) / 128;
-  if (ctas >= kNumSms) return 1;
-  // time ~ waves of CTAs x (key blocks per range + ~2 blocks of per-CTA fixed cost)
-  int best = 1;
-  long long best_cost = -1;
-  for (int n = 1; n <= std::min(kMaxSplits, n_kv); ++n) {
-    const long long per = (n_kv + n - 1) / n;
-    const long long ranges = (n_kv + per - 1) / per;
-    const long long waves = (ctas * ranges + kNumSms - 1) / kNumSms;
-    const long long cost = waves * (per + 2);
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best = static_cast<int>(ranges);
-    }
-  }
-  return best;
+  return attn::tc_split_count(B, H_q, H_kv, S_q, S_k);
 }
 
 attn_status_t attn_fwd_qk8(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H_q,
@@ -457,7 +481,7 @@ attn_status_t attn_fwd_split_qk8(const void* q, const void* k, const void* v, vo
                                  void* workspace, int B, int H_q, int H_kv, int S_q, int S_k, int D, int causal,
                                  float scale, int n_splits, void* stream) {
   if (n_splits < 0 || n_splits > kMaxSplits) return ATTN_ERR_INVALID_ARG;
-  if (n_splits == 0) n_splits = attn_fwd_split_count(B, H_q, H_kv, S_q, S_k, causal);
+  if (n_splits == 0) n_splits = attn::tc_split_count(B, H_q, H_kv, S_q, S_k);
   return run_fwd(q, k, v, o, lse, workspace, B, H_q, H_kv, S_q, S_k, D, causal, scale, nullptr, n_splits, stream,
                  true);
 }

@@ -389,12 +389,21 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
       mbar_wait_drain(bar(L::B_DRAIN), 0, 1000000000ull);
     }
   } else if (warp < 8) {
-    // ===================== softmax / dS: thread = (key row, half of the 64 queries) =====================
-    const int r = threadIdx.x & 127;   // key row == TMEM lane
+    // ===================== softmax / dS =====================
+    // Warp w covers TMEM lanes (key rows) of quadrant w % 4 and query half hc = w / 4.
+    // Each thread holds 4 key rows x 8 queries (shape 16x256b): rows 32 (w % 4) + 16 h +
+    // lane/4 + 8 v (h, v in {0, 1}), queries 32 hc + 8 k + 2 (lane % 4) + {0, 1} (k < 4),
+    // so it needs only 8 of the per-query terms -lse2 and delta, which the warp reads
+    // with one 8-byte load per term and k (4 distinct addresses: one wavefront).
+    const int r = threadIdx.x & 127;   // epilogue: key row == TMEM lane
     const int hc = threadIdx.x >> 7;   // query half: columns [32 hc, 32 hc + 32)
     const int key = k0 + r;
     const bool valid_key = live && key < p.S_k;
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int t0 = lane & 3, t1 = lane >> 2;
+    int row_key[4];  // [2 h + v]: the key of this thread's row (h, v)
+#pragma unroll
+    for (int hv = 0; hv < 4; ++hv) row_key[hv] = k0 + (warp & 3) * 32 + 16 * (hv >> 1) + t1 + 8 * (hv & 1);
     const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
     bool ok = true;
     for (int i = 0; i < m; ++i) {
@@ -405,57 +414,88 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
       ok = mbar_wait(bar(L::B_S_FULL), i & 1, ctl);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sv[32], dp[32];
-      tmem_ld32(tmem + lane_addr + L::X_COL + 32 * hc, sv);
-      tmem_ld32(tmem + lane_addr + L::Y_COL + 32 * hc, dp);
-      tmem_ld_wait(sv);
-      tmem_ld_wait(dp);
-      const float4* nl4 = reinterpret_cast<const float4*>(sptr + L::LD_OFF + st * 512) + 8 * hc;
-      const float4* dl4 = reinterpret_cast<const float4*>(sptr + L::LD_OFF + st * 512 + 256) + 8 * hc;
-      // causal: key visible to query q0 + c iff c >= key - diag - q0; keys past S_k see nothing
-      const int c_first = (!valid_key ? L::BQ : (CAUSAL ? key - diag - q0 : 0)) - 32 * hc;
-      const bool masked = __any_sync(0xffffffffu, c_first > 0);
-      uint32_t pp[16], pd[16];
+      uint32_t sv[32], dp[32];  // [16 h + 4 k + 2 v + j]
+      tmem_ld16x256_x4(tmem + lane_addr + L::X_COL + 32 * hc, sv);
+      tmem_ld16x256_x4(tmem + lane_addr + (16u << 16) + L::X_COL + 32 * hc, sv + 16);
+      tmem_ld16x256_x4(tmem + lane_addr + L::Y_COL + 32 * hc, dp);
+      tmem_ld16x256_x4(tmem + lane_addr + (16u << 16) + L::Y_COL + 32 * hc, dp + 16);
+      const float2* nl2 = reinterpret_cast<const float2*>(sptr + L::LD_OFF + st * 512) + 16 * hc + t0;
+      const float2* dl2 = reinterpret_cast<const float2*>(sptr + L::LD_OFF + st * 512 + 256) + 16 * hc + t0;
+      float2 nlk[4], dlk[4];
 #pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
-        const float4 nlv = nl4[c4];
-        const float4 dlv = dl4[c4];
+      for (int k = 0; k < 4; ++k) {
+        nlk[k] = nl2[4 * k];
+        dlk[k] = dl2[4 * k];
+      }
+      tmem_ld_wait16(sv);
+      tmem_ld_wait16(sv + 16);
+      tmem_ld_wait16(dp);
+      tmem_ld_wait16(dp + 16);
+      // causal: key visible to query q0 + c iff c >= key - diag - q0; keys past S_k see nothing.
+      // c_first is relative to this thread's first query column 32 hc + 2 (lane % 4).
+      int c_first[4];
+      bool any_mask = false;
 #pragma unroll
-        for (int h2 = 0; h2 < 2; ++h2) {
-          const int cp = 2 * c4 + h2;
-          const float na = h2 ? nlv.z : nlv.x, nb = h2 ? nlv.w : nlv.y;
-          const float da = h2 ? dlv.z : dlv.x, dbv = h2 ? dlv.w : dlv.y;
-          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[2 * cp]), __uint_as_float(sv[2 * cp + 1])), c2,
-                                     f2_pack(na, nb));
-          float x0, x1;
-          f2_unpack(x2, x0, x1);
-          float p0 = exp2_mufu(x0), p1 = exp2_mufu(x1);
-          if (masked) {
-            if (2 * cp < c_first) p0 = 0.f;
-            if (2 * cp + 1 < c_first) p1 = 0.f;
+      for (int hv = 0; hv < 4; ++hv) {
+        const bool vk = live && row_key[hv] < p.S_k;
+        c_first[hv] = (!vk ? L::BQ : (CAUSAL ? row_key[hv] - diag - q0 : 0)) - 32 * hc - 2 * t0;
+        any_mask |= c_first[hv] > 0;
+      }
+      const bool masked = __any_sync(0xffffffffu, any_mask);
+      uint32_t pp[16], pd[16];  // [8 h + 2 k + v]: the bf16 pair (queries 2 j) of row (h, v)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            const int e = 16 * h + 4 * k + 2 * v;
+            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2,
+                                       f2_pack(nlk[k].x, nlk[k].y));
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            float p0 = exp2_mufu(x0), p1 = exp2_mufu(x1);
+            if (masked) {
+              const int cf = c_first[2 * h + v];
+              if (8 * k < cf) p0 = 0.f;
+              if (8 * k + 1 < cf) p1 = 0.f;
+            }
+            const uint64_t g2 = f2_sub(f2_pack(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
+                                       f2_pack(dlk[k].x, dlk[k].y));
+            float d0, d1;
+            f2_unpack(f2_mul(f2_pack(p0, p1), g2), d0, d1);
+            pp[8 * h + 2 * k + v] = pack_bf16x2(p0, p1);
+            pd[8 * h + 2 * k + v] = pack_bf16x2(d0, d1);
           }
-          const uint64_t g2 = f2_sub(f2_pack(__uint_as_float(dp[2 * cp]), __uint_as_float(dp[2 * cp + 1])),
-                                     f2_pack(da, dbv));
-          float d0, d1;
-          f2_unpack(f2_mul(f2_pack(p0, p1), g2), d0, d1);
-          pp[cp] = pack_bf16x2(p0, p1);
-          pd[cp] = pack_bf16x2(d0, d1);
         }
       }
-      // dS^T row r into the 128B-swizzled MN-major operand: 16-byte chunk c goes to chunk c ^ (r % 8)
-      uint8_t* dsrow = sptr + L::DS_OFF + db * L::DS_BYTES + r * 128;
+      // dS^T rows into the 128B-swizzled MN-major operand: the 4-byte pair of queries
+      // 32 hc + 8 k + 2 (lane % 4) sits in 16-byte chunk 4 hc + k of its row, and chunk c of
+      // row R at chunk c ^ (R % 8).  A warp's store covers 8 rows x 16 B: conflict-free.
+      uint8_t* dsb = sptr + L::DS_OFF + db * L::DS_BYTES;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        *reinterpret_cast<uint4*>(dsrow + (((4 * hc + c) ^ (r & 7)) << 4)) =
-            make_uint4(pd[4 * c], pd[4 * c + 1], pd[4 * c + 2], pd[4 * c + 3]);
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int v = 0; v < 2; ++v) {
+          const int R = (warp & 3) * 32 + 16 * h + t1 + 8 * v;
+          uint8_t* row = dsb + R * 128 + 4 * t0;
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            *reinterpret_cast<uint32_t*>(row + (((4 * hc + k) ^ (R & 7)) << 4)) = pd[8 * h + 2 * k + v];
+        }
+      }
       fence_proxy_async_smem();
       if (i >= 1) {  // dV_{i-1}, dK_{i-1} have read the previous P^T, dS^T
         ok = mbar_wait(bar(L::B_PD_FREE), (i - 1) & 1, ctl);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
       }
-      tmem_st16(tmem + lane_addr + L::P_COL + 16 * hc, pp);  // P^T (bf16 pairs)
-      tmem_st16(tmem + lane_addr + L::DS_COL + 16 * hc, pd);  // dS^T
+      // P^T, dS^T (bf16 pairs; column = query / 2) with shape 16x128b: packed column
+      // 16 hc + 4 k + lane % 4 of rows (h, v)
+      tmem_st16x128_x4(tmem + lane_addr + L::P_COL + 16 * hc, pp);
+      tmem_st16x128_x4(tmem + lane_addr + (16u << 16) + L::P_COL + 16 * hc, pp + 8);
+      tmem_st16x128_x4(tmem + lane_addr + L::DS_COL + 16 * hc, pd);
+      tmem_st16x128_x4(tmem + lane_addr + (16u << 16) + L::DS_COL + 16 * hc, pd + 8);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive_warp(bar(L::B_DS_READY));

@@ -226,6 +226,9 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
   const int lane = threadIdx.x & 31;
   const bool dual = p.dual != 0;
   const int tile_pos = L::BM >> p.gp_log2;  // query positions per tile
+  // split ranges: the merge of the ranges may start launching now (it waits on the
+  // device for this grid's results)
+  if (p.n_splits > 1) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int diag = p.S_k - p.S_q;           // bottom-right causal: key j visible to row i iff j <= i + diag
 
   // ---- work items.  Item n is the work of block n of a one-CTA-per-unit grid:
@@ -617,6 +620,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
         break;
       }
       int nb, kb0, lim, lim_tile;  // the key-block loop needs only these (the rest is decoded again after it)
+      bool idle;                   // every row of this warp is padding (past S_q)
       {
         const Unit w = decode(item);
         const int row0 = w.q0 + (dual ? 0 : t * tile_pos);  // first query position of the tile
@@ -625,6 +629,9 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
         kb0 = w.j0 * L::BN;
         lim = min(qi + (CAUSAL ? diag : p.S_k), p.S_k - 1);  // last visible key of this row
         lim_tile = CAUSAL ? row0 + diag : p.S_k - 1;         // last key every row of the tile sees
+        // rows are query-major (row r: position r / gp), so a decode tile's real rows are
+        // its first gp * S_q: the warps past them have nothing to compute
+        idle = row0 + ((((warp & 3) * 32)) >> p.gp_log2) >= p.S_q;
       }
       float m_used = -INFINITY;
       float l = 0.f;
@@ -637,6 +644,13 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
         if (j == nb - 1) mbar_arrive_warp(bar(L::B_ITEM_READ));
         ok = mbar_wait(bar(L::B_S_FULL + t), (sc + j) & 1, ctl);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        if (idle) {
+          // no row to compute: publish both halves of P(j) (their rows only ever reach
+          // padding rows of O) at the pace of S(j), like the tile's other warps
+          mbar_arrive_warp(bar(L::B_P_FULL + 2 * t));
+          mbar_arrive_warp(bar(L::B_P_FULL + 2 * t + 1));
+          continue;
+        }
         tc_fence_after();
         uint32_t sr[128];
         const uint32_t s_addr = tmem + lane_addr + L::s_col(t);
@@ -861,6 +875,89 @@ __global__ void __launch_bounds__(256) attn_fwd_combine_kernel(const FwdParams p
 #pragma unroll
     for (int i = 0; i < PER / 2; ++i) dst[i] = pack_bf16x2(acc[2 * i] * inv, acc[2 * i + 1] * inv);
     if (lane == 0) p.lse[lse_row] = sum > 0.f ? m + logf(sum) : -INFINITY;
+  }
+}
+
+// Merge of the ranges for few output rows (decode shapes): one CTA per row, its 8
+// warps taking the ranges in turn, so a row's partials load in parallel instead of
+// one range after another.  Same identity as attn_fwd_combine_kernel:
+//   lse = log sum_s exp(lse_s),   O = sum_s exp(lse_s - lse) O_s.
+template <int D>
+__global__ void __launch_bounds__(256) attn_fwd_merge_rows_kernel(const FwdParams p) {
+  constexpr int PER = D / 32;
+  __shared__ float red_m[8], red_w[8], lse_s[128];
+  __shared__ __align__(16) float red_o[8][D];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // launched as a programmatic dependent of the forward: wait for its results
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const long long rows = static_cast<long long>(p.B) * p.S_q * p.H_q;
+  const size_t lse_stride = static_cast<size_t>(p.B) * p.H_q * p.S_q;
+  for (long long w = blockIdx.x; w < rows; w += gridDim.x) {
+    const int h = static_cast<int>(w % p.H_q);
+    const long long bq = w / p.H_q;
+    const int q = static_cast<int>(bq % p.S_q);
+    const int b = static_cast<int>(bq / p.S_q);
+    const size_t lse_row = (static_cast<size_t>(b) * p.H_q + h) * p.S_q + q;
+    // the row's largest lse_s (thread t holds range t; at most 128 ranges)
+    const float ls = tid < p.n_splits ? p.lse_part[tid * lse_stride + lse_row] : -INFINITY;
+    if (tid < 128) lse_s[tid] = ls;
+    float m = ls;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) red_m[warp] = m;
+    __syncthreads();
+    m = red_m[0];
+#pragma unroll
+    for (int k = 1; k < 8; ++k) m = fmaxf(m, red_m[k]);
+    // warp k: ranges k, k + 8, ...
+    float acc[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) acc[i] = 0.f;
+    float wsum = 0.f;
+    if (m > -INFINITY) {
+      // ranges warp, warp + 8, ... (at most 16 per warp): every load issued before the sums
+#pragma unroll
+      for (int s = warp; s < 128; s += 8) {
+        if (s >= p.n_splits) break;
+        const float lss = lse_s[s];
+        const float wgt = lss == -INFINITY ? 0.f : exp2_mufu((lss - m) * 1.4426950408889634f);
+        wsum += wgt;
+        const float* src = p.o_part + (static_cast<size_t>(s) * rows + w) * D + lane * PER;
+        if constexpr (PER == 4) {
+          const float4 v = *reinterpret_cast<const float4*>(src);
+          acc[0] += wgt * v.x;
+          acc[1] += wgt * v.y;
+          acc[2] += wgt * v.z;
+          acc[3] += wgt * v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2*>(src);
+          acc[0] += wgt * v.x;
+          acc[1] += wgt * v.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i) red_o[warp][lane * PER + i] = acc[i];
+    if (lane == 0) red_w[warp] = wsum;
+    __syncthreads();
+    if (warp == 0) {
+      float sum = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) sum += red_w[k];
+      float o[PER];
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        o[i] = 0.f;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) o[i] += red_o[k][lane * PER + i];
+      }
+      const float inv = sum > 0.f ? 1.f / sum : 0.f;
+      uint32_t* dst = reinterpret_cast<uint32_t*>(p.o + w * D + lane * PER);
+#pragma unroll
+      for (int i = 0; i < PER / 2; ++i) dst[i] = pack_bf16x2(o[2 * i] * inv, o[2 * i + 1] * inv);
+      if (lane == 0) p.lse[lse_row] = sum > 0.f ? m + logf(sum) : -INFINITY;
+    }
+    __syncthreads();  // red_* are reused by the next row
   }
 }
 

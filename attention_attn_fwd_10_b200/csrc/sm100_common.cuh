@@ -615,6 +615,26 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
+// Shape 16x256b, 4 repeats: lanes base + lane/4 and base + lane/4 + 8 of the
+// 16-lane group at `taddr`, 32 columns.  r[4 k + 0..1] = row base + lane/4,
+// columns 8 k + 2 (lane % 4) + {0, 1}; r[4 k + 2..3] = the same columns of row
+// base + lane/4 + 8.
+__device__ __forceinline__ void tmem_ld16x256_x4(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : ATTN_R8(r, 0), ATTN_R8(r, 8)
+      : "r"(taddr));
+}
+
+// Shape 16x128b, 4 repeats: r[2 k + j] goes to row base + lane/4 + 8 j, column
+// 4 k + lane % 4 (16 columns).
+__device__ __forceinline__ void tmem_st16x128_x4(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x128b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), ATTN_I8(r, 0)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
