@@ -915,24 +915,37 @@ __global__ void __launch_bounds__(256) attn_fwd_merge_rows_kernel(const FwdParam
     for (int i = 0; i < PER; ++i) acc[i] = 0.f;
     float wsum = 0.f;
     if (m > -INFINITY) {
-      // ranges warp, warp + 8, ... (at most 16 per warp): every load issued before the sums
+      // ranges warp, warp + 8, ... (at most 16 per warp), in groups of 4 whose loads
+      // are all issued (predicated) before any of them is used
+#pragma unroll 1
+      for (int s0 = warp; s0 < p.n_splits; s0 += 32) {
+        float4 v4[4];
 #pragma unroll
-      for (int s = warp; s < 128; s += 8) {
-        if (s >= p.n_splits) break;
-        const float lss = lse_s[s];
-        const float wgt = lss == -INFINITY ? 0.f : exp2_mufu((lss - m) * 1.4426950408889634f);
-        wsum += wgt;
-        const float* src = p.o_part + (static_cast<size_t>(s) * rows + w) * D + lane * PER;
-        if constexpr (PER == 4) {
-          const float4 v = *reinterpret_cast<const float4*>(src);
-          acc[0] += wgt * v.x;
-          acc[1] += wgt * v.y;
-          acc[2] += wgt * v.z;
-          acc[3] += wgt * v.w;
-        } else {
-          const float2 v = *reinterpret_cast<const float2*>(src);
-          acc[0] += wgt * v.x;
-          acc[1] += wgt * v.y;
+        for (int u = 0; u < 4; ++u) {
+          const int s = s0 + 8 * u;
+          v4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (s < p.n_splits) {
+            const float* src = p.o_part + (static_cast<size_t>(s) * rows + w) * D + lane * PER;
+            if constexpr (PER == 4) {
+              v4[u] = *reinterpret_cast<const float4*>(src);
+            } else {
+              const float2 v = *reinterpret_cast<const float2*>(src);
+              v4[u] = make_float4(v.x, v.y, 0.f, 0.f);
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int s = s0 + 8 * u;
+          const float lss = s < p.n_splits ? lse_s[s] : -INFINITY;
+          const float wgt = lss == -INFINITY ? 0.f : exp2_mufu((lss - m) * 1.4426950408889634f);
+          wsum += wgt;
+          acc[0] += wgt * v4[u].x;
+          acc[1] += wgt * v4[u].y;
+          if constexpr (PER == 4) {
+            acc[2] += wgt * v4[u].z;
+            acc[3] += wgt * v4[u].w;
+          }
         }
       }
     }
