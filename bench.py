@@ -543,9 +543,14 @@ def run_configs(attn, dev, flush, peaks):
     c = clk.summary()
     bytes_alg = sum(t.numel() * t.element_size() for t in (q, k, v, o, lse))
     gbs = bytes_alg / (ms * 1e-3) / 1e9
+    # What one plain pass over the same K and V bytes takes here (two torch reductions,
+    # a library kernel used only as a yardstick): a 134 MB read does not reach the
+    # copy bandwidth of a GB-sized stream (start-up and drain are a large share of it).
+    ms_read, _ = timed_calls(lambda: (k.sum(dtype=torch.float32), v.sum(dtype=torch.float32)), flush, stream)
     out["decode_split_B1_Hq32_Hkv8_Sq1_Sk32768_D128"] = {
         "us": round(ms * 1e3, 2), "gbs": round(gbs, 1), "frac_of_hbm": round(gbs / hbm, 4), "n_splits": n,
-        "algorithmic_bytes": bytes_alg, "reps": reps, "sm_mhz": c["sm_mhz"], "clock_samples": c.get("samples")}
+        "algorithmic_bytes": bytes_alg, "reps": reps, "sm_mhz": c["sm_mhz"], "clock_samples": c.get("samples"),
+        "plain_read_of_kv_us": round(ms_read * 1e3, 2), "plain_read_over_decode": round(ms_read / ms, 4)}
     del q, k, v, o, lse, ws, x
 
     # the backward workload in its deterministic mode (fixed dQ order), and both modes
