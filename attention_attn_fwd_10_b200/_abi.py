@@ -42,6 +42,7 @@ EXPORTED = (
     "attn_device_status",
     "attn_set_wait_limit_ns",
     "attn_exp2_poly_eval",
+    "attn_read_probe",
 )
 
 
@@ -89,6 +90,7 @@ _SIGNATURES = {
     "attn_device_status": (_i, [_vp]),
     "attn_set_wait_limit_ns": (None, [ctypes.c_ulonglong]),
     "attn_exp2_poly_eval": (_i, [_vp, _vp, ctypes.c_longlong, _vp]),
+    "attn_read_probe": (_i, [_vp, ctypes.c_longlong, _vp, _vp]),
 }
 
 _lib = None

@@ -258,6 +258,24 @@ cudaError_t launch_bwd_pair(const CUtensorMap& mk, const CUtensorMap& mv, const 
 // kernel on another stream is never lost between a read and a clear).
 __global__ void take_status_kernel(int* status, int* taken) { *taken = atomicExch(status, 0); }
 
+// One plain pass over n16 16-byte words, four loads in flight per thread; the
+// XOR of everything read goes to a branch that keeps the loads alive (its
+// condition is practically never true).
+__global__ void read_probe_kernel(const uint4* __restrict__ x, long long n16, unsigned long long* sink) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  uint32_t acc = 0;
+  for (; i + 3 * stride < n16; i += 4 * stride) {
+    const uint4 a = __ldg(x + i), b = __ldg(x + i + stride), c = __ldg(x + i + 2 * stride), d = __ldg(x + i + 3 * stride);
+    acc ^= (a.x ^ a.y ^ a.z ^ a.w) ^ (b.x ^ b.y ^ b.z ^ b.w) ^ (c.x ^ c.y ^ c.z ^ c.w) ^ (d.x ^ d.y ^ d.z ^ d.w);
+  }
+  for (; i < n16; i += stride) {
+    const uint4 a = __ldg(x + i);
+    acc ^= a.x ^ a.y ^ a.z ^ a.w;
+  }
+  if (acc == 0x9E3779B9u) atomicAdd(sink, 1ull);
+}
+
 // Evaluates the kernels' packed-pair cubic on x[2i], x[2i+1] (the last element of
 // an odd-length array is paired with itself).
 __global__ void exp2_poly_eval_kernel(const float* x, float* y, long long n) {
@@ -663,5 +681,29 @@ attn_status_t attn_exp2_poly_eval(const float* x, float* y, long long n, void* s
   exp2_poly_eval_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
+
+attn_status_t attn_read_probe(const void* x, long long bytes, unsigned long long* sink, void* stream) {
+  if (bytes < 0 || (bytes & 15) || (bytes > 0 && (!x || !sink)) || (reinterpret_cast<uintptr_t>(x) & 15) ||
+      (reinterpret_cast<uintptr_t>(sink) & 7))
+    return ATTN_ERR_INVALID_ARG;
+  if (bytes == 0) return ATTN_OK;
+  read_probe_kernel<<<kNumSms * 4, 512, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<const uint4*>(x),
+                                                                                  bytes / 16, sink);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+#ifdef ATTN_TIMELINE
+// Timeline build only (include/attn_timeline.h).
+attn_status_t attn_timeline_read(long long* events, long long* t0, int next_cta) {
+  if (!events || !t0) return ATTN_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(events, attn::g_timeline, sizeof(attn::g_timeline)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(t0, attn::g_timeline_t0, sizeof(long long)) != cudaSuccess) return ATTN_ERR_CUDA;
+  static long long zeros[attn::kTimelineEvents][attn::kTimelineBlocks];
+  if (cudaMemcpyToSymbol(attn::g_timeline, zeros, sizeof(zeros)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaMemcpyToSymbol(attn::g_timeline_cta, &next_cta, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+#endif
 
 }  // extern "C"

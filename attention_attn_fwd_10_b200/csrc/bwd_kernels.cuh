@@ -214,6 +214,12 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
   const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // timeline build only (events per query block: 0 S^T/dP^T issued, 1 S^T ready at
+  // the softmax, 2 dS^T published, 3 dS^T seen by the issuer, 4 dV/dK issued, 5 dQ^T
+  // issued, 6 dQ^T ready at the staging warps, 7 dQ tile staged, 8 reduce-add issued,
+  // 9 its source read)
+  [[maybe_unused]] const bool tl = ATTN_TL_ON();
+  ATTN_TL_T0(tl);
 
   // Work item: the block index, or in the deterministic instance a ticket taken
   // from a global counter when the CTA starts.  Items are ordered so that the
@@ -345,6 +351,7 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
         if (ok) {
           tc_fence_after();
           issue_s_dp(0);
+          ATTN_TL(tl, 0, 0);
         }
       }
       for (int i = 0; ok && i < m; ++i) {
@@ -353,6 +360,7 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
         const int db = i & 1;             // dS^T buffer of block i
         const uint32_t sb = sbase + L::STAGE_OFF + st * L::STAGE_BYTES;
         if (!mbar_wait(bar(L::B_DS_READY), i & 1, ctl)) break;
+        ATTN_TL(tl, 3, i);
         tc_fence_after();
         // the next block's S^T, dP^T first: the softmax warpgroup starts on them while
         // the tensor pipe runs dV_i, dK_i, dQ^T_i
@@ -360,6 +368,7 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
           if (!mbar_wait(bar(L::B_QDO_FULL + st1), ((i + 1) / L::NST) & 1, ctl)) break;
           tc_fence_after();
           issue_s_dp(st1);
+          ATTN_TL(tl, 0, i + 1);
         }
         // dV += P^T dO_i ; dK += dS^T Q_i   (16 queries per MMA: 8 TMEM columns, 2048 B of the stage)
 #pragma unroll
@@ -372,6 +381,7 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
                     HI, IDESC_G, (i > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bar(L::B_PD_FREE));
         umma_commit(bar(L::B_QDO_EMPTY + st));
+        ATTN_TL(tl, 4, i);
         if (i >= 1) {
           if (!mbar_wait(bar(L::B_DQ_FREE), (i - 1) & 1, ctl)) break;
           tc_fence_after();
@@ -383,6 +393,7 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
           umma_ss_h(tmem + L::DQ_COL, kT_lo + kk * 128, HI, sdesc_lo(ds, L::DS_BYTES) + kk * 128, HI, IDESC_Q,
                     kk > 0 ? 1u : 0u);
         umma_commit(bar(L::B_DQ_FULL));
+        ATTN_TL(tl, 5, i);
       }
       if (ok) umma_commit(bar(L::B_D_FINAL));
       umma_commit(bar(L::B_DRAIN));
@@ -412,6 +423,7 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
       const int q0 = (qb0 + i % per_head) * L::BQ;
       // S_FULL(i) is committed after dQ^T_{i-2}, so dS^T buffer `db` is free as well.
       ok = mbar_wait(bar(L::B_S_FULL), i & 1, ctl);
+      if (threadIdx.x == 0) ATTN_TL(tl, 1, i);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       uint32_t sv[32], dp[32];  // [16 h + 4 k + 2 v + j]
@@ -499,6 +511,7 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive_warp(bar(L::B_DS_READY));
+      if (threadIdx.x == 0) ATTN_TL(tl, 2, i);
     }
     // ---- epilogue: dV, dK (scaled) -> bf16; this thread writes head dims [D/2 hc, D/2 (hc + 1))
     if (ok && m > 0) {
@@ -547,6 +560,7 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     for (int i = 0; i < m; ++i) {
       bool ok = mbar_wait(bar(L::B_DQ_FULL), i & 1, ctl);
+      if (wl == 0) ATTN_TL(tl, 6, i);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       uint32_t v[64];
@@ -567,6 +581,7 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
         if (d >= 0) stage[c * D + d] = __uint_as_float(v[c]);
       fence_proxy_async_smem();
       mbar_arrive_warp(bar(L::B_STAGED + buf));
+      if (wl == 0) ATTN_TL(tl, 7, i);
     }
   } else if (warp == L::WARP_RED) {
     // ===================== dQ reduce issue: one TMA reduce-add per staged tile =====================
@@ -592,6 +607,7 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
         }
         tma_reduce_add_4d(&tm_dqacc, sbase + L::DQ_STAGE_OFF + buf * L::DQ_STAGE_BYTES, 0, h, qb * L::BQ, b);
         bulk_commit_group();
+        ATTN_TL(tl, 8, i);
         if (DET) {
           bulk_wait_all();  // the additions are performed
           fence_proxy_async_global();
@@ -600,6 +616,7 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
         } else {
           bulk_wait_read_all();  // the tile has been read
         }
+        ATTN_TL(tl, 9, i);
         mbar_arrive(bar(L::B_STAGE_FREE + buf));
       }
       bulk_wait_all();

@@ -225,6 +225,12 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const bool dual = p.dual != 0;
+  // timeline build only (events: 0/1 S_t ready at the softmax, 2/3 row max done,
+  // 4/5 P_t published, 6/7 PV_t issued, 8/9 next S_t issued, 10 V block ready at the
+  // issuer, 15 V block load issued, per block of the tile; 11/12 O_t final at the
+  // softmax, 13/14 epilogue done, per unit)
+  [[maybe_unused]] const bool tl = ATTN_TL_ON();
+  ATTN_TL_T0(tl);
   const int tile_pos = L::BM >> p.gp_log2;  // query positions per tile
   // split ranges: the merge of the ranges may start launching now (it waits on the
   // device for this grid's results)
@@ -382,6 +388,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
             for (int x = 0; x < L::V_NBOX; ++x)
               tma_load_4d(sbase + L::v_off(s) + x * L::BOX_BYTES, &tm_v, bar(L::B_V_FULL + s),
                           x * 64, w.hkv, (w.j0 + j) * L::BN, w.b);
+            ATTN_TL(tl, 15, vn);
             ++vn;
           }
         }
@@ -490,8 +497,9 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
             for (int t = 0; t < 2; ++t) {
               if (!ok || j >= w.nblk(t)) continue;
               const int vs = vc % L::VST_DUAL;
-              ok = mbar_wait(bar(L::B_V_FULL + vs), (vc / L::VST_DUAL) & 1, ctl) &&
-                   mbar_wait(bar(L::B_P_FULL + 2 * t), ((t == 0 ? pc0 : pc1) + j) & 1, ctl);
+              ok = mbar_wait(bar(L::B_V_FULL + vs), (vc / L::VST_DUAL) & 1, ctl);
+              ATTN_TL(tl, 10, vc);
+              ok = ok && mbar_wait(bar(L::B_P_FULL + 2 * t), ((t == 0 ? pc0 : pc1) + j) & 1, ctl);
               if (!ok) break;
               tc_fence_after();
               issue_pv_half(t, vs, j > 0, 0);
@@ -499,6 +507,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
               if (!ok) break;
               tc_fence_after();
               issue_pv_half(t, vs, j > 0, 1);
+              ATTN_TL(tl, 6 + t, (t == 0 ? pc0 : pc1) + j);
               if (j == w.nblk(t) - 1) umma_commit(bar(L::B_O_FINAL + t));
               umma_commit(bar(L::B_V_EMPTY + vs));
               ++vc;
@@ -538,6 +547,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
             const int vs = vc % L::VST;
             const int ks1 = kc % L::KST;
             if (!(ok = mbar_wait(bar(L::B_V_FULL + vs), (vc / L::VST) & 1, ctl))) break;
+            ATTN_TL(tl, 10, vc);
             bool k_next_ready = false;
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
@@ -550,6 +560,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
               if (!ok) break;
               tc_fence_after();
               issue_pv_half(t, vs, j > 0, 1);
+              ATTN_TL(tl, 6 + t, (t == 0 ? pc0 : pc1) + j);
               if (j == w.nblk(t) - 1) umma_commit(bar(L::B_O_FINAL + t));
               if (j + 1 < w.nblk(t)) {
                 if (!k_next_ready) {
@@ -558,6 +569,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
                   k_next_ready = true;
                 }
                 issue_s(t, ks1);
+                ATTN_TL(tl, 8 + t, (t == 0 ? pc0 : pc1) + j + 1);
                 if (j + 2 == w.nblk(t)) umma_commit(bar(L::B_Q_EMPTY + t));  // the unit's last S_t
               }
             }
@@ -643,6 +655,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
       for (int j = 0; j < nb; ++j) {
         if (j == nb - 1) mbar_arrive_warp(bar(L::B_ITEM_READ));
         ok = mbar_wait(bar(L::B_S_FULL + t), (sc + j) & 1, ctl);
+        if (row == 0) ATTN_TL(tl, 0 + t, sc + j);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         if (idle) {
           // no row to compute: publish both halves of P(j) (their rows only ever reach
@@ -679,6 +692,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
           if (j > 0) ++rescales;
         }
         const float m_eff = (m_used == -INFINITY) ? 0.f : m_used;
+        if (row == 0) ATTN_TL(tl, 2 + t, sc + j);
         if (j > 0 && __any_sync(0xffffffffu, resc)) {
           // PV_t(j-1) completed before S_t(j) was issued, so O_t is final up to block
           // j-1; it is rescaled before any part of P_t(j) is published.
@@ -709,6 +723,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
           tc_fence_before();
           mbar_arrive_warp(bar(L::B_P_FULL + 2 * t + hf));
         }
+        if (row == 0) ATTN_TL(tl, 4 + t, sc + j);
       }
       sc += nb;
       if (p.rescale_count != nullptr && rescales) atomicAdd(p.rescale_count, (unsigned long long)rescales);
@@ -719,6 +734,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
       // ---- epilogue: O / l -> bf16 (or the split's fp32 O_s), lse
       if (ok && nb > 0) {
         ok = mbar_wait(bar(L::B_O_FINAL + t), oc & 1, ctl);
+        if (row == 0) ATTN_TL(tl, 11 + t, u);
         ok = __all_sync(0xffffffffu, ok);
         ++oc;
       }
@@ -794,6 +810,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
             else
               p.lse[(static_cast<size_t>(w.b) * p.H_q + h) * p.S_q + qi] = lse_v;
           }
+          if (row == 0) ATTN_TL(tl, 13 + t, u);
         }
       }
     }

@@ -27,6 +27,35 @@ enum DeviceError : int {
 };
 
 // ----------------------------------------------------------------------------
+// Optional timeline, compiled in only with -DATTN_TIMELINE (a separate library,
+// libattn_timeline.so; the default build has none of it): one chosen CTA records
+// clock64() at fixed points of its pipeline, event ev of its block i, so a host
+// tool can print the block cycle.  Events never change what a kernel computes.
+#ifdef ATTN_TIMELINE
+constexpr int kTimelineEvents = 16, kTimelineBlocks = 256;
+__device__ long long g_timeline[kTimelineEvents][kTimelineBlocks];
+__device__ long long g_timeline_t0;
+__device__ int g_timeline_cta = -1;
+#define ATTN_TL_ON() (static_cast<int>(blockIdx.x) == ::attn::g_timeline_cta)
+#define ATTN_TL(on, ev, i)                                                        \
+  do {                                                                            \
+    if ((on) && (i) >= 0 && (i) < ::attn::kTimelineBlocks) ::attn::g_timeline[(ev)][(i)] = clock64(); \
+  } while (0)
+#define ATTN_TL_T0(on)                                            \
+  do {                                                            \
+    if ((on) && threadIdx.x == 0) ::attn::g_timeline_t0 = clock64(); \
+  } while (0)
+#else
+#define ATTN_TL_ON() false
+#define ATTN_TL(on, ev, i) \
+  do {                     \
+  } while (0)
+#define ATTN_TL_T0(on) \
+  do {                 \
+  } while (0)
+#endif
+
+// ----------------------------------------------------------------------------
 // Generic helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

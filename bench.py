@@ -543,10 +543,21 @@ def run_configs(attn, dev, flush, peaks):
     c = clk.summary()
     bytes_alg = sum(t.numel() * t.element_size() for t in (q, k, v, o, lse))
     gbs = bytes_alg / (ms * 1e-3) / 1e9
-    # What one plain pass over the same K and V bytes takes here (two torch reductions,
-    # a library kernel used only as a yardstick): a 134 MB read does not reach the
-    # copy bandwidth of a GB-sized stream (start-up and drain are a large share of it).
-    ms_read, _ = timed_calls(lambda: (k.sum(dtype=torch.float32), v.sum(dtype=torch.float32)), flush, stream)
+    # What one plain pass over as many bytes as K and V takes here (the library's
+    # read probe): a 134 MB read does not reach the copy bandwidth of a GB-sized
+    # stream, start-up and drain being a large share of it.
+    kv_bytes = (k.numel() * k.element_size() + v.numel() * v.element_size() + 15) // 16 * 16
+    rbuf = torch.ones(kv_bytes // 4, dtype=torch.int32, device=dev)
+    sink = torch.zeros(1, dtype=torch.int64, device=dev)
+    lib = attn.load()
+
+    def read_once():
+        code = lib.attn_read_probe(rbuf.data_ptr(), kv_bytes, sink.data_ptr(), stream.cuda_stream)
+        if code != 0:
+            raise RuntimeError(f"attn_read_probe failed: {code}")
+
+    ms_read, _ = timed_calls(read_once, flush, stream)
+    del rbuf, sink
     out["decode_split_B1_Hq32_Hkv8_Sq1_Sk32768_D128"] = {
         "us": round(ms * 1e3, 2), "gbs": round(gbs, 1), "frac_of_hbm": round(gbs / hbm, 4), "n_splits": n,
         "algorithmic_bytes": bytes_alg, "reps": reps, "sm_mhz": c["sm_mhz"], "clock_samples": c.get("samples"),

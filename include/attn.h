@@ -309,6 +309,16 @@ void attn_set_wait_limit_ns(unsigned long long ns);
  */
 attn_status_t attn_exp2_poly_eval(const float* x, float* y, long long n, void* stream);
 
+/*
+ * Diagnostic: reads `bytes` bytes at device pointer x once (16-byte loads, four
+ * in flight per thread, four CTAs of 512 threads per SM) and folds them into the
+ * device word *sink, so the caller can time a plain read of as many bytes as a
+ * bytes-bound call moves: the yardstick for the split-KV forward on decoding
+ * shapes.  x and sink 16- and 8-byte aligned, bytes >= 0 and a multiple of 16;
+ * otherwise ATTN_ERR_INVALID_ARG.
+ */
+attn_status_t attn_read_probe(const void* x, long long bytes, unsigned long long* sink, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

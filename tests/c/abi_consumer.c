@@ -13,7 +13,7 @@ int main(void) {
       (void*)attn_fwd_split,        (void*)attn_fwd_split_qk8,   (void*)attn_fwd_split_count,
       (void*)attn_fwd_split_workspace_size, (void*)attn_bwd_workspace_size, (void*)attn_bwd,
       (void*)attn_bwd_ex,           (void*)attn_bwd_noalloc,     (void*)attn_device_status,
-      (void*)attn_set_wait_limit_ns, (void*)attn_exp2_poly_eval};
+      (void*)attn_set_wait_limit_ns, (void*)attn_exp2_poly_eval, (void*)attn_read_probe};
   for (size_t i = 0; i < sizeof(entry_points) / sizeof(entry_points[0]); ++i)
     if (!entry_points[i]) return 1;
   attn_fwd_options_t opt;

@@ -89,6 +89,16 @@ def test_exp2_eval_rejects_bad_arguments(lib):
     assert lib.attn_exp2_poly_eval(None, None, 0, None) == 0
 
 
+def test_read_probe_rejects_bad_arguments(lib):
+    sink = ctypes.c_void_p(0x1000)
+    assert lib.attn_read_probe(ctypes.c_void_p(0x1000), -16, sink, None) == 1   # negative size
+    assert lib.attn_read_probe(ctypes.c_void_p(0x1000), 24, sink, None) == 1    # not a multiple of 16
+    assert lib.attn_read_probe(ctypes.c_void_p(0x1008), 32, sink, None) == 1    # x not 16-byte aligned
+    assert lib.attn_read_probe(ctypes.c_void_p(0x1000), 32, ctypes.c_void_p(0x1004), None) == 1  # sink
+    assert lib.attn_read_probe(None, 32, sink, None) == 1
+    assert lib.attn_read_probe(None, 0, None, None) == 0                        # nothing to read
+
+
 def test_fwd_split_count(lib):
     # enough CTAs already: no split
     assert lib.attn_fwd_split_count(2, 16, 16, 8192, 8192, 1) == 1
@@ -154,3 +164,14 @@ def test_header_is_c99_and_links(lib, tmp_path):
     run = subprocess.run([str(exe)], capture_output=True, text=True)
     assert run.returncode == 0, (run.returncode, run.stdout, run.stderr)
     assert "abi 4" in run.stdout
+
+
+def test_timeline_only_in_the_timeline_build(lib):
+    """include/attn_timeline.h declares the timeline read-out; the default library
+    carries no timeline, the -DATTN_TIMELINE build exports it."""
+    text = open(os.path.join(ROOT, "include", "attn_timeline.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    assert sorted(set(re.findall(r"\b(attn_[a-z0-9_]+)\s*\(", text))) == ["attn_timeline_read"]
+    assert not hasattr(lib, "attn_timeline_read")
+    tl = ctypes.CDLL(build.build(timeline=True))
+    assert hasattr(tl, "attn_timeline_read")
