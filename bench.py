@@ -681,7 +681,7 @@ def run_profile(args):
     ws = torch.empty(attn.bwd_workspace_size(wb.B, wb.H_q, wb.S_q, wb.D), dtype=torch.uint8, device="cuda")
     for _ in range(args.warmup + args.steps):
         if args.profile == "fwd":
-            attn.fwd(q, k, v, causal=wf.causal, scale=wf.scale, out=o, lse=lse)
+            attn.fwd(q, k, v, causal=wf.causal, scale=wf.scale, out=o, lse=lse, poly_exp_every=args.poly_exp_every)
         else:
             attn.bwd(q, k, v, o, lse, do, causal=wb.causal, scale=wb.scale, workspace=ws,
                      cta_mode=2 if args.profile == "bwd_pairs" else 0)
@@ -777,6 +777,8 @@ def main():
     ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration measurements")
     ap.add_argument("--profile", choices=("fwd", "bwd", "bwd_pairs", "decode"), default=None,
                     help="only launch one pass W+K times (driver for ncu captures); prints no JSON")
+    ap.add_argument("--poly-exp-every", type=int, default=8, choices=(0, 4, 8),
+                    help="--profile fwd: one column pair in N on the FMA-pipe cubic (0: MUFU only)")
     ap.add_argument("--variants", action="store_true",
                     help="side measurements (bf16 / e4m3 Q-K forward, decode shapes, deterministic backward); "
                          "prints lines, not the JSON contract")
