@@ -217,7 +217,8 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
   // timeline build only (events per query block: 0 S^T/dP^T issued, 1 S^T ready at
   // the softmax, 2 dS^T published, 3 dS^T seen by the issuer, 4 dV/dK issued, 5 dQ^T
   // issued, 6 dQ^T ready at the staging warps, 7 dQ tile staged, 8 reduce-add issued,
-  // 9 its source read)
+  // 9 its source read (fixed dQ order: its additions done and the turn passed on),
+  // 10 fixed dQ order: the turn received)
   [[maybe_unused]] const bool tl = ATTN_TL_ON();
   ATTN_TL_T0(tl);
 
@@ -603,6 +604,7 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
           // J: the last tile whose first visited block, max(0, (128 J - diag) / 64), is <= qb
           const int J = CAUSAL ? min(p.n_kv_tiles - 1, (64 * qb + 63 + (p.S_k - p.S_q)) / 128) : p.n_kv_tiles - 1;
           if (!sem_wait_eq(sem, J - j, ctl)) break;
+          ATTN_TL(tl, 10, i);
           fence_proxy_async_global();
         }
         tma_reduce_add_4d(&tm_dqacc, sbase + L::DQ_STAGE_OFF + buf * L::DQ_STAGE_BYTES, 0, h, qb * L::BQ, b);

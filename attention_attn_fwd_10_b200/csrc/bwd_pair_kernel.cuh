@@ -134,6 +134,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
   const WaitCtl ctl{abort_flag, p.status, p.wait_limit_ns};
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // timeline build only (events per query block, as in the one-CTA pass: 0 S^T/dP^T
+  // issued, 1 S^T ready at the softmax, 2 dS^T published, 3 dS^T seen by the issuer,
+  // 4 dV/dK issued, 5 dQ^T issued, 6 dQ^T ready at the staging warps, 7 dQ tile
+  // staged, 8 reduce-add issued, 9 its source read (fixed order: done, turn passed on),
+  // 10 fixed order: turn received; and 11 dS^T half sent to the other CTA, 12 both
+  // CTAs' dS^T operands complete at the issuer; the issuer's events in rank 0 only)
+  [[maybe_unused]] const bool tl = ATTN_TL_ON();
+  ATTN_TL_T0(tl);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::N_BARS; ++i) {
@@ -292,6 +300,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
         if (ok) {
           tc_fence_after();
           issue_s_dp(0);
+          ATTN_TL(tl, 0, 0);
         }
       }
       for (int i = 0; ok && i < m; ++i) {
@@ -303,6 +312,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
           ok = false;
           break;
         }
+        ATTN_TL(tl, 3, i);
         tc_fence_after();
         if (i + 1 < m) {
           const uint32_t par = ((i + 1) / L::NST) & 1;
@@ -312,6 +322,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
           }
           tc_fence_after();
           issue_s_dp(st1);
+          ATTN_TL(tl, 0, i + 1);
         }
         // dV += P^T dO_i ; dK += dS^T Q_i  (16 queries per MMA: 8 TMEM columns, 2 KB of the column box)
         const uint32_t dob_lo = sdesc_lo(sb + L::ST_DOB, L::QBOX), qb_lo = sdesc_lo(sb + L::ST_QB, L::QBOX);
@@ -327,6 +338,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
         umma2_commit(pbar(L::B_PD_FREE));
         umma2_commit(bar(L::B_QDO_EMPTY + st));
         umma2_commit(pbar(L::B_QDO_EMPTY + st));
+        ATTN_TL(tl, 4, i);
         // dQ^T_i needs both CTAs' dS^T operands complete and dQ^T_{i-1} read out
         const uint32_t dpar = (i / L::NDS) & 1;
         if (!mbar_wait(bar(L::B_DS_IN + db), dpar, ctl) || !mbar_wait(bar(L::B_DS_PEER + db), dpar, ctl) ||
@@ -334,6 +346,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
           ok = false;
           break;
         }
+        ATTN_TL(tl, 12, i);
         if (i + L::NDS < m) mbar_arrive_expect_tx(bar(L::B_DS_IN + db), L::HALF_DS);
         tc_fence_after();
         // dQ_i^T = K^T dS_i^T over the pair's 256 keys: 16 keys per MMA = 2 KB of K^T, 1 KB of dS^T
@@ -343,6 +356,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
           umma2_ss_h(tmem + L::DQ_COL, kt_lo + kk * 128, HI, ds_lo + kk * 64, HI64, IDESC_Q, kk > 0 ? 1u : 0u);
         umma2_commit(bar(L::B_DQ_FULL));
         umma2_commit(pbar(L::B_DQ_FULL));
+        ATTN_TL(tl, 5, i);
       }
       if (ok) {
         umma2_commit(bar(L::B_D_FINAL));
@@ -371,6 +385,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
       const int st = i % L::NST;
       const int q0 = (qb0 + i % per_head) * L::BQ;
       ok = mbar_wait(bar(L::B_S_FULL), i & 1, ctl);
+      if (threadIdx.x == 0) ATTN_TL(tl, 1, i);
       if (ok) ok = mbar_wait(bar(L::B_QDO_FULL + st), (i / L::NST) & 1, ctl);  // -lse2, delta
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
@@ -439,6 +454,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive_cl_warp(ds_ready);
+      if (threadIdx.x == 0) ATTN_TL(tl, 2, i);
     }
     // ---- epilogue: dV, dK (scaled) -> bf16; this thread writes head dims [64 hc, 64 hc + 64)
     if (ok && m > 0) {
@@ -478,13 +494,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
   } else if (warp < 12) {
     // ===================== dQ staging: thread = (head dim, query half) =====================
     // TMEM lane l = 32 (warp % 4) + lane: head dim 64 rank + (l % 64), queries 32 (l / 64) + [0, 32)
-    const int tl = (warp & 3) * 32 + lane;
-    const int dl = tl & 63;
-    const int qh = tl >> 6;
+    const int tml = (warp & 3) * 32 + lane;
+    const int dl = tml & 63;
+    const int qh = tml >> 6;
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t dq_free = lbar(L::B_DQ_FREE);
     for (int i = 0; i < m; ++i) {
       bool ok = mbar_wait(bar(L::B_DQ_FULL), i & 1, ctl);
+      if (threadIdx.x == 256) ATTN_TL(tl, 6, i);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       uint32_t v[32];
@@ -502,6 +519,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
       for (int c = 0; c < 32; ++c) stage[(qh * 32 + c) * 64 + dl] = __uint_as_float(v[c]);
       fence_proxy_async_smem();
       mbar_arrive_warp(bar(L::B_STAGED + buf));
+      if (threadIdx.x == 256) ATTN_TL(tl, 7, i);
     }
   } else if (warp == L::WARP_RED) {
     // ===================== dQ reduce issue: one 64 x 64 TMA reduce-add per block =====================
@@ -518,11 +536,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
         if (DET) {
           const int Jt = CAUSAL ? min(p.n_kv_tiles - 1, (64 * qb + 63 + (p.S_k - p.S_q)) / 128) : p.n_kv_tiles - 1;
           if (!sem_wait_ge(sem, 2 * (Jt / 2 - pj), ctl)) break;
+          ATTN_TL(tl, 10, i);
           fence_proxy_async_global();
         }
         tma_reduce_add_4d(&tm_dqacc, sbase + L::DQ_STAGE_OFF + buf * L::DQ_STAGE_BYTES, static_cast<int>(rank) * 64,
                           h, qb * L::BQ, b);
         bulk_commit_group();
+        ATTN_TL(tl, 8, i);
         if (DET) {
           bulk_wait_all();
           fence_proxy_async_global();
@@ -531,6 +551,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
         } else {
           bulk_wait_read_all();
         }
+        ATTN_TL(tl, 9, i);
         mbar_arrive(bar(L::B_STAGE_FREE + buf));
       }
       bulk_wait_all();
@@ -547,6 +568,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
         bulk_copy_to_peer(mapa_shared(sbase + L::DS_OFF + db * L::DS_BYTES + static_cast<int>(rank) * L::HALF_DS, peer),
                           sbase + L::DSX_OFF + x * L::HALF_DS, L::HALF_DS, pbar(L::B_DS_IN + db));
         bulk_commit_group();
+        ATTN_TL(tl, 11, i);
         bulk_wait_read_all();
         mbar_arrive(bar(L::B_DSX_FREE + x));
         if (rank == 1) {  // tell rank 0 that rank 1's operand is complete for block i

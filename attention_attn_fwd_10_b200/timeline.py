@@ -1,12 +1,14 @@
 """Per-block clock64 timeline of one CTA, from the timeline build of the library.
 
     python -m attention_attn_fwd_10_b200.timeline fwd [--cta 0 300] [--S 8192]
-    python -m attention_attn_fwd_10_b200.timeline bwd [--cta 0 40]
+    python -m attention_attn_fwd_10_b200.timeline bwd [--cta 0 40] [--deterministic]
+    python -m attention_attn_fwd_10_b200.timeline bwd_pairs [--cta 0 40] [--deterministic]
     python -m attention_attn_fwd_10_b200.timeline decode [--cta 0] [--S 32768]
 
 Builds libattn_timeline.so if needed (the same sources with -DATTN_TIMELINE), loads
 it instead of libattn.so, runs on N(0, 1) inputs the causal B2 H16 S D128 forward (one
-CTA per work unit), the backward main pass, or (`decode`) the split-KV forward of one
+CTA per work unit), the backward main pass (one CTA per key tile, or `bwd_pairs`: CTA
+pairs, whose even CTA holds the MMA issuer), or (`decode`) the split-KV forward of one
 query row per head of B1 H32/8 against S keys, and prints, for each selected CTA,
 the first and last blocks' event times (SM clocks from the CTA's start) and the
 median of each step between events over the steady-state blocks.  The events are
@@ -35,12 +37,17 @@ FWD_STEPS = [("S_A ready -> row max done", 0, 2, 0), ("row max done -> P_A publi
              ("V load issued -> V ready at the issuer", 15, 10, 0),
              ("period: S_A(j) ready -> S_A(j+1) ready", 0, 0, 1)]
 BWD_NAMES = {0: "S/dP iss", 1: "S ready", 2: "dS pub", 3: "dS seen", 4: "dV/dK iss", 5: "dQ iss",
-             6: "dQ ready", 7: "staged", 8: "red iss", 9: "red read"}
+             6: "dQ ready", 7: "staged", 8: "red iss", 9: "red done", 10: "turn"}
 BWD_STEPS = [("S^T/dP^T issued -> S^T ready at the softmax", 0, 1, 0), ("S^T ready -> dS^T published", 1, 2, 0),
              ("dS^T published -> seen by the issuer", 2, 3, 0), ("dS^T seen -> dV/dK issued", 3, 4, 0),
              ("dV/dK issued -> dQ^T issued", 4, 5, 0), ("dQ^T issued -> ready at staging", 5, 6, 0),
              ("dQ^T ready -> tile staged", 6, 7, 0), ("staged -> reduce-add issued", 7, 8, 0),
-             ("reduce-add issued -> source read", 8, 9, 0), ("period: S^T ready(i) -> S^T ready(i+1)", 1, 1, 1)]
+             ("reduce-add issued -> source read (fixed order: done)", 8, 9, 0),
+             ("staged -> turn received (fixed order)", 7, 10, 0),
+             ("period: S^T ready(i) -> S^T ready(i+1)", 1, 1, 1)]
+PAIR_NAMES = {**BWD_NAMES, 11: "dS sent", 12: "dS both"}
+PAIR_STEPS = BWD_STEPS[:2] + [("dS^T published -> half sent to the other CTA", 2, 11, 0),
+                              ("dS^T published -> both CTAs' operands complete", 2, 12, 0)] + BWD_STEPS[2:]
 
 
 def _load_timeline_lib() -> ctypes.CDLL:
@@ -76,11 +83,12 @@ def _report(ev: np.ndarray, t0: int, names: dict, steps: list, out=print) -> Non
 
 def main(argv=None) -> None:
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
-    ap.add_argument("pass_", choices=("fwd", "bwd", "decode"), metavar="fwd|bwd|decode")
+    ap.add_argument("pass_", choices=("fwd", "bwd", "bwd_pairs", "decode"), metavar="fwd|bwd|bwd_pairs|decode")
     ap.add_argument("--cta", type=int, nargs="+", default=None, help="CTA indices to record (blockIdx.x)")
     ap.add_argument("--B", type=int, default=2)
     ap.add_argument("--H", type=int, default=16)
     ap.add_argument("--S", type=int, default=8192)
+    ap.add_argument("--deterministic", action="store_true", help="bwd: the fixed-order dQ instance")
     args = ap.parse_args(argv)
 
     lib = _load_timeline_lib()
@@ -109,10 +117,12 @@ def main(argv=None) -> None:
     if args.pass_ == "fwd":
         run = lambda: attn_fwd(q, k, v, causal=True, scale=scale, out=o, lse=lse, persistent=False)  # noqa: E731
         names, steps = FWD_NAMES, FWD_STEPS
-    elif args.pass_ == "bwd":
+    elif args.pass_ in ("bwd", "bwd_pairs"):
         do = torch.randn(B, S, H, D, device=dev).to(torch.bfloat16)
-        run = lambda: attn_bwd(q, k, v, o, lse, do, causal=True, scale=scale, cta_mode=1)  # noqa: E731
-        names, steps = BWD_NAMES, BWD_STEPS
+        mode = 1 if args.pass_ == "bwd" else 2
+        run = lambda: attn_bwd(q, k, v, o, lse, do, causal=True, scale=scale, cta_mode=mode,  # noqa: E731
+                               deterministic=args.deterministic)
+        names, steps = (BWD_NAMES, BWD_STEPS) if mode == 1 else (PAIR_NAMES, PAIR_STEPS)
     for cta in ctas:
         _read(lib, cta)
         for _ in range(3):  # warm-up calls, recorded and discarded

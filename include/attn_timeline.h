@@ -15,7 +15,12 @@
  * backward main pass (one CTA per key tile) records, per query block:
  * 0 S^T/dP^T issued, 1 S^T ready at the softmax, 2 dS^T published, 3 dS^T seen by
  * the issuer, 4 dV/dK issued, 5 dQ^T issued, 6 dQ^T ready at the staging warps,
- * 7 the dQ tile staged, 8 its reduce-add issued, 9 its source read.  Events that
+ * 7 the dQ tile staged, 8 its reduce-add issued, 9 its source read (in the fixed
+ * dQ order: its additions performed and the turn passed on), 10 (fixed dQ order)
+ * the turn received, before the reduce-add is issued.  The pair backward records
+ * the same events (the issuer's in the even CTA of a pair only) and 11 its dS^T
+ * half sent to the other CTA, 12 both CTAs' dS^T operands complete at the issuer.
+ * Events that
  * did not happen read 0.  The recording changes no result of any kernel.
  */
 #ifndef ATTN_TIMELINE_H
