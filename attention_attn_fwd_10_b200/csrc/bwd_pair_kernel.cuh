@@ -139,7 +139,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
   // 4 dV/dK issued, 5 dQ^T issued, 6 dQ^T ready at the staging warps, 7 dQ tile
   // staged, 8 reduce-add issued, 9 its source read (fixed order: done, turn passed on),
   // 10 fixed order: turn received; and 11 dS^T half sent to the other CTA, 12 both
-  // CTAs' dS^T operands complete at the issuer; the issuer's events in rank 0 only)
+  // CTAs' dS^T operands complete at the issuer, 13 (rank 1) the other CTA's half
+  // landed; the issuer's events in rank 0 only)
   [[maybe_unused]] const bool tl = ATTN_TL_ON();
   ATTN_TL_T0(tl);
 
@@ -573,6 +574,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
         mbar_arrive(bar(L::B_DSX_FREE + x));
         if (rank == 1) {  // tell rank 0 that rank 1's operand is complete for block i
           if (!mbar_wait(bar(L::B_DS_IN + db), (i / L::NDS) & 1, ctl)) break;
+          ATTN_TL(tl, 13, i);
           if (i + L::NDS < m) mbar_arrive_expect_tx(bar(L::B_DS_IN + db), L::HALF_DS);
           mbar_arrive_cl(lbar(L::B_DS_PEER + db));
         }
