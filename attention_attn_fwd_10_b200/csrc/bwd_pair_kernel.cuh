@@ -138,9 +138,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BwdPairLayout<DET>::
   // issued, 1 S^T ready at the softmax, 2 dS^T published, 3 dS^T seen by the issuer,
   // 4 dV/dK issued, 5 dQ^T issued, 6 dQ^T ready at the staging warps, 7 dQ tile
   // staged, 8 reduce-add issued, 9 its source read (fixed order: done, turn passed on),
-  // 10 fixed order: turn received; and 11 dS^T half sent to the other CTA, 12 both
-  // CTAs' dS^T operands complete at the issuer, 13 (rank 1) the other CTA's half
-  // landed; the issuer's events in rank 0 only)
+  // 10 fixed order: turn received; and 11 dS^T half sent to the other CTA, 12 the
+  // issuer has both CTAs' dS^T halves and the previous dQ^T read out, 13 (rank 1)
+  // the other CTA's half landed; the issuer's events in rank 0 only)
   [[maybe_unused]] const bool tl = ATTN_TL_ON();
   ATTN_TL_T0(tl);
 

@@ -47,7 +47,7 @@ BWD_STEPS = [("S^T/dP^T issued -> S^T ready at the softmax", 0, 1, 0), ("S^T rea
              ("period: S^T ready(i) -> S^T ready(i+1)", 1, 1, 1)]
 PAIR_NAMES = {**BWD_NAMES, 11: "dS sent", 12: "dS both", 13: "peer half"}
 PAIR_STEPS = BWD_STEPS[:2] + [("dS^T published -> half sent to the other CTA", 2, 11, 0),
-                              ("dS^T published -> both CTAs' operands complete", 2, 12, 0),
+                              ("dS^T published -> dQ^T inputs ready at the issuer", 2, 12, 0),
                               ("S^T ready -> dS^T half sent", 1, 11, 0),
                               ("S^T ready -> the other CTA's half landed (odd CTA)", 1, 13, 0)] + BWD_STEPS[2:]
 

@@ -19,8 +19,8 @@
  * dQ order: its additions performed and the turn passed on), 10 (fixed dQ order)
  * the turn received, before the reduce-add is issued.  The pair backward records
  * the same events (the issuer's in the even CTA of a pair only) and 11 its dS^T
- * half sent to the other CTA, 12 both CTAs' dS^T operands complete at the issuer,
- * 13 (odd CTA) the even CTA's half landed.
+ * half sent to the other CTA, 12 the issuer holds both CTAs' dS^T halves and the
+ * previous dQ^T has been read out, 13 (odd CTA) the even CTA's half landed.
  * Events that
  * did not happen read 0.  The recording changes no result of any kernel.
  */
