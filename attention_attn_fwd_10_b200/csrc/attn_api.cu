@@ -214,8 +214,23 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   static CUcontext seen[kMaxDevices] = {};
   const cudaError_t attr_err = smem_opt_in(kern, L::SMEM_BYTES, seen);
   if (attr_err != cudaSuccess) return attr_err;
-  kern<<<grid, L::THREADS, L::SMEM_BYTES, st>>>(mq, mk, mv, p);
-  return cudaGetLastError();
+  if (p.unit_base < 0) {
+    kern<<<grid, L::THREADS, L::SMEM_BYTES, st>>>(mq, mk, mv, p);
+    return cudaGetLastError();
+  }
+  // the tail launch: a programmatic dependent of the grid before it, so its CTAs take
+  // the SMs that grid leaves as its last CTAs finish (it reads none of that grid's results)
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(L::THREADS);
+  cfg.dynamicSmemBytes = L::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, p);
 }
 
 template <int D, bool CAUSAL, bool QK8 = false, bool PV8 = false>
@@ -353,6 +368,7 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   // one tile holds every query row: tile B takes half of the key blocks instead of idling
   p.dual = S_q <= 128 / gp ? 1 : 0;
   p.persistent = (opt.persistent && !p.dual) ? 1 : 0;
+  p.unit_base = -1;
   if (n_splits > 1) {
     const size_t rows = static_cast<size_t>(n_splits) * B * H_q * S_q;
     p.o_part = static_cast<float*>(workspace);
@@ -365,21 +381,38 @@ attn_status_t run_fwd(const void* q, const void* k, const void* v, void* o, floa
   p.wait_limit_ns = g_wait_limit_ns.load();
   const long long grid_ll = static_cast<long long>(p.n_units) * B * (H_q / gp) * n_splits;
   if (grid_ll > 2147483647LL) return ATTN_ERR_UNSUPPORTED;  // one CTA per (unit, head pack, range)
-  const unsigned grid = static_cast<unsigned>(grid_ll);
+  // Last wave: equal-length (non-causal) units fill ceil(units / SMs) waves, the last
+  // one partly.  When it holds at most half as many units as there are SMs, those
+  // units go to a second launch as the dual stream (both tiles on one 128-row half,
+  // odd and even key blocks), two CTAs per unit, so they finish in about half a wave.
+  int tail = 0;
+  if (p.persistent && !causal && n_splits == 1 && gp == 1 && grid_ll > kNumSms) {
+    const int r = static_cast<int>(grid_ll % kNumSms);
+    if (r > 0 && r <= kNumSms / 2) tail = r;
+  }
+  const unsigned grid = static_cast<unsigned>(grid_ll - tail);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t err;
-  if (pv8)
-    err = causal ? launch_fwd_poly<128, true, true, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s)
-                 : launch_fwd_poly<128, false, true, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s);
-  else if (qk8)
-    err = causal ? launch_fwd_poly<128, true, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s)
-                 : launch_fwd_poly<128, false, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s);
-  else if (D == 128)
-    err = causal ? launch_fwd_poly<128, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s)
-                 : launch_fwd_poly<128, false>(opt.poly_exp_every, mq, mk, mv, p, grid, s);
-  else
-    err = causal ? launch_fwd_poly<64, true>(opt.poly_exp_every, mq, mk, mv, p, grid, s)
-                 : launch_fwd_poly<64, false>(opt.poly_exp_every, mq, mk, mv, p, grid, s);
+  auto launch = [&](const FwdParams& pl, unsigned g) {
+    if (pv8)
+      return causal ? launch_fwd_poly<128, true, true, true>(opt.poly_exp_every, mq, mk, mv, pl, g, s)
+                    : launch_fwd_poly<128, false, true, true>(opt.poly_exp_every, mq, mk, mv, pl, g, s);
+    if (qk8)
+      return causal ? launch_fwd_poly<128, true, true>(opt.poly_exp_every, mq, mk, mv, pl, g, s)
+                    : launch_fwd_poly<128, false, true>(opt.poly_exp_every, mq, mk, mv, pl, g, s);
+    if (D == 128)
+      return causal ? launch_fwd_poly<128, true>(opt.poly_exp_every, mq, mk, mv, pl, g, s)
+                    : launch_fwd_poly<128, false>(opt.poly_exp_every, mq, mk, mv, pl, g, s);
+    return causal ? launch_fwd_poly<64, true>(opt.poly_exp_every, mq, mk, mv, pl, g, s)
+                  : launch_fwd_poly<64, false>(opt.poly_exp_every, mq, mk, mv, pl, g, s);
+  };
+  cudaError_t err = launch(p, grid);
+  if (err == cudaSuccess && tail > 0) {
+    FwdParams pt = p;
+    pt.dual = 1;
+    pt.persistent = 0;
+    pt.unit_base = static_cast<int>(grid);
+    err = launch(pt, 2u * static_cast<unsigned>(tail));
+  }
   if (err != cudaSuccess) return ATTN_ERR_CUDA;
   if (n_splits > 1) {
     const long long rows = static_cast<long long>(B) * S_q * H_q;

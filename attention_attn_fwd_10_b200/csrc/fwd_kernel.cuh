@@ -70,6 +70,10 @@ struct FwdParams {
   // not started yet (cluster launch control) and processes it with the barriers,
   // rings and tensor memory it already holds.  Not with the dual stream.
   int persistent;
+  // Tail launch (>= 0): this grid runs, as the dual stream, the work units from item
+  // unit_base on of a grid launched just before it with the same parameters; its item
+  // n is the 128-row half n % 2 of that grid's item unit_base + n / 2.  -1 otherwise.
+  int unit_base;
   float scale_log2;  // scale * log2(e)
   float tau;         // rescale threshold (base-2 units); 0 = rescale on every increase
   int* status;       // device status word
@@ -232,9 +236,9 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
   [[maybe_unused]] const bool tl = ATTN_TL_ON();
   ATTN_TL_T0(tl);
   const int tile_pos = L::BM >> p.gp_log2;  // query positions per tile
-  // split ranges: the merge of the ranges may start launching now (it waits on the
-  // device for this grid's results)
-  if (p.n_splits > 1) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // A programmatic dependent may start launching now: the merge of split ranges (it
+  // waits on the device for this grid's results) or the tail launch (independent work).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int diag = p.S_k - p.S_q;           // bottom-right causal: key j visible to row i iff j <= i + diag
 
   // ---- work items.  Item n is the work of block n of a one-CTA-per-unit grid:
@@ -254,6 +258,11 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
   };
   auto decode = [&](int item) {
     Unit w;
+    int sub = 0;  // tail launch: which 128-row half of the 256-row unit
+    if (p.unit_base >= 0) {
+      sub = item & 1;
+      item = p.unit_base + (item >> 1);
+    }
     const int BH = p.B * (p.H_q >> p.gp_log2);  // (batch, head pack) pairs
     w.split = item % p.n_splits;
     const int cta = item / p.n_splits;
@@ -267,7 +276,7 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
     w.b = bh / (p.H_q >> p.gp_log2);
     w.h0 = (bh - w.b * (p.H_q >> p.gp_log2)) << p.gp_log2;  // first query head of the pack
     w.hkv = w.h0 / (p.H_q / p.H_kv);
-    w.q0 = u * 2 * tile_pos;  // first query position of the unit
+    w.q0 = (2 * u + sub) * tile_pos;  // first query position of the unit
     // Key block of tile t's step j: j0 + j (both tiles take the same blocks), or in the
     // dual stream j0 + 2j + t.
     w.j0 = w.split * p.split_blocks;

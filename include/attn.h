@@ -96,9 +96,14 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
  *                       for causal -- and runs it with the barriers, rings and
  *                       tensor memory it holds, loading the next unit's tiles
  *                       while it finishes the current one (a persistent tile
- *                       scheduler; Blackwell cluster launch control).  0 = one
- *                       CTA per unit.  Ignored when one tile holds every query
- *                       row (the two tiles then split the keys instead).
+ *                       scheduler; Blackwell cluster launch control).  With it,
+ *                       a non-causal forward whose units leave a last wave of at
+ *                       most half the SMs runs those units in a second launch,
+ *                       two CTAs per unit (each on 128 rows, its two tiles
+ *                       splitting the keys), started as the first launch's CTAs
+ *                       finish.  0 = one CTA per unit.  Ignored when one tile
+ *                       holds every query row (the two tiles then split the keys
+ *                       instead).
  */
 typedef struct {
   float rescale_threshold;
