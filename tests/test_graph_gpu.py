@@ -42,3 +42,29 @@ def test_fwd_bwd_step_in_a_cuda_graph():
     assert torch.equal(dk, ref[3]) and torch.equal(dv, ref[4])
     # dQ sums the key tiles' parts in completion order: equal up to fp32 reassociation
     assert (dq.float() - ref[2].float()).abs().max() <= 1e-2 * ref[2].float().abs().max()
+
+
+def test_fwd_with_split_last_wave_in_a_cuda_graph():
+    # a non-causal grid of 152 units on 148 SMs: its last 4 units run in the second,
+    # programmatically dependent launch; both launches are captured and replayed
+    import attention_attn_fwd_10_b200 as attn
+
+    w = workloads.small(B=1, H_q=38, H_kv=38, S_q=1024, S_k=1024, D=128, causal=False, seed=9)
+    x = workloads.make_inputs(w)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H_q, w.S_q), dtype=torch.float32, device="cuda")
+    attn.fwd(q, k, v, causal=False, scale=w.scale, out=o, lse=lse)
+    torch.cuda.synchronize()
+    ref = [o.clone(), lse.clone()]
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        attn.fwd(q, k, v, causal=False, scale=w.scale, out=o, lse=lse, stream=s)
+    o.zero_()
+    lse.zero_()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert attn.device_status() == 0
+    assert torch.equal(o, ref[0]) and torch.equal(lse, ref[1])
