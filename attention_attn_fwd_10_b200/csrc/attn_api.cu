@@ -597,6 +597,7 @@ attn_status_t attn_bwd_ex(const void* q, const void* k, const void* v, const voi
   // with the number of dQ adders), one CTA per tile otherwise -- the faster kernel of
   // each mode on B200
   const bool pairs = cta_mode == 2 || (cta_mode == 0 && det && D == 128);
+  p.persistent = det ? 0 : 1;  // the one-CTA-per-tile pass in the normal dQ order
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);

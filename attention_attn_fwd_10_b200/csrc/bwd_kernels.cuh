@@ -53,6 +53,10 @@ struct BwdParams {
   float* delta;             // [B, H_q, S_pad] (workspace)
   int* dq_sem;              // [B, H_q, S_pad / 64] dQ turn counters (workspace; deterministic mode)
   int* ticket;              // work-item counter of the deterministic main pass (workspace)
+  // Main pass, normal dQ order: persistent CTAs (after its key tile a CTA takes over
+  // the tile of a CTA that has not started, by cluster launch control, loading the new
+  // tile's K and V while it finishes the old one's epilogue).  0 = one CTA per tile.
+  int persistent;
   __nv_bfloat16* dq;        // [B, S_q, H_q, D]
   __nv_bfloat16* dk;        // [B, S_k, H_kv, D]
   __nv_bfloat16* dv;        // [B, S_k, H_kv, D]
@@ -175,11 +179,18 @@ struct BwdLayout {
   static constexpr int B_DRAIN = B_S_FULL + 6;
   static constexpr int B_STAGED = B_S_FULL + 7;   // [NDQ] 4 warp arrivals: dQ_i staged in tile i % NDQ
   static constexpr int B_STAGE_FREE = B_S_FULL + 7 + NDQ;  // [NDQ] the reduce of that tile has read it
-  static constexpr int N_BARS = B_S_FULL + 7 + 2 * NDQ;
-  static constexpr int TMEM_SLOT_OFF = BAR_OFF + 8 * N_BARS;
+  static constexpr int B_KV_EMPTY = B_S_FULL + 7 + 2 * NDQ;  // the tile's last MMAs have read K, V
+  static constexpr int B_D_EMPTY = B_KV_EMPTY + 1;  // 8 warp arrivals: the epilogue has read dV, dK
+  static constexpr int B_ITEM_FULL = B_KV_EMPTY + 2;  // [u % 2] the scheduler published tile u's item
+  static constexpr int B_ITEM_READ = B_KV_EMPTY + 4;  // every role read the current item (15 arrivals)
+  static constexpr int B_CLC = B_KV_EMPTY + 5;        // cluster launch control response written
+  static constexpr int N_BARS = B_KV_EMPTY + 6;
+  static constexpr int ITEM_READERS = 15;  // TMA, MMA, 8 softmax warps, 4 dQ staging warps, reduce
+  static constexpr int CLC_OFF = (BAR_OFF + 8 * N_BARS + 15) / 16 * 16;  // 16-byte response
+  static constexpr int ITEM_OFF = CLC_OFF + 16;                         // items of tiles u % 2
+  static constexpr int TMEM_SLOT_OFF = ITEM_OFF + 8;
   static constexpr int ABORT_OFF = TMEM_SLOT_OFF + 4;
-  static constexpr int TICKET_OFF = ABORT_OFF + 4;
-  static constexpr int SMEM_USED = TICKET_OFF + 4;
+  static constexpr int SMEM_USED = ABORT_OFF + 4;
   static constexpr int SMEM_BYTES = (SMEM_USED + 1024) > 122880 ? (SMEM_USED + 1024) : 122880;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   // tensor memory columns (512): S^T 64 | dP^T 64 | P^T 32 | dS^T 32 | dV D | dK D | dQ^T 64
@@ -192,10 +203,10 @@ struct BwdLayout {
   static constexpr uint32_t DQ_COL = 192 + 2 * D;   // 64 columns
   static constexpr uint32_t TMEM_COLS = 512;
   // warps 0-7 softmax / dS (two warps per key row, 32 queries each), 8-11 dQ
-  // staging, 12 TMA, 13 TMEM + MMA, 14 dQ reduce issue, 15 idle; 128 registers
-  // per thread.
+  // staging, 12 TMA, 13 TMEM + MMA, 14 dQ reduce issue, 15 work scheduler; 128
+  // registers per thread.
   static constexpr int THREADS = 512;
-  static constexpr int WARP_TMA = 12, WARP_MMA = 13, WARP_RED = 14;
+  static constexpr int WARP_TMA = 12, WARP_MMA = 13, WARP_RED = 14, WARP_SCHED = 15;
 };
 
 template <int D, bool CAUSAL, bool DET>
@@ -222,20 +233,24 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
   [[maybe_unused]] const bool tl = ATTN_TL_ON();
   ATTN_TL_T0(tl);
 
-  // Work item: the block index, or in the deterministic instance a ticket taken
-  // from a global counter when the CTA starts.  Items are ordered so that the
-  // dQ additions an item waits for belong to items with smaller numbers; with
-  // tickets those items were claimed by CTAs that had already started, so every
-  // wait ends whatever order the hardware dispatches the blocks in.
-  if (DET && threadIdx.x == 0)
-    *reinterpret_cast<volatile int*>(sptr + L::TICKET_OFF) = atomicAdd(p.ticket, 1);
-
+  // Work items: key tiles.  The first is the block index, or in the deterministic
+  // instance a ticket taken from a global counter when the CTA starts.  Items are
+  // ordered so that the dQ additions an item waits for belong to items with smaller
+  // numbers; with tickets those items were claimed by CTAs that had already started,
+  // so every wait ends whatever order the hardware dispatches the blocks in.  With
+  // persistent CTAs (normal dQ order only), the scheduler warp then claims the item
+  // of a block that has not started (cluster launch control, the hardware's launch
+  // order) once every role has read the current one; -1 = no more work.
+  volatile int* item_slot = reinterpret_cast<volatile int*>(sptr + L::ITEM_OFF);
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::N_BARS; ++i)
-      mbar_init(bar(i), i == L::B_DS_READY ? 8u
-                        : (i == L::B_DQ_FREE || (i >= L::B_STAGED && i < L::B_STAGED + L::NDQ)) ? 4u : 1u);
+      mbar_init(bar(i), i == L::B_DS_READY || i == L::B_D_EMPTY ? 8u
+                        : (i == L::B_DQ_FREE || (i >= L::B_STAGED && i < L::B_STAGED + L::NDQ)) ? 4u
+                        : i == L::B_ITEM_READ ? static_cast<uint32_t>(L::ITEM_READERS) : 1u);
     *abort_flag = 0;
+    item_slot[0] = DET ? atomicAdd(p.ticket, 1) : static_cast<int>(blockIdx.x);
     fence_mbar_init();
+    mbar_arrive(bar(L::B_ITEM_FULL));
   }
   if (warp == L::WARP_MMA) {
     tmem_alloc(sbase + L::TMEM_SLOT_OFF, L::TMEM_COLS);
@@ -255,66 +270,113 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
   // ---- work decode: groups of bh_group (batch, kv head) pairs run together, so
   // the dQ accumulator rows and Q / dO tiles they share stay in L2; inside a
   // group, causal tiles with the most query blocks (low key index) come first
-  const int item = DET ? *reinterpret_cast<volatile int*>(sptr + L::TICKET_OFF) : static_cast<int>(blockIdx.x);
-  // A ticket beyond the grid would mean the counter was not reset before the
-  // launch: such a CTA touches nothing and records an error.
-  const bool live = item < static_cast<int>(gridDim.x);
-  if (!live && threadIdx.x == 0) atomicExch(p.status, kDevWaitTimeout);
-  const int BH = p.B * p.H_kv;
-  const int per_group = p.bh_group * p.n_kv_tiles;
-  const int grp = item / per_group;
-  const int within = item - grp * per_group;
-  const int gs = min(p.bh_group, BH - grp * p.bh_group);
-  // deterministic instance: highest key tile first (see the dQ reduce below)
-  const int j = DET ? p.n_kv_tiles - 1 - within / gs : within / gs;
-  const int bh = grp * p.bh_group + (within % gs);
-  const int b = bh / p.H_kv;
-  const int hkv = bh - b * p.H_kv;
+  struct Item {
+    bool live;  // a ticket beyond the grid (the counter was not reset) touches nothing
+    int b, hkv, j, k0, qb0, per_head, m;  // m: query blocks this tile visits
+  };
   const int G = p.H_q / p.H_kv;
-  const int k0 = j * L::BN;
   const int diag = p.S_k - p.S_q;  // key k visible to query q iff k <= q + diag
-  const int n_qb = p.S_pad / L::BQ;
-  int qb0 = 0;
-  if (CAUSAL) {
-    const int first_q = k0 - diag;  // first query that sees key k0
-    qb0 = first_q <= 0 ? 0 : min(n_qb, first_q / L::BQ);
-  }
-  const int per_head = n_qb - qb0;
-  const int m = live ? G * per_head : 0;  // query blocks this CTA visits
+  auto decode = [&](int item) {
+    Item w;
+    w.live = item < static_cast<int>(gridDim.x);
+    const int BH = p.B * p.H_kv;
+    const int per_group = p.bh_group * p.n_kv_tiles;
+    const int grp = item / per_group;
+    const int within = item - grp * per_group;
+    const int gs = min(p.bh_group, BH - grp * p.bh_group);
+    // deterministic instance: highest key tile first (see the dQ reduce below)
+    w.j = DET ? p.n_kv_tiles - 1 - within / gs : within / gs;
+    const int bh = grp * p.bh_group + (within % gs);
+    w.b = bh / p.H_kv;
+    w.hkv = bh - w.b * p.H_kv;
+    w.k0 = w.j * L::BN;
+    const int n_qb = p.S_pad / L::BQ;
+    w.qb0 = 0;
+    if (CAUSAL) {
+      const int first_q = w.k0 - diag;  // first query that sees key k0
+      w.qb0 = first_q <= 0 ? 0 : min(n_qb, first_q / L::BQ);
+    }
+    w.per_head = n_qb - w.qb0;
+    w.m = w.live ? G * w.per_head : 0;
+    return w;
+  };
+  // Tile u's item (-1 = no more work), or -2 once a wait was abandoned.
+  auto read_item = [&](int u) -> int {
+    if (!mbar_wait(bar(L::B_ITEM_FULL + (u & 1)), (u >> 1) & 1, ctl)) return -2;
+    return item_slot[u & 1];
+  };
+  if (threadIdx.x == 0 && item_slot[0] >= static_cast<int>(gridDim.x)) atomicExch(p.status, kDevWaitTimeout);
 
-
-  if (warp == L::WARP_TMA) {
+  if (warp == L::WARP_SCHED) {
+    // ===================== work scheduler =====================
+    if (lane == 0) {
+      int item = item_slot[0];
+      uint32_t clc_phase = 0;
+      for (int u = 0;; ++u) {
+        if (!mbar_wait(bar(L::B_ITEM_READ), u & 1, ctl)) break;
+        int next = -1;
+        if (p.persistent && !DET && item >= 0) {
+          mbar_arrive_expect_tx(bar(L::B_CLC), 16);
+          clc_try_cancel(sbase + L::CLC_OFF, bar(L::B_CLC));
+          if (!mbar_wait(bar(L::B_CLC), clc_phase, ctl)) break;
+          clc_phase ^= 1;
+          next = clc_cancelled_block(sbase + L::CLC_OFF);
+        }
+        item_slot[(u + 1) & 1] = next;
+        mbar_arrive(bar(L::B_ITEM_FULL + ((u + 1) & 1)));
+        item = next;
+        if (next < 0) break;
+      }
+    }
+  } else if (warp == L::WARP_TMA) {
     // ===================== TMA producer =====================
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar(L::B_KV_FULL), 2 * L::KV_TILE);
-#pragma unroll
-      for (int x = 0; x < L::NBOX; ++x) {
-        tma_load_4d(sbase + L::K_OFF + x * L::KBOX_BYTES, &tm_k, bar(L::B_KV_FULL), x * 64, hkv, k0, b);
-        tma_load_4d(sbase + L::V_OFF + x * L::KBOX_BYTES, &tm_v, bar(L::B_KV_FULL), x * 64, hkv, k0, b);
-      }
-      int issued = 0;
-      for (int i = 0; i < m; ++i) {
-        const int st = i % L::NST;
-        if (i >= L::NST && !mbar_wait(bar(L::B_QDO_EMPTY + st), ((i / L::NST) - 1) & 1, ctl)) break;
-        const int h = hkv * G + i / per_head;
-        const int q0 = (qb0 + i % per_head) * L::BQ;
-        const uint32_t sb = sbase + L::STAGE_OFF + st * L::STAGE_BYTES;
-        const uint32_t fb = bar(L::B_QDO_FULL + st);
-        mbar_arrive_expect_tx(fb, 2 * L::Q_TILE + 512);
+      int g = 0;   // Q/dO blocks loaded (all tiles): ring stage g % NST
+      int nkv = 0; // K/V tiles loaded
+      bool ok = true;
+      for (int u = 0; ok; ++u) {
+        const int item = read_item(u);
+        if (item < 0) {
+          if (item == -1) mbar_arrive(bar(L::B_ITEM_READ));
+          break;
+        }
+        const Item w = decode(item);
+        if (w.m == 0) mbar_arrive(bar(L::B_ITEM_READ));
+        // the previous tile's last MMAs have read its K and V
+        if (nkv > 0 && !(ok = mbar_wait(bar(L::B_KV_EMPTY), (nkv - 1) & 1, ctl))) break;
+        mbar_arrive_expect_tx(bar(L::B_KV_FULL), 2 * L::KV_TILE);
 #pragma unroll
         for (int x = 0; x < L::NBOX; ++x) {
-          tma_load_4d(sb + L::ST_Q + x * L::QBOX_BYTES, &tm_q, fb, x * 64, h, q0, b);
-          tma_load_4d(sb + L::ST_DO + x * L::QBOX_BYTES, &tm_do, fb, x * 64, h, q0, b);
+          tma_load_4d(sbase + L::K_OFF + x * L::KBOX_BYTES, &tm_k, bar(L::B_KV_FULL), x * 64, w.hkv, w.k0, w.b);
+          tma_load_4d(sbase + L::V_OFF + x * L::KBOX_BYTES, &tm_v, bar(L::B_KV_FULL), x * 64, w.hkv, w.k0, w.b);
         }
-        const size_t r = (static_cast<size_t>(b) * p.H_q + h) * p.S_pad + q0;
-        bulk_load(sbase + L::LD_OFF + st * 512, p.nlse2 + r, 256, fb);
-        bulk_load(sbase + L::LD_OFF + st * 512 + 256, p.delta + r, 256, fb);
-        issued = i + 1;
+        ++nkv;
+        for (int i = 0; i < w.m; ++i, ++g) {
+          const int st = g % L::NST;
+          if (g >= L::NST && !(ok = mbar_wait(bar(L::B_QDO_EMPTY + st), ((g / L::NST) - 1) & 1, ctl))) break;
+          const int h = w.hkv * G + i / w.per_head;
+          const int q0 = (w.qb0 + i % w.per_head) * L::BQ;
+          const uint32_t sb = sbase + L::STAGE_OFF + st * L::STAGE_BYTES;
+          const uint32_t fb = bar(L::B_QDO_FULL + st);
+          mbar_arrive_expect_tx(fb, 2 * L::Q_TILE + 512);
+#pragma unroll
+          for (int x = 0; x < L::NBOX; ++x) {
+            tma_load_4d(sb + L::ST_Q + x * L::QBOX_BYTES, &tm_q, fb, x * 64, h, q0, w.b);
+            tma_load_4d(sb + L::ST_DO + x * L::QBOX_BYTES, &tm_do, fb, x * 64, h, q0, w.b);
+          }
+          const size_t r = (static_cast<size_t>(w.b) * p.H_q + h) * p.S_pad + q0;
+          bulk_load(sbase + L::LD_OFF + st * 512, p.nlse2 + r, 256, fb);
+          bulk_load(sbase + L::LD_OFF + st * 512 + 256, p.delta + r, 256, fb);
+          // the next tile is claimed when this one's last loads are issued, so a CTA
+          // does not hold on to pending work while it still has much of its own
+          if (i == w.m - 1) mbar_arrive(bar(L::B_ITEM_READ));
+        }
       }
-      mbar_wait_drain(bar(L::B_KV_FULL), 0, 1000000000ull);
-      for (int st = 0; st < L::NST && st < issued; ++st) {
-        const int uses = (issued - 1 - st) / L::NST + 1;
-        mbar_wait_drain(bar(L::B_QDO_FULL + st), (uses - 1) & 1, 1000000000ull);
+      // Drain: every load this thread issued has landed before the CTA may exit.
+      if (nkv > 0) mbar_wait_drain(bar(L::B_KV_FULL), (nkv - 1) & 1, 1000000000ull);
+      for (int i = 0; i < L::NST && i < g; ++i) {
+        const int n = g - 1 - i;
+        mbar_wait_drain(bar(L::B_QDO_FULL + n % L::NST), (n / L::NST) & 1, 1000000000ull);
       }
     }
   } else if (warp == L::WARP_MMA) {
@@ -346,57 +408,67 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
         }
         umma_commit(bar(L::B_S_FULL));
       };
-      bool ok = mbar_wait(bar(L::B_KV_FULL), 0, ctl);
-      if (ok && m > 0) {
-        ok = mbar_wait(bar(L::B_QDO_FULL), 0, ctl);
-        if (ok) {
+      int g = 0;  // query blocks processed (all tiles): the per-block barriers' phases
+      bool ok = true;
+      for (int u = 0; ok; ++u) {
+        const int item = read_item(u);
+        if (item != -2) mbar_arrive(bar(L::B_ITEM_READ));
+        if (item < 0) break;
+        const Item w = decode(item);
+        if (!(ok = mbar_wait(bar(L::B_KV_FULL), u & 1, ctl))) break;
+        if (w.m > 0) {
+          if (!(ok = mbar_wait(bar(L::B_QDO_FULL + g % L::NST), (g / L::NST) & 1, ctl))) break;
           tc_fence_after();
-          issue_s_dp(0);
-          ATTN_TL(tl, 0, 0);
+          issue_s_dp(g % L::NST);
+          ATTN_TL(tl, 0, g);
         }
+        // dV, dK of the previous tile have been read out by its epilogue
+        if (u > 0 && !(ok = mbar_wait(bar(L::B_D_EMPTY), (u - 1) & 1, ctl))) break;
+        for (int i = 0; i < w.m; ++i, ++g) {
+          const int st = g % L::NST;        // Q/dO stage of block g
+          const int st1 = (g + 1) % L::NST;
+          const int db = g & 1;             // dS^T buffer of block g
+          const uint32_t sb = sbase + L::STAGE_OFF + st * L::STAGE_BYTES;
+          if (!(ok = mbar_wait(bar(L::B_DS_READY), g & 1, ctl))) break;
+          ATTN_TL(tl, 3, g);
+          tc_fence_after();
+          // the next block's S^T, dP^T first: the softmax warpgroup starts on them while
+          // the tensor pipe runs dV_i, dK_i, dQ^T_i
+          if (i + 1 < w.m) {
+            if (!(ok = mbar_wait(bar(L::B_QDO_FULL + st1), ((g + 1) / L::NST) & 1, ctl))) break;
+            tc_fence_after();
+            issue_s_dp(st1);
+            ATTN_TL(tl, 0, g + 1);
+          }
+          // dV += P^T dO_i ; dK += dS^T Q_i   (16 queries per MMA: 8 TMEM columns, 2048 B of the stage)
+#pragma unroll
+          for (int kk = 0; kk < L::BQ / 16; ++kk)
+            umma_ts_h(tmem + L::DV_COL, tmem + L::P_COL + kk * 8, sdesc_lo(sb + L::ST_DO, L::QBOX_BYTES) + kk * 128,
+                      HI, IDESC_G, (i > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < L::BQ / 16; ++kk)
+            umma_ts_h(tmem + L::DK_COL, tmem + L::DS_COL + kk * 8, sdesc_lo(sb + L::ST_Q, L::QBOX_BYTES) + kk * 128,
+                      HI, IDESC_G, (i > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(bar(L::B_PD_FREE));
+          umma_commit(bar(L::B_QDO_EMPTY + st));
+          ATTN_TL(tl, 4, g);
+          if (g >= 1) {
+            if (!(ok = mbar_wait(bar(L::B_DQ_FREE), (g - 1) & 1, ctl))) break;
+            tc_fence_after();
+          }
+          // dQ_i^T = K_j^T dS_i^T : 16 keys per MMA = 2048 B of K_j and of dS^T
+          const uint32_t ds = sbase + L::DS_OFF + db * L::DS_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < L::BN / 16; ++kk)
+            umma_ss_h(tmem + L::DQ_COL, kT_lo + kk * 128, HI, sdesc_lo(ds, L::DS_BYTES) + kk * 128, HI, IDESC_Q,
+                      kk > 0 ? 1u : 0u);
+          umma_commit(bar(L::B_DQ_FULL));
+          ATTN_TL(tl, 5, g);
+        }
+        if (!ok) break;
+        umma_commit(bar(L::B_D_FINAL));   // dV, dK of this tile complete
+        umma_commit(bar(L::B_KV_EMPTY));  // its K, V read by every MMA
       }
-      for (int i = 0; ok && i < m; ++i) {
-        const int st = i % L::NST;        // Q/dO stage of block i
-        const int st1 = (i + 1) % L::NST;
-        const int db = i & 1;             // dS^T buffer of block i
-        const uint32_t sb = sbase + L::STAGE_OFF + st * L::STAGE_BYTES;
-        if (!mbar_wait(bar(L::B_DS_READY), i & 1, ctl)) break;
-        ATTN_TL(tl, 3, i);
-        tc_fence_after();
-        // the next block's S^T, dP^T first: the softmax warpgroup starts on them while
-        // the tensor pipe runs dV_i, dK_i, dQ^T_i
-        if (i + 1 < m) {
-          if (!mbar_wait(bar(L::B_QDO_FULL + st1), ((i + 1) / L::NST) & 1, ctl)) break;
-          tc_fence_after();
-          issue_s_dp(st1);
-          ATTN_TL(tl, 0, i + 1);
-        }
-        // dV += P^T dO_i ; dK += dS^T Q_i   (16 queries per MMA: 8 TMEM columns, 2048 B of the stage)
-#pragma unroll
-        for (int kk = 0; kk < L::BQ / 16; ++kk)
-          umma_ts_h(tmem + L::DV_COL, tmem + L::P_COL + kk * 8, sdesc_lo(sb + L::ST_DO, L::QBOX_BYTES) + kk * 128,
-                    HI, IDESC_G, (i > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < L::BQ / 16; ++kk)
-          umma_ts_h(tmem + L::DK_COL, tmem + L::DS_COL + kk * 8, sdesc_lo(sb + L::ST_Q, L::QBOX_BYTES) + kk * 128,
-                    HI, IDESC_G, (i > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(bar(L::B_PD_FREE));
-        umma_commit(bar(L::B_QDO_EMPTY + st));
-        ATTN_TL(tl, 4, i);
-        if (i >= 1) {
-          if (!mbar_wait(bar(L::B_DQ_FREE), (i - 1) & 1, ctl)) break;
-          tc_fence_after();
-        }
-        // dQ_i^T = K_j^T dS_i^T : 16 keys per MMA = 2048 B of K_j and of dS^T
-        const uint32_t ds = sbase + L::DS_OFF + db * L::DS_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < L::BN / 16; ++kk)
-          umma_ss_h(tmem + L::DQ_COL, kT_lo + kk * 128, HI, sdesc_lo(ds, L::DS_BYTES) + kk * 128, HI, IDESC_Q,
-                    kk > 0 ? 1u : 0u);
-        umma_commit(bar(L::B_DQ_FULL));
-        ATTN_TL(tl, 5, i);
-      }
-      if (ok) umma_commit(bar(L::B_D_FINAL));
       umma_commit(bar(L::B_DRAIN));
       mbar_wait_drain(bar(L::B_DRAIN), 0, 1000000000ull);
     }
@@ -409,145 +481,154 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
     // with one 8-byte load per term and k (4 distinct addresses: one wavefront).
     const int r = threadIdx.x & 127;   // epilogue: key row == TMEM lane
     const int hc = threadIdx.x >> 7;   // query half: columns [32 hc, 32 hc + 32)
-    const int key = k0 + r;
-    const bool valid_key = live && key < p.S_k;
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int t0 = lane & 3, t1 = lane >> 2;
-    int row_key[4];  // [2 h + v]: the key of this thread's row (h, v)
-#pragma unroll
-    for (int hv = 0; hv < 4; ++hv) row_key[hv] = k0 + (warp & 3) * 32 + 16 * (hv >> 1) + t1 + 8 * (hv & 1);
     const uint64_t c2 = f2_pack(p.scale_log2, p.scale_log2);
+    int g = 0;  // query blocks processed (all tiles): the per-block barriers' phases
     bool ok = true;
-    for (int i = 0; i < m; ++i) {
-      const int st = i % L::NST;  // Q/dO stage (its -lse2, delta)
-      const int db = i & 1;       // dS^T buffer
-      const int q0 = (qb0 + i % per_head) * L::BQ;
-      // S_FULL(i) is committed after dQ^T_{i-2}, so dS^T buffer `db` is free as well.
-      ok = mbar_wait(bar(L::B_S_FULL), i & 1, ctl);
-      if (threadIdx.x == 0) ATTN_TL(tl, 1, i);
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sv[32], dp[32];  // [16 h + 4 k + 2 v + j]
-      tmem_ld16x256_x4(tmem + lane_addr + L::X_COL + 32 * hc, sv);
-      tmem_ld16x256_x4(tmem + lane_addr + (16u << 16) + L::X_COL + 32 * hc, sv + 16);
-      tmem_ld16x256_x4(tmem + lane_addr + L::Y_COL + 32 * hc, dp);
-      tmem_ld16x256_x4(tmem + lane_addr + (16u << 16) + L::Y_COL + 32 * hc, dp + 16);
-      const float2* nl2 = reinterpret_cast<const float2*>(sptr + L::LD_OFF + st * 512) + 16 * hc + t0;
-      const float2* dl2 = reinterpret_cast<const float2*>(sptr + L::LD_OFF + st * 512 + 256) + 16 * hc + t0;
-      float2 nlk[4], dlk[4];
+    for (int u = 0; ok; ++u) {
+      const int item = read_item(u);
+      if (item != -2) mbar_arrive_warp(bar(L::B_ITEM_READ));
+      if (item < 0) break;
+      const Item w = decode(item);
+      const int key = w.k0 + r;
+      const bool valid_key = w.live && key < p.S_k;
+      int row_key[4];  // [2 h + v]: the key of this thread's row (h, v)
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        nlk[k] = nl2[4 * k];
-        dlk[k] = dl2[4 * k];
-      }
-      tmem_ld_wait16(sv);
-      tmem_ld_wait16(sv + 16);
-      tmem_ld_wait16(dp);
-      tmem_ld_wait16(dp + 16);
-      // causal: key visible to query q0 + c iff c >= key - diag - q0; keys past S_k see nothing.
-      // c_first is relative to this thread's first query column 32 hc + 2 (lane % 4).
-      int c_first[4];
-      bool any_mask = false;
-#pragma unroll
-      for (int hv = 0; hv < 4; ++hv) {
-        const bool vk = live && row_key[hv] < p.S_k;
-        c_first[hv] = (!vk ? L::BQ : (CAUSAL ? row_key[hv] - diag - q0 : 0)) - 32 * hc - 2 * t0;
-        any_mask |= c_first[hv] > 0;
-      }
-      const bool masked = __any_sync(0xffffffffu, any_mask);
-      uint32_t pp[16], pd[16];  // [8 h + 2 k + v]: the bf16 pair (queries 2 j) of row (h, v)
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-#pragma unroll
-          for (int v = 0; v < 2; ++v) {
-            const int e = 16 * h + 4 * k + 2 * v;
-            const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2,
-                                       f2_pack(nlk[k].x, nlk[k].y));
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            float p0 = exp2_mufu(x0), p1 = exp2_mufu(x1);
-            if (masked) {
-              const int cf = c_first[2 * h + v];
-              if (8 * k < cf) p0 = 0.f;
-              if (8 * k + 1 < cf) p1 = 0.f;
-            }
-            const uint64_t g2 = f2_sub(f2_pack(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
-                                       f2_pack(dlk[k].x, dlk[k].y));
-            float d0, d1;
-            f2_unpack(f2_mul(f2_pack(p0, p1), g2), d0, d1);
-            pp[8 * h + 2 * k + v] = pack_bf16x2(p0, p1);
-            pd[8 * h + 2 * k + v] = pack_bf16x2(d0, d1);
-          }
-        }
-      }
-      // dS^T rows into the 128B-swizzled MN-major operand: the 4-byte pair of queries
-      // 32 hc + 8 k + 2 (lane % 4) sits in 16-byte chunk 4 hc + k of its row, and chunk c of
-      // row R at chunk c ^ (R % 8).  A warp's store covers 8 rows x 16 B: conflict-free.
-      uint8_t* dsb = sptr + L::DS_OFF + db * L::DS_BYTES;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int v = 0; v < 2; ++v) {
-          const int R = (warp & 3) * 32 + 16 * h + t1 + 8 * v;
-          uint8_t* row = dsb + R * 128 + 4 * t0;
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            *reinterpret_cast<uint32_t*>(row + (((4 * hc + k) ^ (R & 7)) << 4)) = pd[8 * h + 2 * k + v];
-        }
-      }
-      fence_proxy_async_smem();
-      if (i >= 1) {  // dV_{i-1}, dK_{i-1} have read the previous P^T, dS^T
-        ok = mbar_wait(bar(L::B_PD_FREE), (i - 1) & 1, ctl);
+      for (int hv = 0; hv < 4; ++hv) row_key[hv] = w.k0 + (warp & 3) * 32 + 16 * (hv >> 1) + t1 + 8 * (hv & 1);
+      for (int i = 0; i < w.m; ++i, ++g) {
+        const int st = g % L::NST;  // Q/dO stage (its -lse2, delta)
+        const int db = g & 1;       // dS^T buffer
+        const int q0 = (w.qb0 + i % w.per_head) * L::BQ;
+        // S_FULL(g) is committed after dQ^T_{g-2}, so dS^T buffer `db` is free as well.
+        ok = mbar_wait(bar(L::B_S_FULL), g & 1, ctl);
+        if (threadIdx.x == 0) ATTN_TL(tl, 1, g);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after();
-      }
-      // P^T, dS^T (bf16 pairs; column = query / 2) with shape 16x128b: packed column
-      // 16 hc + 4 k + lane % 4 of rows (h, v)
-      tmem_st16x128_x4(tmem + lane_addr + L::P_COL + 16 * hc, pp);
-      tmem_st16x128_x4(tmem + lane_addr + (16u << 16) + L::P_COL + 16 * hc, pp + 8);
-      tmem_st16x128_x4(tmem + lane_addr + L::DS_COL + 16 * hc, pd);
-      tmem_st16x128_x4(tmem + lane_addr + (16u << 16) + L::DS_COL + 16 * hc, pd + 8);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive_warp(bar(L::B_DS_READY));
-      if (threadIdx.x == 0) ATTN_TL(tl, 2, i);
-    }
-    // ---- epilogue: dV, dK (scaled) -> bf16; this thread writes head dims [D/2 hc, D/2 (hc + 1))
-    if (ok && m > 0) {
-      ok = mbar_wait(bar(L::B_D_FINAL), 0, ctl);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
-      tc_fence_after();
-      const size_t rowoff = ((static_cast<size_t>(b) * p.S_k + key) * p.H_kv + hkv) * D;
-#pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t col = which == 0 ? L::DV_COL : L::DK_COL;
-        const float sc = which == 0 ? 1.f : p.scale;
-        __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + rowoff;
-#pragma unroll 1
-        for (int ch = (D / 64) * hc; ch < (D / 64) * (hc + 1); ++ch) {
-          uint32_t v[32];
-          if (m > 0) {
-            tmem_ld32(tmem + lane_addr + col + ch * 32, v);
-            tmem_ld_wait(v);
-          } else {
+        uint32_t sv[32], dp[32];  // [16 h + 4 k + 2 v + j]
+        tmem_ld16x256_x4(tmem + lane_addr + L::X_COL + 32 * hc, sv);
+        tmem_ld16x256_x4(tmem + lane_addr + (16u << 16) + L::X_COL + 32 * hc, sv + 16);
+        tmem_ld16x256_x4(tmem + lane_addr + L::Y_COL + 32 * hc, dp);
+        tmem_ld16x256_x4(tmem + lane_addr + (16u << 16) + L::Y_COL + 32 * hc, dp + 16);
+        const float2* nl2 = reinterpret_cast<const float2*>(sptr + L::LD_OFF + st * 512) + 16 * hc + t0;
+        const float2* dl2 = reinterpret_cast<const float2*>(sptr + L::LD_OFF + st * 512 + 256) + 16 * hc + t0;
+        float2 nlk[4], dlk[4];
 #pragma unroll
-            for (int t = 0; t < 32; ++t) v[t] = 0u;
+        for (int k = 0; k < 4; ++k) {
+          nlk[k] = nl2[4 * k];
+          dlk[k] = dl2[4 * k];
+        }
+        tmem_ld_wait16(sv);
+        tmem_ld_wait16(sv + 16);
+        tmem_ld_wait16(dp);
+        tmem_ld_wait16(dp + 16);
+        // causal: key visible to query q0 + c iff c >= key - diag - q0; keys past S_k see nothing.
+        // c_first is relative to this thread's first query column 32 hc + 2 (lane % 4).
+        int c_first[4];
+        bool any_mask = false;
+#pragma unroll
+        for (int hv = 0; hv < 4; ++hv) {
+          const bool vk = w.live && row_key[hv] < p.S_k;
+          c_first[hv] = (!vk ? L::BQ : (CAUSAL ? row_key[hv] - diag - q0 : 0)) - 32 * hc - 2 * t0;
+          any_mask |= c_first[hv] > 0;
+        }
+        const bool masked = __any_sync(0xffffffffu, any_mask);
+        uint32_t pp[16], pd[16];  // [8 h + 2 k + v]: the bf16 pair (queries 2 j) of row (h, v)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+              const int e = 16 * h + 4 * k + 2 * v;
+              const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), c2,
+                                         f2_pack(nlk[k].x, nlk[k].y));
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              float p0 = exp2_mufu(x0), p1 = exp2_mufu(x1);
+              if (masked) {
+                const int cf = c_first[2 * h + v];
+                if (8 * k < cf) p0 = 0.f;
+                if (8 * k + 1 < cf) p1 = 0.f;
+              }
+              const uint64_t g2 = f2_sub(f2_pack(__uint_as_float(dp[e]), __uint_as_float(dp[e + 1])),
+                                         f2_pack(dlk[k].x, dlk[k].y));
+              float d0, d1;
+              f2_unpack(f2_mul(f2_pack(p0, p1), g2), d0, d1);
+              pp[8 * h + 2 * k + v] = pack_bf16x2(p0, p1);
+              pd[8 * h + 2 * k + v] = pack_bf16x2(d0, d1);
+            }
           }
-          uint32_t pk[16];
+        }
+        // dS^T rows into the 128B-swizzled MN-major operand: the 4-byte pair of queries
+        // 32 hc + 8 k + 2 (lane % 4) sits in 16-byte chunk 4 hc + k of its row, and chunk c of
+        // row R at chunk c ^ (R % 8).  A warp's store covers 8 rows x 16 B: conflict-free.
+        uint8_t* dsb = sptr + L::DS_OFF + db * L::DS_BYTES;
 #pragma unroll
-          for (int t = 0; t < 16; ++t)
-            pk[t] = pack_bf16x2(__uint_as_float(v[2 * t]) * sc, __uint_as_float(v[2 * t + 1]) * sc);
-          if (valid_key) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 32);
+        for (int h = 0; h < 2; ++h) {
 #pragma unroll
-            for (int t = 0; t < 4; ++t) d4[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+          for (int v = 0; v < 2; ++v) {
+            const int R = (warp & 3) * 32 + 16 * h + t1 + 8 * v;
+            uint8_t* row = dsb + R * 128 + 4 * t0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              *reinterpret_cast<uint32_t*>(row + (((4 * hc + k) ^ (R & 7)) << 4)) = pd[8 * h + 2 * k + v];
+          }
+        }
+        fence_proxy_async_smem();
+        if (g >= 1) {  // dV, dK of the previous block have read the previous P^T, dS^T
+          ok = mbar_wait(bar(L::B_PD_FREE), (g - 1) & 1, ctl);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+          tc_fence_after();
+        }
+        // P^T, dS^T (bf16 pairs; column = query / 2) with shape 16x128b: packed column
+        // 16 hc + 4 k + lane % 4 of rows (h, v)
+        tmem_st16x128_x4(tmem + lane_addr + L::P_COL + 16 * hc, pp);
+        tmem_st16x128_x4(tmem + lane_addr + (16u << 16) + L::P_COL + 16 * hc, pp + 8);
+        tmem_st16x128_x4(tmem + lane_addr + L::DS_COL + 16 * hc, pd);
+        tmem_st16x128_x4(tmem + lane_addr + (16u << 16) + L::DS_COL + 16 * hc, pd + 8);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive_warp(bar(L::B_DS_READY));
+        if (threadIdx.x == 0) ATTN_TL(tl, 2, g);
+      }
+      if (!ok) break;
+      // ---- epilogue: dV, dK (scaled) -> bf16; this thread writes head dims [D/2 hc, D/2 (hc + 1))
+      ok = mbar_wait(bar(L::B_D_FINAL), u & 1, ctl);
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        tc_fence_after();
+        const size_t rowoff = ((static_cast<size_t>(w.b) * p.S_k + key) * p.H_kv + w.hkv) * D;
+#pragma unroll 1
+        for (int which = 0; which < 2; ++which) {
+          const uint32_t col = which == 0 ? L::DV_COL : L::DK_COL;
+          const float sc = which == 0 ? 1.f : p.scale;
+          __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + rowoff;
+#pragma unroll 1
+          for (int ch = (D / 64) * hc; ch < (D / 64) * (hc + 1); ++ch) {
+            uint32_t v[32];
+            if (w.m > 0) {
+              tmem_ld32(tmem + lane_addr + col + ch * 32, v);
+              tmem_ld_wait(v);
+            } else {
+#pragma unroll
+              for (int t = 0; t < 32; ++t) v[t] = 0u;
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int t = 0; t < 16; ++t)
+              pk[t] = pack_bf16x2(__uint_as_float(v[2 * t]) * sc, __uint_as_float(v[2 * t + 1]) * sc);
+            if (valid_key) {
+              uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 32);
+#pragma unroll
+              for (int t = 0; t < 4; ++t) d4[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+            }
           }
         }
       }
+      // dV, dK read out: the next tile's first dV, dK MMAs may overwrite them
+      tc_fence_before();
+      mbar_arrive_warp(bar(L::B_D_EMPTY));
     }
   } else if (warp < 12) {
     // ===================== dQ reduction warpgroup: thread = head-dim index =====================
@@ -559,67 +640,83 @@ __global__ void __launch_bounds__(BwdLayout<D, DET>::THREADS, 1)
     const int wl = (warp & 3) * 32 + lane;  // this thread's TMEM lane
     const int d = D == 128 ? wl : ((lane < 16) ? (warp & 3) * 16 + lane : -1);
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    for (int i = 0; i < m; ++i) {
-      bool ok = mbar_wait(bar(L::B_DQ_FULL), i & 1, ctl);
-      if (wl == 0) ATTN_TL(tl, 6, i);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      uint32_t v[64];
-      tmem_ld32(tmem + lane_addr + L::DQ_COL, v);
-      tmem_ld32(tmem + lane_addr + L::DQ_COL + 32, v + 32);
-      tmem_ld_wait(v);
-      tmem_ld_wait(v + 32);
-      tc_fence_before();
-      mbar_arrive_warp(bar(L::B_DQ_FREE));
-      const int buf = i % L::NDQ;
-      if (i >= L::NDQ) {  // the reduce of block i - NDQ has read this tile
-        ok = mbar_wait(bar(L::B_STAGE_FREE + buf), ((i / L::NDQ) - 1) & 1, ctl);
-        if (!__all_sync(0xffffffffu, ok)) break;
-      }
-      float* stage = reinterpret_cast<float*>(sptr + L::DQ_STAGE_OFF + buf * L::DQ_STAGE_BYTES);
+    int g = 0;  // query blocks processed (all tiles)
+    bool ok = true;
+    for (int u = 0; ok; ++u) {
+      const int item = read_item(u);
+      if (item != -2) mbar_arrive_warp(bar(L::B_ITEM_READ));
+      if (item < 0) break;
+      const int m = decode(item).m;
+      for (int i = 0; i < m; ++i, ++g) {
+        ok = mbar_wait(bar(L::B_DQ_FULL), g & 1, ctl);
+        if (wl == 0) ATTN_TL(tl, 6, g);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t v[64];
+        tmem_ld32(tmem + lane_addr + L::DQ_COL, v);
+        tmem_ld32(tmem + lane_addr + L::DQ_COL + 32, v + 32);
+        tmem_ld_wait(v);
+        tmem_ld_wait(v + 32);
+        tc_fence_before();
+        mbar_arrive_warp(bar(L::B_DQ_FREE));
+        const int buf = g % L::NDQ;
+        if (g >= L::NDQ) {  // the reduce of block g - NDQ has read this tile
+          ok = mbar_wait(bar(L::B_STAGE_FREE + buf), ((g / L::NDQ) - 1) & 1, ctl);
+          if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        }
+        float* stage = reinterpret_cast<float*>(sptr + L::DQ_STAGE_OFF + buf * L::DQ_STAGE_BYTES);
 #pragma unroll
-      for (int c = 0; c < L::BQ; ++c)
-        if (d >= 0) stage[c * D + d] = __uint_as_float(v[c]);
-      fence_proxy_async_smem();
-      mbar_arrive_warp(bar(L::B_STAGED + buf));
-      if (wl == 0) ATTN_TL(tl, 7, i);
+        for (int c = 0; c < L::BQ; ++c)
+          if (d >= 0) stage[c * D + d] = __uint_as_float(v[c]);
+        fence_proxy_async_smem();
+        mbar_arrive_warp(bar(L::B_STAGED + buf));
+        if (wl == 0) ATTN_TL(tl, 7, g);
+      }
     }
   } else if (warp == L::WARP_RED) {
     // ===================== dQ reduce issue: one TMA reduce-add per staged tile =====================
     if (lane == 0) {
-      for (int i = 0; i < m; ++i) {
-        const int buf = i % L::NDQ;
-        if (!mbar_wait(bar(L::B_STAGED + buf), (i / L::NDQ) & 1, ctl)) break;
-        const int h = hkv * G + i / per_head;
-        const int qb = qb0 + i % per_head;
-        // Deterministic mode: the key tiles that see query block qb are 0..J (lower
-        // keys are visible to more queries).  They add their parts in the order J,
-        // J - 1, ..., 0 -- the order in which they reach the block, since tile j
-        // starts its sweep two blocks before tile j - 1 -- so tile j waits for
-        // J - j others.  High tiles have the smaller work-item numbers, so tile
-        // j + 1's item was claimed by a CTA that started before this one: it is
-        // running or done, and the wait always ends.
-        int* sem = p.dq_sem + (static_cast<size_t>(b) * p.H_q + h) * (p.S_pad / 64) + qb;
-        if (DET) {
-          // J: the last tile whose first visited block, max(0, (128 J - diag) / 64), is <= qb
-          const int J = CAUSAL ? min(p.n_kv_tiles - 1, (64 * qb + 63 + (p.S_k - p.S_q)) / 128) : p.n_kv_tiles - 1;
-          if (!sem_wait_eq(sem, J - j, ctl)) break;
-          ATTN_TL(tl, 10, i);
-          fence_proxy_async_global();
+      int g = 0;  // query blocks processed (all tiles)
+      bool ok = true;
+      for (int u = 0; ok; ++u) {
+        const int item = read_item(u);
+        if (item != -2) mbar_arrive(bar(L::B_ITEM_READ));
+        if (item < 0) break;
+        const Item w = decode(item);
+        for (int i = 0; i < w.m; ++i, ++g) {
+          const int buf = g % L::NDQ;
+          if (!(ok = mbar_wait(bar(L::B_STAGED + buf), (g / L::NDQ) & 1, ctl))) break;
+          const int h = w.hkv * G + i / w.per_head;
+          const int qb = w.qb0 + i % w.per_head;
+          // Deterministic mode: the key tiles that see query block qb are 0..J (lower
+          // keys are visible to more queries).  They add their parts in the order J,
+          // J - 1, ..., 0 -- the order in which they reach the block, since tile j
+          // starts its sweep two blocks before tile j - 1 -- so tile j waits for
+          // J - j others.  High tiles have the smaller work-item numbers, so tile
+          // j + 1's item was claimed by a CTA that started before this one: it is
+          // running or done, and the wait always ends.
+          int* sem = p.dq_sem + (static_cast<size_t>(w.b) * p.H_q + h) * (p.S_pad / 64) + qb;
+          if (DET) {
+            // J: the last tile whose first visited block, max(0, (128 J - diag) / 64), is <= qb
+            const int J = CAUSAL ? min(p.n_kv_tiles - 1, (64 * qb + 63 + (p.S_k - p.S_q)) / 128) : p.n_kv_tiles - 1;
+            if (!(ok = sem_wait_eq(sem, J - w.j, ctl))) break;
+            ATTN_TL(tl, 10, g);
+            fence_proxy_async_global();
+          }
+          tma_reduce_add_4d(&tm_dqacc, sbase + L::DQ_STAGE_OFF + buf * L::DQ_STAGE_BYTES, 0, h, qb * L::BQ, w.b);
+          bulk_commit_group();
+          ATTN_TL(tl, 8, g);
+          if (DET) {
+            bulk_wait_all();  // the additions are performed
+            fence_proxy_async_global();
+            __threadfence();
+            sem_release_add(sem);
+          } else {
+            bulk_wait_read_all();  // the tile has been read
+          }
+          ATTN_TL(tl, 9, g);
+          mbar_arrive(bar(L::B_STAGE_FREE + buf));
         }
-        tma_reduce_add_4d(&tm_dqacc, sbase + L::DQ_STAGE_OFF + buf * L::DQ_STAGE_BYTES, 0, h, qb * L::BQ, b);
-        bulk_commit_group();
-        ATTN_TL(tl, 8, i);
-        if (DET) {
-          bulk_wait_all();  // the additions are performed
-          fence_proxy_async_global();
-          __threadfence();
-          sem_release_add(sem);
-        } else {
-          bulk_wait_read_all();  // the tile has been read
-        }
-        ATTN_TL(tl, 9, i);
-        mbar_arrive(bar(L::B_STAGE_FREE + buf));
       }
       bulk_wait_all();
     }

@@ -242,7 +242,10 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
  *   cta_mode : how the main pass maps key tiles to CTAs.  0 (default) = the
  *       faster kernel of each mode on B200: CTA pairs for the deterministic
  *       instance at D = 128, one CTA per tile otherwise.  1 = one CTA per
- *       128-key tile (every MMA on one SM).  2 = CTA pairs (clusters of two CTAs on
+ *       128-key tile (every MMA on one SM); in the normal dQ order these CTAs
+ *       are persistent: a CTA that finishes its tile takes over the tile of a
+ *       CTA that has not started (cluster launch control) and loads its K and V
+ *       while it writes the old tile's dK and dV.  2 = CTA pairs (clusters of two CTAs on
  *       adjacent key tiles whose tensor cores execute each MMA together,
  *       cta_group::2: "AI Infra series ch. 6", section 7 item 3): half of each
  *       B operand per CTA and half the dQ reduce-adds, at the cost of a dS^T
