@@ -73,3 +73,17 @@ def test_split_kv_decode_shapes(S_q, S_k, H_q, H_kv, causal):
     o_ref, lse_ref = ref.forward(q8.float(), k8.float(), x["v"], causal, w.scale)
     parity.check_o(o, o_ref, w.name)
     parity.check_lse(lse, lse_ref, w.name)
+
+
+def test_last_wave_in_halves():
+    # 152 non-causal units on 148 SMs: the last 4 run in the second launch as the dual
+    # stream (with 8-bit Q/K its V ring keeps two stages); every row of the heads that
+    # hold them and of the first against the oracle
+    w = workloads.small(B=1, H_q=38, S_q=1024, S_k=1024, D=128, causal=False, seed=11)
+    q, k, x, o, lse = _run(w)
+    o_c, lse_c = o.cpu(), lse.cpu()
+    rows = list(range(w.S_q))
+    for h in (0, 34, 35, 36, 37):
+        o_ref, lse_ref = ref.forward_rows(q, k, x["v"], False, w.scale, 0, h, rows)
+        parity.check_o(o_c[0, rows, h, :], o_ref, f"{w.name} h={h}")
+        parity.check_lse(lse_c[0, h, rows], lse_ref, f"{w.name} h={h}")
