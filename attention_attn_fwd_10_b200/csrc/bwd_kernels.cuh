@@ -6,9 +6,14 @@
 //   2. attn_bwd_kernel             KV-stationary main pass (below)
 //   3. attn_bwd_convert_kernel     dQ = scale * dQ_acc -> bf16
 //
-// Main pass: one CTA owns one 128-key tile (K_j, V_j) of one (batch, kv head)
-// and visits every 64-query block (Q_i, dO_i) of every query head of the
-// group that sees it.  P is recomputed from lse rather than stored
+// Main pass: a CTA owns one 128-key tile (K_j, V_j) of one (batch, kv head) at
+// a time and visits every 64-query block (Q_i, dO_i) of every query head of the
+// group that sees it.  In the normal dQ order the CTA is persistent: a scheduler
+// warp claims the tile of a CTA that has not started (cluster launch control)
+// when the current tile's last loads are issued, and the new tile's K and V load
+// once the old tile's last MMAs have read theirs (KV_EMPTY), while the old tile's
+// dK and dV are written out; the new tile's first dV/dK MMA waits for that
+// epilogue to have read the accumulators (D_EMPTY).  P is recomputed from lse rather than stored
 // ("AI Infra series ch. 6, GPU performance engineering (II)", section 5,
 // recomputation).  Per query block, all on tcgen05 with fp32 accumulation:
 //   S^T  = K_j Q_i^T      (128 x 64, TMEM X)     dP^T = V_j dO_i^T   (TMEM Y)
@@ -37,7 +42,7 @@
 // (thread = head-dim row of dQ^T; at D = 64 dQ^T is an M = 64 accumulator whose
 // rows 16w..16w+15 sit in lanes 32w..32w+15, so half of each warp is idle);
 // warp 12 TMA producer; warp 13 TMEM allocator and MMA issuer; warp 14 issues
-// the dQ reduce-adds; warp 15 idle.  Head dims 64 and 128.
+// the dQ reduce-adds; warp 15 work scheduler.  Head dims 64 and 128.
 #pragma once
 
 #include "sm100_common.cuh"

@@ -10,7 +10,11 @@
 //   warp  8     TMA producer: Q_A, Q_B once, then K_j into a 3-stage ring
 //   warp  9     TMEM allocator and single-thread tcgen05.mma issuer
 //   warp  10    TMA producer: V_j into a 2-stage ring
-//   warp  11    idle (it completes the third warpgroup)
+//   warp  11    work scheduler: with persistent CTAs, claims the unit of a CTA
+//               that has not started (cluster launch control) for this one
+// A non-causal grid whose last wave would hold at most half as many units as there
+// are SMs leaves those units to a second launch of this kernel, two CTAs per unit,
+// each running the dual stream on 128 of its rows (FwdParams::unit_base).
 // K_j is released as soon as both tiles' S(j) have completed and V_j once both
 // PV(j) have, so the next loads start a full MMA group earlier than with a
 // shared K/V stage.
