@@ -662,11 +662,13 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
       float l = 0.f;
       unsigned rescales = 0;
       // The next unit is claimed once every role has read this one; the softmax
-      // warps count as having read it only when they start the unit's last block,
-      // so a CTA does not hold on to pending work while it still has much of its own.
+      // warps count as having read it only when they start the unit's 8th-last block:
+      // early enough for the next unit's Q and first K/V tiles to arrive before this
+      // unit ends, late enough that a CTA does not hold on to pending work while it
+      // still has much of its own.
       if (nb == 0) mbar_arrive_warp(bar(L::B_ITEM_READ));
       for (int j = 0; j < nb; ++j) {
-        if (j == nb - 1) mbar_arrive_warp(bar(L::B_ITEM_READ));
+        if (j == (nb > 8 ? nb - 8 : 0)) mbar_arrive_warp(bar(L::B_ITEM_READ));
         ok = mbar_wait(bar(L::B_S_FULL + t), (sc + j) & 1, ctl);
         if (row == 0) ATTN_TL(tl, 0 + t, sc + j);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
