@@ -133,6 +133,28 @@ def test_deterministic_and_overwrites_poison():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("D", [64, 128])
+def test_output_at_16_byte_offset(causal, D):
+    # O at a 16- but not 32-byte aligned address (the contract asks for 16): the result
+    # equals the one written to an aligned O, and matches the oracle
+    w = workloads.small(B=1, H_q=2, S_q=300, S_k=300, D=D, causal=causal, seed=31)
+    x = workloads.make_inputs(w)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    o_al, lse_al = _attn().fwd(q, k, v, causal=causal, scale=w.scale)
+    assert o_al.data_ptr() % 32 == 0
+    buf = torch.full((q.numel() + 8,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    o = buf[8:].view(q.shape)
+    assert o.data_ptr() % 32 == 16
+    lse = torch.full_like(lse_al, float("nan"))
+    _attn().fwd(q, k, v, causal=causal, scale=w.scale, out=o, lse=lse)
+    torch.cuda.synchronize()
+    assert _attn().device_status() == 0
+    assert torch.equal(o, o_al) and torch.equal(lse, lse_al)
+    o_ref, lse_ref = ref.forward(x["q"], x["k"], x["v"], causal, w.scale)
+    parity.check_o(o, o_ref, w.name)
+
+
 def test_host_buffers_round_trip():
     w = workloads.small(B=1, H_q=2, S_q=300, S_k=300, D=64, causal=False, seed=9)
     x = workloads.make_inputs(w)
