@@ -814,9 +814,20 @@ __global__ void __launch_bounds__(FwdLayout<D, QK8, PV8>::THREADS, 1)
               uint32_t pkd[8];
 #pragma unroll
               for (int i = 0; i < 8; ++i) pkd[i] = pack_bf16x2(ov[2 * i], ov[2 * i + 1]);
-              uint4* dst = reinterpret_cast<uint4*>(p.o + ((static_cast<size_t>(w.b) * p.S_q + qi) * p.H_q + h) * D + ch * 16);
-              dst[0] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
-              dst[1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
+              __nv_bfloat16* dst = p.o + ((static_cast<size_t>(w.b) * p.S_q + qi) * p.H_q + h) * D + ch * 16;
+              // Non-causal units are short enough that the epilogue is a visible share of
+              // them: one 256-bit store per chunk when O is 32-byte aligned (every row
+              // chunk then is).  The causal kernel keeps two 16-byte stores, which
+              // measured faster there.
+              bool wide = false;
+              if constexpr (!CAUSAL) wide = (reinterpret_cast<uintptr_t>(p.o) & 31u) == 0;
+              if (wide) {
+                st_global_v8(dst, pkd);
+              } else {
+                uint4* d4 = reinterpret_cast<uint4*>(dst);
+                d4[0] = make_uint4(pkd[0], pkd[1], pkd[2], pkd[3]);
+                d4[1] = make_uint4(pkd[4], pkd[5], pkd[6], pkd[7]);
+              }
             }
           }
           if (valid) {

@@ -136,8 +136,9 @@ def test_deterministic_and_overwrites_poison():
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("D", [64, 128])
 def test_output_at_16_byte_offset(causal, D):
-    # O at a 16- but not 32-byte aligned address (the contract asks for 16): the result
-    # equals the one written to an aligned O, and matches the oracle
+    # O at a 16- but not 32-byte aligned address (the contract asks for 16; the
+    # non-causal epilogue then writes with 16-byte stores instead of 256-bit ones): the
+    # result equals the one written to an aligned O, and matches the oracle
     w = workloads.small(B=1, H_q=2, S_q=300, S_k=300, D=D, causal=causal, seed=31)
     x = workloads.make_inputs(w)
     q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
